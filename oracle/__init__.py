@@ -1,0 +1,208 @@
+"""CPU oracle of the NVFP4 attention cache -- TEST INFRASTRUCTURE ONLY.
+
+The arithmetic lives in ``kvq_oracle.c`` (plain C: fp32 quantiser steps in a
+fixed order, fp64 attention).  This module compiles it with gcc, loads it with
+ctypes and marshals numpy arrays; it computes nothing itself.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` import this package.  The CUDA library (``bit_attention_decode_b200``)
+never imports it and it never imports the library.
+
+Parity status of each function (the pins live in ``tests/test_oracle_*.py``):
+  e2m1_encode / e2m1_value   pinned (grid golden file, exhaustive brute force)
+  e4m3_encode / e4m3_value   pinned (exhaustive brute force, torch float8 cast)
+  transform_keys             pinned (scipy Hadamard, H H^T = 128 I, invariance)
+  calibrate                  pinned (hand-built windows with known maxima)
+  quantize_rows              pinned (absmax/24 closed form, exact-scale blocks,
+                             error bound, brute-force per-block search)
+  dequantize_rows            pinned (products of the pinned format values)
+  attention                  pinned (numpy/scipy softmax formula, one token,
+                             equal keys, smoothing invariance)
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kvq_oracle.c")
+_LIB_DIR = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_LIB_DIR, "libkvq_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+HEAD_DIM = 128
+BLOCK = 16
+
+CFLAGS = ["-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+          "-fPIC", "-shared", "-lm"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/_build/libkvq_oracle.so``."""
+    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
+        return _LIB
+    os.makedirs(_LIB_DIR, exist_ok=True)
+    tmp = _LIB + f".tmp{os.getpid()}"
+    subprocess.run(["gcc", *CFLAGS, _SRC, "-o", tmp], check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i64, i32, f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_float
+        lib.oracle_e2m1_value.restype = ctypes.c_double
+        lib.oracle_e2m1_value.argtypes = [ctypes.c_uint32]
+        lib.oracle_e4m3_value.restype = ctypes.c_double
+        lib.oracle_e4m3_value.argtypes = [ctypes.c_uint32]
+        lib.oracle_e2m1_encode_n.argtypes = [P, P, i64]
+        lib.oracle_e4m3_encode_n.argtypes = [P, P, i64]
+        lib.oracle_transform_keys.argtypes = [P, P, i64, i32, i32, P]
+        lib.oracle_calibrate.argtypes = [P, P, i32, i32, i32, i32, i32, i32, P, P, P, P]
+        lib.oracle_quantize_rows.argtypes = [P, i64, f32, P, P]
+        lib.oracle_dequantize_rows.argtypes = [P, P, i64, f32, P]
+        lib.oracle_attention.argtypes = [P, i32, i32, i32, i32, P, i32, P, P, i32, P]
+        for name in ("oracle_e2m1_encode_n", "oracle_e4m3_encode_n", "oracle_transform_keys",
+                     "oracle_calibrate", "oracle_quantize_rows", "oracle_dequantize_rows",
+                     "oracle_attention"):
+            getattr(lib, name).restype = None
+        _lib = lib
+        return lib
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a, dtype=dtype)
+    return a, a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f32(x):
+    """Host fp32 copy of an array or tensor (bf16 widens exactly)."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return x.detach().to("cpu", torch.float32).contiguous().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+# ---------------------------------------------------------------- formats
+def e2m1_value(codes) -> np.ndarray:
+    lib = _load()
+    codes = np.asarray(codes, dtype=np.uint32)
+    table = np.array([lib.oracle_e2m1_value(c) for c in range(16)])
+    return table[codes & 15]
+
+
+def e4m3_value(codes) -> np.ndarray:
+    lib = _load()
+    codes = np.asarray(codes, dtype=np.uint32)
+    table = np.array([lib.oracle_e4m3_value(c) for c in range(256)])
+    return table[codes & 255]
+
+
+def e2m1_encode(x) -> np.ndarray:
+    x, px = _c(_f32(x), np.float32)
+    out = np.empty(x.shape, np.uint8)
+    _load().oracle_e2m1_encode_n(px, out.ctypes.data_as(ctypes.c_void_p), x.size)
+    return out
+
+
+def e4m3_encode(x) -> np.ndarray:
+    x, px = _c(_f32(x), np.float32)
+    out = np.empty(x.shape, np.uint8)
+    _load().oracle_e4m3_encode_n(px, out.ctypes.data_as(ctypes.c_void_p), x.size)
+    return out
+
+
+# ---------------------------------------------------------------- method steps
+def calibrate(k_calib, v_calib, exclude_pos0: bool = True, hadamard: bool = False):
+    """k/v_calib [L][W][T][H][D] -> (s, inv_s [L][H][D] fp32, g_K, g_V [L] fp32)."""
+    k, pk = _c(_f32(k_calib), np.float32)
+    v, pv = _c(_f32(v_calib), np.float32)
+    L, W, T, H, D = k.shape
+    assert D == HEAD_DIM and v.shape == k.shape
+    s = np.empty((L, H, D), np.float32)
+    inv = np.empty((L, H, D), np.float32)
+    gk = np.empty(L, np.float32)
+    gv = np.empty(L, np.float32)
+    P = ctypes.c_void_p
+    _load().oracle_calibrate(pk, pv, L, W, T, H, int(bool(exclude_pos0)), int(bool(hadamard)),
+                             s.ctypes.data_as(P), inv.ctypes.data_as(P),
+                             gk.ctypes.data_as(P), gv.ctypes.data_as(P))
+    return s, inv, gk, gv
+
+
+def transform_keys(k, inv_s, hadamard: bool = False) -> np.ndarray:
+    """k [n][H][D], inv_s [H][D] -> transformed keys [n][H][D] (fp32)."""
+    k, pk = _c(_f32(k), np.float32)
+    inv, pi = _c(_f32(inv_s), np.float32)
+    n, H, D = k.shape
+    y = np.empty_like(k)
+    _load().oracle_transform_keys(pk, pi, n, H, int(bool(hadamard)), y.ctypes.data_as(ctypes.c_void_p))
+    return y
+
+
+def quantize_rows(y, g: float):
+    """y [..., D] fp32 -> (codes [..., D] uint8 one code per byte, sf [..., D/16] uint8)."""
+    y, py = _c(_f32(y), np.float32)
+    n = y.size // HEAD_DIM
+    codes = np.empty(y.shape, np.uint8)
+    sf = np.empty(y.shape[:-1] + (HEAD_DIM // BLOCK,), np.uint8)
+    P = ctypes.c_void_p
+    _load().oracle_quantize_rows(py, n, float(g), codes.ctypes.data_as(P), sf.ctypes.data_as(P))
+    return codes, sf
+
+
+def dequantize_rows(codes, sf, g: float) -> np.ndarray:
+    codes, pc = _c(codes, np.uint8)
+    sf, ps = _c(sf, np.uint8)
+    x = np.empty(codes.shape, np.float64)
+    _load().oracle_dequantize_rows(pc, ps, codes.size // HEAD_DIM, float(g),
+                                   x.ctypes.data_as(ctypes.c_void_p))
+    return x
+
+
+def attention(q, q_start: int, s, kx, vx, hadamard: bool = False) -> np.ndarray:
+    """q [Tq][Hq][D]; s [Hkv][D]; kx, vx [T][Hkv][D] fp64 -> out [Tq][Hq][D] fp64."""
+    q, pq = _c(_f32(q), np.float32)
+    s, ps = _c(_f32(s), np.float32)
+    kx, pk = _c(kx, np.float64)
+    vx, pv = _c(vx, np.float64)
+    Tq, Hq, D = q.shape
+    T, Hkv, _ = kx.shape
+    out = np.empty((Tq, Hq, D), np.float64)
+    _load().oracle_attention(pq, Tq, int(q_start), Hq, Hkv, ps, int(bool(hadamard)), pk, pv, T,
+                             out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+# ---------------------------------------------------------------- composites
+def quantize_kv(k, v, inv_s, g_k: float, g_v: float, hadamard: bool = False):
+    """Quantise one layer's tokens: k, v [n][H][D] -> dict of codes and scales."""
+    y = transform_keys(k, inv_s, hadamard)
+    kc, ksf = quantize_rows(y, g_k)
+    vc, vsf = quantize_rows(_f32(v), g_v)
+    return {"kc": kc, "ksf": ksf, "vc": vc, "vsf": vsf}
+
+
+def decode_reference(q, k, v, s, inv_s, g_k, g_v, hadamard=False, q_start=None):
+    """Quantise a sequence's K/V, dequantise, and attend with q [Tq][Hq][D]."""
+    qz = quantize_kv(k, v, inv_s, g_k, g_v, hadamard)
+    kx = dequantize_rows(qz["kc"], qz["ksf"], g_k)
+    vx = dequantize_rows(qz["vc"], qz["vsf"], g_v)
+    T = kx.shape[0]
+    if q_start is None:
+        q_start = T - 1
+    return attention(q, q_start, s, kx, vx, hadamard), qz
