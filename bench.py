@@ -1,0 +1,394 @@
+#!/usr/bin/env python
+"""Throughput of the NVFP4 attention-cache hot path on B200; prints one JSON line.
+
+Default workload (N=1): ragged decode -- 36 layers, 32 query / 8 KV heads,
+head_dim 128, batch 64 with lengths uniform on [1024, 8192], a paged NVFP4
+cache of 16-token pages in shuffled order.  One step = append one new token
+per sequence into every layer (kvq_quantize_append) + one decode of every
+layer (kvq_decode_attention).  The 64 steps of the workload are cycled.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
+
+With N > 1 (torchrun) every rank runs its own replica of the workload (the
+path has no exchange step: independent sequences); the reported value is the
+sum over ranks, timed as the max over ranks.  ``--impl reference`` times the
+CPU oracle on bounded samples of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "NVFP4-KV decode attention tokens/s; achieved HBM GB/s vs B200 peak"
+FALLBACK_HBM_GBS = 6650.0
+TOKEN_LAYER_BYTES = 1152          # packed K+V codes and scales of 8 heads
+QO_BYTES_PER_SEQ_LAYER = 32 * 128 * 2 * 2   # bf16 query in + bf16 output
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--workload", default="ragged", choices=["ragged"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ distributed
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(device_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(", ") for r in out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def ncu_traffic(kernel_file: str):
+    """Per-launch DRAM bytes of the decode kernel from the committed ncu summary,
+    or None when the kernel source changed since that capture."""
+    path = os.path.join(ROOT, "profiles", "decode_ragged_ncu.md")
+    src = os.path.join(ROOT, "bit_attention_decode_b200", "csrc", kernel_file)
+    try:
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        vals = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and line.strip().startswith("- "):
+                    k, v = line.strip()[2:].split(":", 1)
+                    vals[k.strip()] = v.strip()
+        if vals.get("kernel_source_sha256_16") != sha:
+            return None
+        return float(vals["dram_bytes_per_full_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------------ workload
+class Ragged:
+    """Device-resident ragged decode workload (one replica)."""
+
+    def __init__(self, kvq, synth):
+        self.kvq = kvq
+        w = synth.WORKLOADS["ragged"]
+        self.w = w
+        L, B, S = w.num_layers, w.batch, w.decode_steps
+        self.L, self.B, self.S = L, B, S
+        dev = "cuda"
+        self.lens = synth.ragged_lengths(w)                          # [B] int32
+        cap = self.lens + S
+        self.page_table, self.num_pages = synth.build_page_table(w, cap)
+        self.shape = kvq.Shape(L, w.num_q_heads, w.num_kv_heads)
+        kc = torch.stack([synth.calibration_windows(w, l, dev)[0] for l in range(L)])
+        vc = torch.stack([synth.calibration_windows(w, l, dev)[1] for l in range(L)])
+        self.calib = kvq.calibrate_smoothing(self.shape, kc, vc, exclude_pos0=True)
+        del kc, vc
+        self.cache = kvq.new_cache(self.shape, self.num_pages, dev)
+        H, D = w.num_kv_heads, w.head_dim
+        self.k_new = torch.empty(S, L, B, H, D, dtype=torch.bfloat16, device=dev)
+        self.v_new = torch.empty_like(self.k_new)
+        pos = torch.arange(S)[:, None] + self.lens[None, :].long()          # [S][B]
+        seq = torch.arange(B)[None, :].expand(S, B)
+        self.slots = synth.slot_mapping(self.page_table, seq.reshape(-1), pos.reshape(-1)).view(S, B).to(dev)
+        prefix_slots = torch.cat([synth.slot_mapping(self.page_table, torch.full((int(n),), b), torch.arange(int(n)))
+                                  for b, n in enumerate(self.lens.tolist())]).to(dev)
+        for l in range(L):
+            ks, vs = [], []
+            for b, n in enumerate(self.lens.tolist()):
+                k, v = synth.sequence_kv(w, l, b, n + S, dev)
+                ks.append(k[:n])
+                vs.append(v[:n])
+                self.k_new[:, l, b] = k[n:]
+                self.v_new[:, l, b] = v[n:]
+            kvq.quantize_append(self.shape, self.calib, self.cache, torch.cat(ks), torch.cat(vs), prefix_slots,
+                                layer0=l)
+            del ks, vs
+        self.q = torch.stack([torch.stack([synth.decode_queries(w, l, s, dev) for l in range(L)])
+                              for s in range(S)])                             # [S][L][B][Hq][D]
+        self.seq_lens = (self.lens[None, :] + torch.arange(1, S + 1)[:, None]).to(torch.int32).to(dev)
+        self.page_table_dev = self.page_table.to(dev)
+        self.out = torch.empty(L, B, w.num_q_heads, D, dtype=torch.bfloat16, device=dev)
+        need = kvq.decode_workspace_bytes(self.shape, L, B, self.page_table.shape[1])
+        self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        self.launches_per_step = 2 + (1 if need else 0)
+        torch.cuda.synchronize()
+
+    def decode_bytes(self, s: int) -> int:
+        valid = int(self.lens.sum()) + self.B * (s + 1)
+        return valid * self.L * TOKEN_LAYER_BYTES + self.B * self.L * QO_BYTES_PER_SEQ_LAYER
+
+    def append(self, s: int):
+        self.kvq.quantize_append(self.shape, self.calib, self.cache, self.k_new[s], self.v_new[s], self.slots[s])
+
+    def decode(self, s: int):
+        self.kvq.decode_attention(self.shape, self.calib, self.cache, self.q[s], self.page_table_dev,
+                                  self.seq_lens[s], out=self.out, workspace=self.ws)
+
+
+def time_device(wl: Ragged, warmup: int, steps: int, world: int):
+    st = torch.cuda.current_stream()
+    for i in range(warmup):
+        s = i % wl.S
+        wl.append(s)
+        wl.decode(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dec_bytes = 0
+    t0.record(st)
+    for i in range(steps):
+        s = (warmup + i) % wl.S
+        wl.append(s)
+        ev[i][0].record(st)
+        wl.decode(s)
+        ev[i][1].record(st)
+        dec_bytes += wl.decode_bytes(s)
+    t1.record(st)
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms = t0.elapsed_time(t1)
+    dec_ms = [a.elapsed_time(b) for a, b in ev]
+    return total_ms, dec_ms, dec_bytes / steps
+
+
+def time_e2e(wl: Ragged, steps: int, world: int):
+    """Same steps through the public API from pinned host buffers, copies inside."""
+    st = torch.cuda.current_stream()
+    S = wl.S
+    hq = wl.q[:min(S, steps)].cpu().pin_memory()
+    hk = wl.k_new[:min(S, steps)].cpu().pin_memory()
+    hv = wl.v_new[:min(S, steps)].cpu().pin_memory()
+    hslots = wl.slots.cpu().pin_memory()
+    hlens = wl.seq_lens.cpu().pin_memory()
+    hout = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(wl.q[0]), torch.empty_like(wl.k_new[0]), torch.empty_like(wl.v_new[0])
+    dslots, dlens = torch.empty_like(wl.slots[0]), torch.empty_like(wl.seq_lens[0])
+    h2d = hq[0].numel() * 2 + hk[0].numel() * 2 * 2 + hslots[0].numel() * 8 + hlens[0].numel() * 4
+    d2h = hout.numel() * 2
+    torch.cuda.synchronize()
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(st)
+    for i in range(steps):
+        s = i % hq.shape[0]
+        dq.copy_(hq[s], non_blocking=True)
+        dk.copy_(hk[s], non_blocking=True)
+        dv.copy_(hv[s], non_blocking=True)
+        dslots.copy_(hslots[s], non_blocking=True)
+        dlens.copy_(hlens[s], non_blocking=True)
+        wl.kvq.quantize_append(wl.shape, wl.calib, wl.cache, dk, dv, dslots)
+        wl.kvq.decode_attention(wl.shape, wl.calib, wl.cache, dq, wl.page_table_dev, dlens, out=wl.out,
+                                workspace=wl.ws)
+        hout.copy_(wl.out, non_blocking=True)
+    t1.record(st)
+    torch.cuda.synchronize()
+    barrier(world)
+    return t0.elapsed_time(t1), h2d, d2h
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample(seconds: float, layers=None):
+    """Time the oracle on (layer, sequence) units of a ragged decode step until
+    `seconds` pass; returns (tokens/s extrapolated to the full step, sample text)."""
+    import numpy as np
+
+    import oracle
+    import synth
+    w = synth.WORKLOADS["ragged"]
+    lens = synth.ragged_lengths(w)
+    units = [(l, b) for l in (layers or range(w.num_layers)) for b in range(w.batch)]
+    done_tok_layers = 0
+    spent = 0.0
+    n_units = 0
+    cal_cache = {}
+    for (l, b) in units:
+        if spent >= seconds:
+            break
+        if l not in cal_cache:
+            kc, vc = synth.calibration_windows(w, l)
+            cal_cache[l] = oracle.calibrate(kc[None], vc[None], exclude_pos0=True)
+        s, inv, gk, gv = cal_cache[l]
+        n = int(lens[b]) + 1
+        k, v = synth.sequence_kv(w, l, b, n)
+        q = synth.decode_queries(w, l, 0)[b][None]
+        k32, v32, q32 = k.float().numpy(), v.float().numpy(), q.float().numpy()
+        t = time.perf_counter()
+        oracle.decode_reference(q32, k32, v32, s[0], inv[0], gk[0], gv[0])
+        spent += time.perf_counter() - t
+        done_tok_layers += n
+        n_units += 1
+    full_tok_layers = (int(lens.sum()) + w.batch) * w.num_layers
+    step_s = spent / done_tok_layers * full_tok_layers
+    sample = (f"{n_units} (layer, sequence) units of a ragged decode step ({done_tok_layers} token-layers, "
+              f"{spent:.1f} s), extrapolated linearly to all 36 layers x 64 sequences")
+    return w.batch / step_s, sample, spent
+
+
+def cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+# ------------------------------------------------------------------ main
+def config_block(wl=None):
+    return {"workload": "ragged decode: 36 layers, 32 q / 8 kv heads, head_dim 128, batch 64, "
+                        "lengths U[1024,8192], 16-token pages in shuffled order, 64 append+decode steps cycled",
+            "batch": 64, "layers": 36, "kv_cache": "nvfp4 (e2m1 codes, e4m3 per-16 scales, fp32 tensor scale)",
+            "l2": "inputs larger than L2 (about 12.4 GB of cache read per step)",
+            "parallelism": "replicas (independent sequences per GPU)"}
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_setup(args)
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        vals = []
+        spent_total = 0.0
+        sample = ""
+        for i in range(args.warmup + args.steps):
+            v, sample, spent = oracle_sample(max(1.0, args.cpu_seconds / 4), layers=[i % 36])
+            if i >= args.warmup:
+                vals.append(v)
+                spent_total += spent
+        value = statistics.median(vals)
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": 64 / value * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": config_block(), "impl": "reference",
+                "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores(), "kind": "oracle",
+                                 "sample": "per step: " + sample},
+                "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import bit_attention_decode_b200 as kvq
+    import synth
+    assert torch.cuda.is_available(), "bench needs a CUDA device"
+    t_setup = time.time()
+    wl = Ragged(kvq, synth)
+    sys.stderr.write(f"[bench] setup {time.time() - t_setup:.1f} s, {wl.num_pages} pages, "
+                     f"cache {wl.cache.data.numel() / 1e9:.2f} GB\n")
+    clock = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    total_ms, dec_ms, dec_bytes = time_device(wl, max(3, args.warmup), args.steps, world)
+    clocks = clock.stop() if clock else None
+    total_ms = max_over_ranks(total_ms, world)
+    value = world * wl.B * args.steps / (total_ms / 1e3)
+    dec_avg_ms = statistics.mean(dec_ms)
+    achieved = dec_bytes / (dec_avg_ms / 1e3) / 1e9
+    peak, peak_kind = measured_peak()
+    traffic = ncu_traffic("kvq_decode.cu")
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_block(wl),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
+                         "kernel": "kvq decode (+split combine)", "alg_bytes_per_launch": dec_bytes},
+            "gpu_launches": wl.launches_per_step * args.steps,
+            "clocks": clocks}
+    if not args.no_e2e:
+        e_ms, h2d, d2h = time_e2e(wl, args.steps, world)
+        e_ms = max_over_ranks(e_ms, world)
+        line["e2e"] = {"value": world * wl.B * args.steps / (e_ms / 1e3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        del wl
+        torch.cuda.empty_cache()
+        v, sample, _ = oracle_sample(args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores(), "kind": "oracle",
+                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

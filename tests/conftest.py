@@ -24,3 +24,22 @@ def read_golden(name):
             if line and not line.startswith("#"):
                 rows.append(line.split())
     return rows
+
+
+@pytest.fixture(scope="session")
+def kvq_lib():
+    """The binding module; builds libkvq.so in-tree first if it is missing."""
+    from bit_attention_decode_b200 import build as _build
+    if not _build.up_to_date():
+        _build.build()
+    import bit_attention_decode_b200 as kvq
+    return kvq
+
+
+@pytest.fixture(scope="session")
+def kvq(kvq_lib):
+    """The binding module on a CUDA device (GPU tests only)."""
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("GPU test run without a CUDA device")
+    return kvq_lib

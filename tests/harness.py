@@ -1,0 +1,142 @@
+"""Test harness: drive the CUDA library and the oracle on the same inputs.
+
+Inputs come from ``synth``; the oracle receives host copies of exactly the
+tensors the library saw.  The cache is read back and unpacked here following
+the byte layout documented in ``include/kvq.h`` (this file's own code, shared
+with neither side).
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import torch
+
+import oracle
+import synth
+
+# ------------------------------------------------------------------ tolerances
+# Attention outputs against the oracle on the same dequantised cache:
+# rel-L2 <= 2e-3 and max-abs <= 1e-2 (fp32 accumulate).  With bf16 outputs the
+# max-abs bound is widened to one bf16 ulp of the oracle value where that is
+# larger, since rounding the output alone can exceed 1e-2 when |o| >= 4.
+REL_L2 = 2e-3
+MAX_ABS = 1e-2
+
+
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    a = np.abs(x).astype(np.float64)
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return 2.0 ** (e - 7)
+
+
+def check_attention(got, want, what=""):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    assert got.shape == want.shape, (got.shape, want.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    err = np.abs(got - want)
+    rel = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
+    bound = np.maximum(MAX_ABS, bf16_ulp(want)) if what.endswith("bf16") else MAX_ABS
+    worst = np.unravel_index(np.argmax(err - bound), err.shape)
+    assert rel <= REL_L2, f"{what}: rel-L2 {rel:.3e} > {REL_L2}"
+    assert np.all(err <= bound), f"{what}: max-abs {err[worst]:.3e} at {worst} (want {want[worst]:.4f})"
+    return rel, float(err.max())
+
+
+# ------------------------------------------------------------------ cache readback
+def unpack_nibbles(b: np.ndarray) -> np.ndarray:
+    """[..., 64] code bytes -> [..., 128] codes (low nibble = even element)."""
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), np.uint8)
+    out[..., 0::2] = b & 0x0F
+    out[..., 1::2] = b >> 4
+    return out
+
+
+def read_tokens(cache_layer: np.ndarray, Hkv: int, page_table_row: np.ndarray, n: int):
+    """Codes and scales of tokens 0..n-1 of one sequence, in logical layout:
+    kc, vc [n][H][128] one code per byte; ksf, vsf [n][H][8]."""
+    tiles = cache_layer.reshape(cache_layer.shape[0], Hkv, 2304)
+    t = np.arange(n)
+    pages = page_table_row[t // 16]
+    off = t % 16
+    sel = tiles[pages]                                   # [n][H][2304]
+    kcb = sel[:, :, 0:1024].reshape(n, Hkv, 16, 64)[np.arange(n), :, off]
+    ksf = sel[:, :, 1024:1152].reshape(n, Hkv, 16, 8)[np.arange(n), :, off]
+    vcb = sel[:, :, 1152:2176].reshape(n, Hkv, 16, 64)[np.arange(n), :, off]
+    vsf = sel[:, :, 2176:2304].reshape(n, Hkv, 8, 16)[np.arange(n), :, :, off]
+    return unpack_nibbles(kcb), ksf, unpack_nibbles(vcb), vsf
+
+
+# ------------------------------------------------------------------ problem setup
+@dataclasses.dataclass
+class Problem:
+    """A workload instance on the device plus what the oracle needs."""
+    w: synth.Workload
+    layers: list
+    lens: torch.Tensor          # [B] int32 cached tokens per sequence
+    page_table: torch.Tensor    # [B][maxp] int32 (host)
+    num_pages: int
+    shape: object
+    calib: object
+    cache: object
+    k_calib: np.ndarray         # [nl][W][T][H][D] fp32 host copies
+    v_calib: np.ndarray
+    seqs: dict                  # (layer index, b) -> (k, v) fp32 host [n][H][D]
+
+
+def build_problem(kvq, w: synth.Workload, lens, layers=None, extra_tokens: int = 0, shuffle: bool = True,
+                  keep_host=True, device="cuda", gen_device="cpu"):
+    """Calibrate, then append each sequence's first lens[b] tokens, one layer at a time."""
+    layers = list(range(w.num_layers)) if layers is None else list(layers)
+    lens = torch.as_tensor(lens, dtype=torch.int32)
+    nl = len(layers)
+    shape = kvq.Shape(num_layers=nl, num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads,
+                      use_hadamard=w.hadamard)
+    kc = torch.stack([synth.calibration_windows(w, l, gen_device)[0] for l in layers])
+    vc = torch.stack([synth.calibration_windows(w, l, gen_device)[1] for l in layers])
+    calib = kvq.calibrate_smoothing(shape, kc.to(device).contiguous(), vc.to(device).contiguous())
+    page_table, num_pages = synth.build_page_table(w, lens + extra_tokens, shuffle=shuffle)
+    cache = kvq.new_cache(shape, num_pages, device)
+    seqs = {}
+    for li, l in enumerate(layers):
+        ks, vs, slots = [], [], []
+        for b in range(len(lens)):
+            n = int(lens[b])
+            k, v = synth.sequence_kv(w, l, b, n + extra_tokens, gen_device)
+            if keep_host:
+                seqs[(li, b)] = (k.float().cpu().numpy(), v.float().cpu().numpy())
+            ks.append(k[:n])
+            vs.append(v[:n])
+            slots.append(synth.slot_mapping(page_table, torch.full((n,), b), torch.arange(n)))
+        k = torch.cat(ks).to(device)
+        v = torch.cat(vs).to(device)
+        sm = torch.cat(slots).to(device)
+        kvq.quantize_append(shape, calib, cache, k.contiguous(), v.contiguous(), sm, layer0=li)
+    return Problem(w, layers, lens, page_table, num_pages, shape, calib, cache,
+                   kc.float().cpu().numpy(), vc.float().cpu().numpy(), seqs)
+
+
+def oracle_calibration(p: Problem):
+    return oracle.calibrate(p.k_calib, p.v_calib, exclude_pos0=True, hadamard=p.w.hadamard)
+
+
+def calib_host(p: Problem):
+    return (p.calib.k_smooth.cpu().numpy(), p.calib.k_inv_smooth.cpu().numpy(),
+            p.calib.k_gscale.cpu().numpy(), p.calib.v_gscale.cpu().numpy())
+
+
+def oracle_sequence(p: Problem, li: int, b: int, n: int, cal):
+    """Oracle codes of tokens 0..n-1 of sequence b in layer li."""
+    s, inv, gk, gv = cal
+    k, v = p.seqs[(li, b)]
+    return oracle.quantize_kv(k[:n], v[:n], inv[li], gk[li], gv[li], p.w.hadamard)
+
+
+def oracle_attend(p: Problem, li: int, b: int, q_rows: np.ndarray, q_start: int, n: int, cal):
+    """Oracle attention of q_rows [Tq][Hq][D] over the first n tokens."""
+    s, inv, gk, gv = cal
+    qz = oracle_sequence(p, li, b, n, cal)
+    kx = oracle.dequantize_rows(qz["kc"], qz["ksf"], gk[li])
+    vx = oracle.dequantize_rows(qz["vc"], qz["vsf"], gv[li])
+    return oracle.attention(q_rows, q_start, s[li], kx, vx, p.w.hadamard)

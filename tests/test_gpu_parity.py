@@ -1,0 +1,164 @@
+"""Parity of the CUDA path with the oracle on small workloads.
+
+Codes and scales must match bit for bit; attention outputs within the
+tolerance stated in tests/harness.py.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import harness
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def small(name="qwen3_8b", **kw):
+    return dataclasses.replace(synth.WORKLOADS[name], **kw)
+
+
+def assert_codes_equal(p, li, b, n, cal):
+    layer = p.cache.data[li].cpu().numpy()
+    kc, ksf, vc, vsf = harness.read_tokens(layer, p.w.num_kv_heads, p.page_table[b].numpy(), n)
+    ref = harness.oracle_sequence(p, li, b, n, cal)
+    for name, got in (("kc", kc), ("ksf", ksf), ("vc", vc), ("vsf", vsf)):
+        want = ref[name]
+        if not np.array_equal(got, want):
+            idx = np.argwhere(got != want)[0]
+            raise AssertionError(f"{name} mismatch layer {li} seq {b} at {tuple(idx)}: "
+                                 f"device {got[tuple(idx)]} oracle {want[tuple(idx)]} ({(got != want).sum()} total)")
+
+
+def decode_all(kvq, p, step=0, out_dtype=torch.float32, lens=None):
+    q = torch.stack([synth.decode_queries(p.w, l, step) for l in p.layers])
+    lens = p.lens if lens is None else lens
+    out = kvq.decode_attention(p.shape, p.calib, p.cache, q.cuda(), p.page_table.cuda(), lens.cuda(),
+                               out_dtype=out_dtype)
+    return q.float().numpy(), out.float().cpu().numpy()
+
+
+def test_tiny_workload_end_to_end(kvq):
+    w = synth.WORKLOADS["tiny"]
+    p = harness.build_problem(kvq, w, lens=[256])
+    cal = harness.oracle_calibration(p)
+    for got, want, name in zip(harness.calib_host(p), cal, ("s", "inv_s", "g_K", "g_V")):
+        np.testing.assert_array_equal(got, want, err_msg=name)
+    assert_codes_equal(p, 0, 0, 256, cal)
+    for dt, tag in ((torch.float32, "f32"), (torch.bfloat16, "bf16")):
+        q, out = decode_all(kvq, p, out_dtype=dt)
+        want = harness.oracle_attend(p, 0, 0, q[0, 0][None], 255, 256, cal)
+        harness.check_attention(out[0, 0], want[0], f"tiny decode {tag}")
+
+
+@pytest.mark.parametrize("hadamard", [False, True])
+def test_ragged_multilayer_bf16(kvq, hadamard):
+    w = small(num_layers=3, batch=4, calib_windows=2, calib_len=64, hadamard=hadamard)
+    lens = [1, 17, 300, 129]
+    p = harness.build_problem(kvq, w, lens=lens, layers=[0, 2])
+    cal = harness.oracle_calibration(p)
+    for got, want in zip(harness.calib_host(p), cal):
+        np.testing.assert_array_equal(got, want)
+    for li in range(2):
+        for b, n in enumerate(lens):
+            assert_codes_equal(p, li, b, n, cal)
+    for dt, tag in ((torch.float32, "f32"), (torch.bfloat16, "bf16")):
+        q, out = decode_all(kvq, p, out_dtype=dt)
+        for li in range(2):
+            for b, n in enumerate(lens):
+                want = harness.oracle_attend(p, li, b, q[li, b][None], n - 1, n, cal)
+                harness.check_attention(out[li, b], want[0], f"layer {li} seq {b} len {n} {tag}")
+
+
+def test_many_units_single_split(kvq):
+    # enough (layer, sequence, head) units that the decode needs no split
+    w = small(num_layers=10, batch=64, calib_windows=1, calib_len=32)
+    lens = (torch.arange(64) % 7 * 9 + 1).tolist()
+    p = harness.build_problem(kvq, w, lens=lens)
+    assert kvq.decode_workspace_bytes(p.shape, 10, 64, p.page_table.shape[1]) == 0
+    cal = harness.oracle_calibration(p)
+    q, out = decode_all(kvq, p, out_dtype=torch.bfloat16)
+    for li in (0, 9):
+        for b in (0, 5, 63):
+            n = lens[b]
+            want = harness.oracle_attend(p, li, b, q[li, b][None], n - 1, n, cal)
+            harness.check_attention(out[li, b], want[0], f"layer {li} seq {b} bf16")
+
+
+def test_long_sequence_many_splits(kvq):
+    w = small(num_layers=1, batch=1, calib_windows=1, calib_len=128)
+    p = harness.build_problem(kvq, w, lens=[5000])
+    assert kvq.decode_workspace_bytes(p.shape, 1, 1, p.page_table.shape[1]) > 0
+    cal = harness.oracle_calibration(p)
+    q, out = decode_all(kvq, p)
+    want = harness.oracle_attend(p, 0, 0, q[0, 0][None], 4999, 5000, cal)
+    harness.check_attention(out[0, 0], want[0], "5000 tokens f32")
+
+
+def test_page_order_does_not_change_results(kvq):
+    w = small(num_layers=1, batch=3, calib_windows=1, calib_len=64)
+    lens = [40, 200, 77]
+    a = harness.build_problem(kvq, w, lens=lens, shuffle=True)
+    b = harness.build_problem(kvq, w, lens=lens, shuffle=False)
+    _, oa = decode_all(kvq, a)
+    _, ob = decode_all(kvq, b)
+    np.testing.assert_array_equal(oa, ob)
+
+
+def test_prefill_chunk(kvq):
+    w = small(num_layers=2, batch=2, calib_windows=1, calib_len=64, prefill_chunk=48)
+    P0 = [100, 33]
+    Tq = 48
+    lens = [n + Tq for n in P0]
+    p = harness.build_problem(kvq, w, lens=lens)
+    cal = harness.oracle_calibration(p)
+    q = torch.stack([synth.prefill_queries(w, l) for l in p.layers])        # [nl][B][Tq][Hq][D]
+    q_start = torch.tensor(P0, dtype=torch.int32)
+    for dt, tag in ((torch.float32, "f32"), (torch.bfloat16, "bf16")):
+        out = kvq.prefill_attention(p.shape, p.calib, p.cache, q.cuda(), q_start.cuda(), p.page_table.cuda(),
+                                    p.lens.cuda(), out_dtype=dt).float().cpu().numpy()
+        for li in range(2):
+            for b in range(2):
+                want = harness.oracle_attend(p, li, b, q[li, b].float().numpy(), P0[b], lens[b], cal)
+                harness.check_attention(out[li, b], want, f"prefill layer {li} seq {b} {tag}")
+
+
+def test_zero_length_gives_zero_rows(kvq):
+    w = small(num_layers=1, batch=2, calib_windows=1, calib_len=32)
+    p = harness.build_problem(kvq, w, lens=[20, 20])
+    _, out = decode_all(kvq, p, lens=torch.tensor([0, 20], dtype=torch.int32))
+    assert np.all(out[0, 0] == 0) and np.any(out[0, 1] != 0)
+
+
+def test_device_faults_are_flagged_not_trapped(kvq):
+    w = small(num_layers=1, batch=2, calib_windows=1, calib_len=32)
+    p = harness.build_problem(kvq, w, lens=[40, 40])
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    # a page id outside the pool: the row is zeroed and BAD_PAGE set
+    pt = p.page_table.clone()
+    pt[1, 1] = p.num_pages + 5
+    q = synth.decode_queries(w, 0, 0)[None].cuda()
+    out = kvq.decode_attention(p.shape, p.calib, p.cache, q, pt.cuda(), p.lens.cuda(), status=status,
+                               out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert status.item() & kvq.DEV_BAD_PAGE
+    assert torch.all(out[0, 1] == 0) and torch.any(out[0, 0] != 0)
+    # a length beyond the page table
+    status.zero_()
+    out = kvq.decode_attention(p.shape, p.calib, p.cache, q, p.page_table.cuda(),
+                               torch.tensor([40, 10 ** 6], dtype=torch.int32, device="cuda"), status=status)
+    torch.cuda.synchronize()
+    assert status.item() & kvq.DEV_BAD_LEN
+    assert torch.all(out[0, 1] == 0)
+    # a slot beyond the cache: skipped and flagged, the rest written
+    status.zero_()
+    before = p.cache.data.clone()
+    k, v = synth.sequence_kv(w, 0, 0, 2, "cuda")
+    slots = torch.tensor([p.num_pages * 16 + 3, 5], dtype=torch.int64, device="cuda")
+    kvq.quantize_append(p.shape, p.calib, p.cache, k.contiguous(), v.contiguous(), slots, status=status)
+    torch.cuda.synchronize()
+    assert status.item() & kvq.DEV_BAD_SLOT
+    changed = (p.cache.data != before).nonzero()
+    assert changed.numel() > 0 and torch.all(changed[:, 1] == 0)           # only page 0 (slot 5) touched
