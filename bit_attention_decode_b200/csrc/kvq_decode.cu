@@ -100,10 +100,10 @@ __device__ __forceinline__ void attend_tokens(const AttnArgs& a, const uint8_t* 
             const uint32_t k01 = e2m1x2_to_f16x2(kc & 0xFFu), k23 = e2m1x2_to_f16x2(kc >> 8);
             const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&k01));
             const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&k23));
-            float s = q[0] * f01.x + q[1] * f01.y + q[2] * f23.x + q[3] * f23.y;
+            // the block scale belongs to this lane's 4 dims (block lane / 4)
+            float s = (q[0] * f01.x + q[1] * f01.y + q[2] * f23.x + q[3] * f23.y) * ksf;
 #pragma unroll
             for (int w = 16; w >= 1; w >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, w);
-            s *= ksf;
             const uint32_t vc = *reinterpret_cast<const uint16_t*>(tile + kVCodes + t * 64 + 2 * lane);
             const float vsf = e4m3_to_f32(tile[kVScales + (lane >> 2) * 16 + t]);
             const uint32_t v01 = e2m1x2_to_f16x2(vc & 0xFFu), v23 = e2m1x2_to_f16x2(vc >> 8);
