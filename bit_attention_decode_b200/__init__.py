@@ -73,6 +73,9 @@ _lib.kvq_prefill_workspace_bytes.argtypes = [_SHP, _I32, _I32, _I32]
 _lib.kvq_prefill_attention.restype = _I32
 _lib.kvq_prefill_attention.argtypes = [_SHP, _CAL, _CCH, _I32, _I32, _P, _I32, _I32, _P, _P, _I32, _P, _I32,
                                        _P, _I32, _P, ctypes.c_size_t, _P, _P]
+_lib.kvq_decode_attention_noalloc.restype = _I32
+_lib.kvq_decode_attention_noalloc.argtypes = [_SHP, _CAL, _CCH, _I32, _I32, _P, _I32, _P, _I32, _P, _I32, _P,
+                                              _I32, _P, _P]
 _lib.kvq_round_e2m1.restype = _I32
 _lib.kvq_round_e2m1.argtypes = [_P, _P, ctypes.c_int64, _P]
 _lib.kvq_round_e4m3.restype = _I32
@@ -80,7 +83,10 @@ _lib.kvq_round_e4m3.argtypes = [_P, _P, ctypes.c_int64, _P]
 
 EXPORTED = ("kvq_page_bytes", "kvq_status_string", "kvq_version", "kvq_calibrate_smoothing",
             "kvq_quantize_append", "kvq_decode_workspace_bytes", "kvq_decode_attention",
-            "kvq_prefill_workspace_bytes", "kvq_prefill_attention", "kvq_round_e2m1", "kvq_round_e4m3")
+            "kvq_prefill_workspace_bytes", "kvq_prefill_attention", "kvq_decode_attention_noalloc",
+            "kvq_round_e2m1", "kvq_round_e4m3")
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class KVQError(RuntimeError):
@@ -230,6 +236,24 @@ def decode_attention(shape: Shape, calib: Calibration, cache: PagedCache, q: tor
                                      layer0, nl, q.data_ptr(), _dtype_code(q), page_table.data_ptr(), maxp,
                                      seq_lens.data_ptr(), B, out.data_ptr(), _dtype_code(out), _ptr(workspace),
                                      ws_bytes, _ptr(status), _stream()), "kvq_decode_attention")
+    return out
+
+
+def decode_attention_noalloc(shape: Shape, calib: Calibration, cache: PagedCache, q: torch.Tensor,
+                             page_table: torch.Tensor, seq_lens: torch.Tensor, out: torch.Tensor,
+                             layer0: int = 0, status: Optional[torch.Tensor] = None):
+    """decode_attention with the library's static scratch array instead of a
+    workspace: for callers that cannot allocate device memory.  ``out`` is
+    required (this call allocates nothing); calls must not overlap on the GPU."""
+    if q.dim() == 3:
+        q = q[None]
+    nl, B = q.shape[0], q.shape[1]
+    _need_cuda(q, page_table, seq_lens, out, status)
+    _check(_lib.kvq_decode_attention_noalloc(ctypes.byref(shape.c()), ctypes.byref(calib.c()),
+                                             ctypes.byref(cache.c()), layer0, nl, q.data_ptr(), _dtype_code(q),
+                                             page_table.data_ptr(), page_table.shape[1], seq_lens.data_ptr(), B,
+                                             out.data_ptr(), _dtype_code(out), _ptr(status), _stream()),
+           "kvq_decode_attention_noalloc")
     return out
 
 

@@ -220,6 +220,35 @@ kvq_status kvq_prefill_attention(const kvq_shape* shape, const kvq_calib* calib,
                                  int32_t* dev_status, void* stream);
 
 /*
+ * kvq_decode_attention_noalloc -- kvq_decode_attention without a workspace
+ * argument, for callers that cannot allocate device memory (code running
+ * inside a host runtime that owns the device-memory budget and forbids
+ * stray allocations, or latency-critical paths that cannot afford
+ * cudaMalloc's implicit device-wide synchronisation).  The pages have no
+ * counterpart to this call; it exists only for such callers.
+ *
+ * Same arguments, results and errors as kvq_decode_attention.  The split-K
+ * scratch is a static device array of KVQ_NOALLOC_SCRATCH_BYTES inside the
+ * library, reserved on every GPU that loads it until the process exits; the
+ * call allocates nothing.  A problem whose kvq_decode_workspace_bytes exceeds
+ * that size returns KVQ_EWORKSPACE and launches nothing.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before
+ *     any stream capture.
+ *   - The array is shared by all calls on a device and keeps the last
+ *     call's contents; the decode writes every partial before reading it, so
+ *     no clearing is needed.  Calls whose GPU work overlaps (other streams,
+ *     other host threads) race on the array: serialise them.
+ */
+#define KVQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+kvq_status kvq_decode_attention_noalloc(const kvq_shape* shape, const kvq_calib* calib, const kvq_cache* cache,
+                                        int32_t layer0, int32_t nlayers, const void* q, int32_t q_dtype,
+                                        const int32_t* page_table, int32_t max_pages_per_seq,
+                                        const int32_t* seq_lens, int32_t batch, void* out, int32_t out_dtype,
+                                        int32_t* dev_status, void* stream);
+
+/*
  * Elementwise format conversions with the kernels' own rounding routines
  * (the ones kvq_quantize_append uses), for checking them against a
  * reference.  x: [n] fp32 device array; codes: [n] bytes, one code per byte
