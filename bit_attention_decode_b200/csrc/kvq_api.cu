@@ -14,10 +14,10 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 kvq_status check_shape(const kvq_shape* s) {
     if (!s) return KVQ_EINVAL;
     if (s->head_dim != kvq::kD || s->page_size != kvq::kPage) return KVQ_EUNSUPPORTED;
-    if (s->num_layers < 1 || s->num_kv_heads < 1 || s->num_kv_heads > 16 || s->num_q_heads < 1)
-        return KVQ_EINVAL;
+    if (s->num_layers < 1 || s->num_kv_heads < 1 || s->num_q_heads < 1) return KVQ_EINVAL;
     if (s->num_q_heads % s->num_kv_heads != 0) return KVQ_EINVAL;
-    if (s->num_q_heads / s->num_kv_heads > 8) return KVQ_EUNSUPPORTED;
+    // one decode CTA holds a warp per kv head; a warp serves up to 4 query heads
+    if (s->num_kv_heads > 8 || s->num_q_heads / s->num_kv_heads > 4) return KVQ_EUNSUPPORTED;
     if (s->use_hadamard != 0 && s->use_hadamard != 1) return KVQ_EINVAL;
     // the rotation's cross-lane butterflies need whole warps of key lanes
     if (s->use_hadamard && (s->num_kv_heads & 1)) return KVQ_EUNSUPPORTED;

@@ -1,0 +1,34 @@
+// kvq_attn.cuh -- argument block and constants shared by the attention kernels.
+#pragma once
+
+#include "kvq_common.cuh"
+
+namespace kvq {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kPartialStride = 132;  // floats per split partial: m, l, pad, pad, o[128]
+
+struct AttnArgs {
+    const uint8_t* cache;      // layer layer0
+    int64_t layer_stride;
+    int num_pages, Hkv, Hq, G, hadamard;
+    const float* smooth;       // [nl][Hkv][D] at layer0
+    const float* gk;           // [nl] at layer0
+    const float* gv;
+    const void* q;             // decode [nl][B][Hq][D]; prefill [nl][B][q_len][Hq][D]
+    const int32_t* page_table;
+    int max_pages;
+    const int32_t* seq_lens;
+    const int32_t* q_start;    // prefill only
+    int batch, q_len;
+    void* out;
+    float* partials;           // decode with splits > 1
+    int splits, pps;
+    int32_t* status;
+};
+
+// tensor-core split-K decode (kvq_decode_tc.cu)
+cudaError_t launch_decode_tc(const AttnArgs& a, int nlayers, bool q_bf16, bool out_bf16, cudaStream_t st);
+size_t decode_tc_smem(int Hkv);
+
+}  // namespace kvq

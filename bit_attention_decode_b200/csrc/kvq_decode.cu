@@ -11,30 +11,9 @@
 
 #include "kvq_common.cuh"
 #include "kvq_internal.h"
+#include "kvq_attn.cuh"
 
 namespace kvq {
-
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kPartialStride = 132;  // floats per split partial: m, l, pad, pad, o[128]
-
-struct AttnArgs {
-    const uint8_t* cache;      // layer layer0
-    int64_t layer_stride;
-    int num_pages, Hkv, Hq, G, hadamard;
-    const float* smooth;       // [nl][Hkv][D] at layer0
-    const float* gk;           // [nl] at layer0
-    const float* gv;
-    const void* q;             // decode [nl][B][Hq][D]; prefill [nl][B][q_len][Hq][D]
-    const int32_t* page_table;
-    int max_pages;
-    const int32_t* seq_lens;
-    const int32_t* q_start;    // prefill only
-    int batch, q_len;
-    void* out;
-    float* partials;           // decode with splits > 1
-    int splits, pps;
-    int32_t* status;
-};
 
 __device__ __forceinline__ void load4(const float* p, float* x) {
     float4 t = *reinterpret_cast<const float4*>(p);
@@ -126,41 +105,6 @@ __device__ __forceinline__ void attend_tokens(const AttnArgs& a, const uint8_t* 
     }
 }
 
-// grid (splits, batch * Hkv, nlayers); block 32 * G: warp w is q head h*G + w.
-template <typename TQ, typename TO>
-__global__ void __launch_bounds__(256) decode_kernel(AttnArgs a) {
-    const int split = blockIdx.x, b = blockIdx.y / a.Hkv, h = blockIdx.y % a.Hkv, li = blockIdx.z;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int hq = h * a.G + warp;
-    const int len = __ldg(a.seq_lens + b);
-    bool bad = false;
-    if (len < 0 || len > a.max_pages * kPage) {
-        bad = true;
-        if (threadIdx.x == 0 && split == 0 && h == 0) set_status(a.status, KVQ_DEV_BAD_LEN);
-    }
-    float q[4];
-    load4(reinterpret_cast<const TQ*>(a.q) + (((size_t)li * a.batch + b) * a.Hq + hq) * kD + 4 * lane, q);
-    query_transform(q, a.smooth + ((size_t)li * a.Hkv + h) * kD, lane, a.hadamard != 0,
-                    __ldg(a.gk + li) * kLog2e * kInvSqrt128);
-    float m = -INFINITY, l = 0.0f, o[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if (!bad) {
-        const int tok0 = split * a.pps * kPage, tok1 = min(len, tok0 + a.pps * kPage);
-        attend_tokens(a, a.cache + (size_t)li * a.layer_stride, b, h, q, tok0, tok1, lane, m, l, o, bad);
-        if (bad && lane == 0) set_status(a.status, KVQ_DEV_BAD_PAGE);
-    }
-    if (a.splits == 1) {
-        const float sc = (bad || l == 0.0f) ? 0.0f : __ldg(a.gv + li) / l;
-        float r[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) r[i] = o[i] * sc;
-        store4(reinterpret_cast<TO*>(a.out) + (((size_t)li * a.batch + b) * a.Hq + hq) * kD + 4 * lane, r);
-    } else {
-        float* part = a.partials + ((((size_t)li * a.batch + b) * a.Hq + hq) * a.splits + split) * kPartialStride;
-        if (lane == 0) { part[0] = bad ? INFINITY : m; part[1] = l; }
-        store4(part + 4 + 4 * lane, o);
-    }
-}
-
 // Log-sum-exp merge of the split partials in split order.  A poisoned split
 // (bad page or length) zeroes the row.  grid (batch * Hq, nlayers), block 128.
 template <typename TO>
@@ -223,12 +167,16 @@ __global__ void __launch_bounds__(256) prefill_kernel(AttnArgs a) {
 
 // ------------------------------------------------------------------ host side
 DecodePlan decode_plan(const kvq_shape& s, int nlayers, int batch, int max_pages) {
-    const long units = (long)nlayers * batch * s.num_kv_heads;
-    const long target = 148L * 16 * 2;   // two waves of CTAs at 16 CTAs per SM
+    // one CTA per (layer, sequence, split) covering all kv heads; aim for two
+    // waves at two resident CTAs per SM, splitting sequences only when the
+    // (layer, sequence) units alone cannot fill the GPU
+    (void)s;
+    const long units = (long)nlayers * batch;
+    const long target = 148L * 2 * 2;
     int splits = 1;
-    if (units < target && max_pages > 4) {
+    if (units < target && max_pages > 8) {
         splits = (int)((target + units - 1) / units);
-        splits = min(splits, (max_pages + 3) / 4);   // at least 4 pages per split
+        splits = min(splits, (max_pages + 7) / 8);   // at least 8 pages per split
     }
     int pps = (max_pages + splits - 1) / splits;
     if (pps < 1) pps = 1;
@@ -277,13 +225,8 @@ kvq_status decode(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cache
     a.pps = p.pages_per_split;
     a.q_len = 1;
     a.partials = reinterpret_cast<float*>(ws);
-    dim3 grid(p.splits, batch * s.num_kv_heads, nlayers);
-    const int threads = 32 * a.G;
     const bool qb = q_dtype == KVQ_BF16, ob = out_dtype == KVQ_BF16;
-    if (qb && ob) decode_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, threads, 0, st>>>(a);
-    else if (qb) decode_kernel<__nv_bfloat16, float><<<grid, threads, 0, st>>>(a);
-    else if (ob) decode_kernel<float, __nv_bfloat16><<<grid, threads, 0, st>>>(a);
-    else decode_kernel<float, float><<<grid, threads, 0, st>>>(a);
+    if (launch_decode_tc(a, nlayers, qb, ob, st) != cudaSuccess) return KVQ_ECUDA;
     if (p.splits > 1) {
         dim3 g2(batch * s.num_q_heads, nlayers);
         if (ob) combine_kernel<__nv_bfloat16><<<g2, kD, 0, st>>>(a.partials, p.splits, a.gv, (__nv_bfloat16*)out, batch * s.num_q_heads);

@@ -1,0 +1,490 @@
+// kvq_decode_tc.cu -- split-K decode over the packed NVFP4 cache, with the
+// per-page contractions on the tensor cores (mma.sync m16n8k16, fp16 in,
+// fp32 accumulate) and the dequantisation in registers.
+//
+// Why tensor cores in a bandwidth-bound kernel: one 16-token page of one kv
+// head is 2304 bytes but carries 16 x 128 x 4 multiply-adds for Q.K and as
+// many for P.V (GQA group of 4).  At the HBM roof that is ~125 FP32 FMAs per
+// clock per SM -- the whole FP32 pipe -- before any dequantisation; the
+// tensor cores take the contractions and leave the ALUs the dequantisation
+// and the online softmax.  Every dequantised E2M1 x E4M3 product is exact in
+// fp16; the query and the probabilities are split into fp16 hi + lo columns,
+// so no operand loses precision beyond fp32 accumulation.
+//
+// Work unit (one CTA): one layer, one sequence, one split of its pages, all
+// kv heads.  Warp Hkv is the producer: it streams whole pages (Hkv x 2304
+// contiguous bytes per layer) into a ring of shared-memory stages with
+// cp.async.bulk and mbarrier transaction counts.  Warps 0..Hkv-1 consume:
+// warp h owns kv head h and its G <= 4 query heads.
+//
+// Method: "NVFP4 attention cache on W4A4 Qwen3-8B" (rstation.ai), setup and
+// observation 2 (the smoothing folded into the query); "QServe
+// SmoothAttention" record, Kernels field (fused attention made memory-bound
+// on the 4-bit cache).
+#include "kvq_attn.cuh"
+#include "kvq_common.cuh"
+#include "kvq_internal.h"
+
+namespace kvq {
+
+constexpr int kStages = 4;
+constexpr unsigned kFull = 0xFFFFFFFFu;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // bounded waits give up after 2 s
+
+// ------------------------------------------------------------------ primitives
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Wait for the phase of `parity` to complete; false after kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (global_ns() - t0 > kWaitLimitNs) return false;
+    }
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void mma16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
+    uint32_t d;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+    return d;
+}
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+    __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+    __half2 r = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ float2 unpack_h2(uint32_t a) {
+    return __half22float2(*reinterpret_cast<__half2*>(&a));
+}
+__device__ __forceinline__ uint32_t bcast_lo(uint32_t h2) { return (h2 & 0xFFFFu) | (h2 << 16); }
+__device__ __forceinline__ uint32_t bcast_hi(uint32_t h2) { return (h2 & 0xFFFF0000u) | (h2 >> 16); }
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// four bytes of E2M1 code pairs -> four f16x2 (byte j -> r[j])
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t* r) {
+    asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %4;\n"
+        "  cvt.rn.f16x2.e2m1x2 %0, b0; cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+        "  cvt.rn.f16x2.e2m1x2 %2, b2; cvt.rn.f16x2.e2m1x2 %3, b3; }"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+        : "r"(w));
+}
+
+template <typename T>
+__device__ __forceinline__ void load32(const T* p, float* x);
+template <>
+__device__ __forceinline__ void load32<float>(const float* p, float* x) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float4 t = __ldg(reinterpret_cast<const float4*>(p) + i);
+        x[4 * i] = t.x; x[4 * i + 1] = t.y; x[4 * i + 2] = t.z; x[4 * i + 3] = t.w;
+    }
+}
+template <>
+__device__ __forceinline__ void load32<__nv_bfloat16>(const __nv_bfloat16* p, float* x) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint4 t = __ldg(reinterpret_cast<const uint4*>(p) + i);
+        uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            x[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+            x[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+    }
+}
+
+__device__ __forceinline__ void store16(float* p, const float* x) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        reinterpret_cast<float4*>(p)[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+}
+__device__ __forceinline__ void store16(__nv_bfloat16* p, const float* x) {
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        __nv_bfloat162 t = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+        w[i] = *reinterpret_cast<uint32_t*>(&t);
+    }
+    reinterpret_cast<uint4*>(p)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4*>(p)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+// ------------------------------------------------------------------ kernel
+// grid (splits, batch, nlayers); block 32 * (Hkv + 1); dynamic smem
+// kStages * Hkv * 2304 + barriers.
+template <typename TQ, typename TO>
+__global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int s_flags;    // 1: a bounded wait gave up
+    __shared__ int s_issued;   // pages the producer issued
+
+    const int Hkv = a.Hkv;
+    const uint32_t page_bytes = (uint32_t)Hkv * kTile;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * page_bytes);
+    uint64_t* empty = full + kStages;
+
+    const int split = blockIdx.x, b = blockIdx.y, li = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int len = __ldg(a.seq_lens + b);
+    const bool bad_len = len < 0 || len > a.max_pages * kPage;
+    const int npages = bad_len ? 0 : (len + kPage - 1) / kPage;
+    const int p0 = split * a.pps;
+    const int n = max(0, min(npages, p0 + a.pps) - p0);
+    const int32_t* pt = a.page_table + (size_t)b * a.max_pages + p0;
+
+    if (threadIdx.x == 0) {
+        s_flags = 0;
+        s_issued = 0;
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], Hkv);
+        }
+        mbar_fence_init();
+    }
+    int badp = 0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int pg = __ldg(pt + i);
+        badp |= (pg < 0 || pg >= a.num_pages);
+    }
+    badp = __syncthreads_or(badp);
+    if (threadIdx.x == 0) {
+        if (bad_len && split == 0) set_status(a.status, KVQ_DEV_BAD_LEN);
+        if (badp) set_status(a.status, KVQ_DEV_BAD_PAGE);
+    }
+    const bool poison = bad_len || badp;
+    const uint8_t* layer_base = a.cache + (size_t)li * a.layer_stride;
+
+    // consumer state (kept in registers across the final barrier)
+    const int g = lane >> 2, c = lane & 3;
+    float o[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
+    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.0f, l_b = 0.0f;
+
+    if (warp == Hkv) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0 && !poison) {
+            int i = 0;
+            for (; i < n; ++i) {
+                const int st = i % kStages;
+                if (i >= kStages && !mbar_wait(&empty[st], ((i / kStages) - 1) & 1)) {
+                    atomicOr(&s_flags, 1);
+                    break;
+                }
+                const int pg = __ldg(pt + i);
+                mbar_arrive_expect_tx(&full[st], page_bytes);
+                bulk_g2s(smem + st * page_bytes, layer_base + (size_t)pg * page_bytes, page_bytes, &full[st]);
+            }
+            s_issued = i;
+        }
+    } else if (!poison) {
+        // ---------------------------------------------------------- consumer
+        const int h = warp;
+        const int G = a.G;
+        const int jq = g & 3;                 // query head of this lane's B-fragment column
+        const bool head_ok = jq < G;
+        // query prologue: lane (g, c) holds dims 32c..32c+31 of head jq
+        float qv[32];
+        {
+            const TQ* qs = reinterpret_cast<const TQ*>(a.q) +
+                           (((size_t)li * a.batch + b) * a.Hq + h * G + (head_ok ? jq : 0)) * kD + 32 * c;
+            load32<TQ>(qs, qv);
+            const float* srow = a.smooth + ((size_t)li * Hkv + h) * kD + 32 * c;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) qv[i] = head_ok ? qv[i] * __ldg(srow + i) : 0.0f;
+            float scale = __ldg(a.gk + li) * kLog2e * kInvSqrt128;
+            if (a.hadamard) {
+#pragma unroll
+                for (int hh = 1; hh < 32; hh <<= 1)
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if ((j & hh) == 0) {
+                            const float x = qv[j], y = qv[j + hh];
+                            qv[j] = x + y;
+                            qv[j + hh] = x - y;
+                        }
+#pragma unroll
+                for (int m = 1; m <= 2; m <<= 1) {
+                    const bool upper = (c & m) != 0;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float y = __shfl_xor_sync(kFull, qv[j], m);
+                        qv[j] = upper ? y - qv[j] : qv[j] + y;
+                    }
+                }
+                scale *= kInvSqrt128;
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) qv[i] *= scale;
+        }
+        // power-of-two normalisation of each head into the fp16 range
+        float mx = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fabsf(qv[i]));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+        int ex = 0;
+        if (mx > 0.0f) {
+            frexpf(mx, &ex);
+            ex = max(ex - 1, -100);
+        }
+        const float sig = ldexpf(1.0f, 14 - ex), isig = ldexpf(1.0f, ex - 14);
+        uint32_t qb[16];
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const float x0 = qv[4 * s + 2 * r] * sig, x1 = qv[4 * s + 2 * r + 1] * sig;
+                const uint32_t hv = pack_h2(x0, x1);
+                const float2 f = unpack_h2(hv);
+                qb[2 * s + r] = (g < 4) ? hv : pack_h2(x0 - f.x, x1 - f.y);
+            }
+        const int ha = 2 * (c & 1), hb = ha + 1;   // heads of this lane's score columns
+        const float isg_a = __shfl_sync(kFull, isig, ha * 4);
+        const float isg_b = __shfl_sync(kFull, isig, hb * 4);
+
+        const uint8_t* my_tile = smem + h * kTile;
+        for (int i = 0; i < n; ++i) {
+            const int st = i % kStages;
+            if (!mbar_wait(&full[st], (i / kStages) & 1)) {
+                atomicOr(&s_flags, 1);
+                break;
+            }
+            const uint8_t* T = my_tile + st * page_bytes;
+            const int nvalid = min(kPage, len - (p0 + i) * kPage);
+            // ---- everything this warp needs from the stage, then release it
+            const uint4 kA = *reinterpret_cast<const uint4*>(T + kKCodes + g * 64 + 16 * c);
+            const uint4 kB = *reinterpret_cast<const uint4*>(T + kKCodes + (g + 8) * 64 + 16 * c);
+            const uint32_t ksA = *reinterpret_cast<const uint16_t*>(T + kKScales + g * 8 + 2 * c);
+            const uint32_t ksB = *reinterpret_cast<const uint16_t*>(T + kKScales + (g + 8) * 8 + 2 * c);
+            const uint2 v0 = *reinterpret_cast<const uint2*>(T + kVCodes + (2 * c) * 64 + 8 * g);
+            const uint2 v1 = *reinterpret_cast<const uint2*>(T + kVCodes + (2 * c + 1) * 64 + 8 * g);
+            const uint2 v2 = *reinterpret_cast<const uint2*>(T + kVCodes + (2 * c + 8) * 64 + 8 * g);
+            const uint2 v3 = *reinterpret_cast<const uint2*>(T + kVCodes + (2 * c + 9) * 64 + 8 * g);
+            uint32_t vs01 = *reinterpret_cast<const uint16_t*>(T + kVScales + 16 * g + 2 * c);
+            uint32_t vs89 = *reinterpret_cast<const uint16_t*>(T + kVScales + 16 * g + 2 * c + 8);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+
+            // ---- S = K q~ : tokens (rows) x [4 heads hi | 4 heads lo] (cols)
+            float sacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            {
+                const uint32_t sfA = e4m3x2_to_f16x2(ksA), sfB = e4m3x2_to_f16x2(ksB);
+                const uint32_t sc[4] = {bcast_lo(sfA), bcast_hi(sfA), bcast_lo(sfB), bcast_hi(sfB)};
+                const uint32_t wa[4] = {kA.x, kA.y, kA.z, kA.w}, wb[4] = {kB.x, kB.y, kB.z, kB.w};
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    uint32_t ra[4], rb[4];
+                    e2m1x8_to_f16x2(wa[w], ra);
+                    e2m1x8_to_f16x2(wb[w], rb);
+                    const uint32_t sa = sc[w >> 1], sb = sc[2 + (w >> 1)];
+                    // word w holds k-steps 2w (bytes 0, 1) and 2w + 1 (bytes 2, 3)
+                    mma16816(sacc, hmul2(ra[0], sa), hmul2(rb[0], sb), hmul2(ra[1], sa), hmul2(rb[1], sb),
+                             qb[4 * w], qb[4 * w + 1]);
+                    mma16816(sacc, hmul2(ra[2], sa), hmul2(rb[2], sb), hmul2(ra[3], sa), hmul2(rb[3], sb),
+                             qb[4 * w + 2], qb[4 * w + 3]);
+                }
+            }
+            // hi + lo columns -> full scores of heads ha, hb for tokens g, g + 8
+            float s0 = sacc[0] + __shfl_xor_sync(kFull, sacc[0], 2);
+            float s1 = sacc[1] + __shfl_xor_sync(kFull, sacc[1], 2);
+            float s2 = sacc[2] + __shfl_xor_sync(kFull, sacc[2], 2);
+            float s3 = sacc[3] + __shfl_xor_sync(kFull, sacc[3], 2);
+            if (nvalid < kPage) {
+                if (g >= nvalid) s0 = s1 = -INFINITY;
+                if (g + 8 >= nvalid) s2 = s3 = -INFINITY;
+                // stale slots past the end may hold anything: zero their value scales
+                const uint32_t m01 = ((2 * c < nvalid) ? 0xFFFFu : 0u) | ((2 * c + 1 < nvalid) ? 0xFFFF0000u : 0u);
+                const uint32_t m89 = ((2 * c + 8 < nvalid) ? 0xFFFFu : 0u) | ((2 * c + 9 < nvalid) ? 0xFFFF0000u : 0u);
+                vs01 = e4m3x2_to_f16x2(vs01) & m01;
+                vs89 = e4m3x2_to_f16x2(vs89) & m89;
+            } else {
+                vs01 = e4m3x2_to_f16x2(vs01);
+                vs89 = e4m3x2_to_f16x2(vs89);
+            }
+            // ---- online softmax (exp2 domain)
+            float pm_a = fmaxf(s0, s2), pm_b = fmaxf(s1, s3);
+#pragma unroll
+            for (int x = 4; x < 32; x <<= 1) {
+                pm_a = fmaxf(pm_a, __shfl_xor_sync(kFull, pm_a, x));
+                pm_b = fmaxf(pm_b, __shfl_xor_sync(kFull, pm_b, x));
+            }
+            pm_a *= isg_a;
+            pm_b *= isg_b;
+            const float mn_a = fmaxf(m_a, pm_a), mn_b = fmaxf(m_b, pm_b);
+            if (__any_sync(kFull, (mn_a > m_a) || (mn_b > m_b))) {
+                const float al_a = fast_exp2(m_a - mn_a), al_b = fast_exp2(m_b - mn_b);
+                l_a *= al_a;
+                l_b *= al_b;
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    o[t][0] *= al_a; o[t][2] *= al_a;
+                    o[t][1] *= al_b; o[t][3] *= al_b;
+                }
+                m_a = mn_a;
+                m_b = mn_b;
+            }
+            // probabilities scaled by 2^15 for the fp16 operand
+            const float ca = 15.0f - m_a, cb = 15.0f - m_b;
+            const float p0 = fast_exp2(fmaf(s0, isg_a, ca)), p1 = fast_exp2(fmaf(s1, isg_b, cb));
+            const float p2 = fast_exp2(fmaf(s2, isg_a, ca)), p3 = fast_exp2(fmaf(s3, isg_b, cb));
+            l_a += p0 + p2;
+            l_b += p1 + p3;
+            // P as the B operand: [tokens] x [4 heads hi | 4 heads lo], via an 8x8 transpose
+            uint32_t m0 = pack_h2(p0, p1), m1 = pack_h2(p2, p3);
+            if (c >= 2) {
+                const float2 f0 = unpack_h2(m0), f1 = unpack_h2(m1);
+                m0 = pack_h2(p0 - f0.x, p1 - f0.y);
+                m1 = pack_h2(p2 - f1.x, p3 - f1.y);
+            }
+            const uint32_t pb0 = movmatrix_t(m0), pb1 = movmatrix_t(m1);
+            // ---- O^T += V^T P : rows = dims 16g + 2t (+1), k = tokens
+            const uint32_t w0[2] = {v0.x, v0.y}, w1[2] = {v1.x, v1.y};
+            const uint32_t w2[2] = {v2.x, v2.y}, w3[2] = {v3.x, v3.y};
+#pragma unroll
+            for (int wi = 0; wi < 2; ++wi) {
+                // pair tokens (2c, 2c+1) and (2c+8, 2c+9) nibble by nibble
+                const uint32_t L01 = (w0[wi] & 0x0F0F0F0Fu) | ((w1[wi] << 4) & 0xF0F0F0F0u);
+                const uint32_t H01 = ((w0[wi] >> 4) & 0x0F0F0F0Fu) | (w1[wi] & 0xF0F0F0F0u);
+                const uint32_t L89 = (w2[wi] & 0x0F0F0F0Fu) | ((w3[wi] << 4) & 0xF0F0F0F0u);
+                const uint32_t H89 = ((w2[wi] >> 4) & 0x0F0F0F0Fu) | (w3[wi] & 0xF0F0F0F0u);
+                uint32_t rl01[4], rh01[4], rl89[4], rh89[4];
+                e2m1x8_to_f16x2(L01, rl01);
+                e2m1x8_to_f16x2(H01, rh01);
+                e2m1x8_to_f16x2(L89, rl89);
+                e2m1x8_to_f16x2(H89, rh89);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    mma16816(o[4 * wi + j], hmul2(rl01[j], vs01), hmul2(rh01[j], vs01), hmul2(rl89[j], vs89),
+                             hmul2(rh89[j], vs89), pb0, pb1);
+            }
+        }
+    }
+
+    __syncthreads();
+    const bool timed_out = s_flags != 0;
+    if (timed_out && threadIdx.x == 32 * Hkv) {
+        // drain: wait (bounded) for every copy still in flight before exiting
+        const int issued = s_issued;
+        for (int st = 0; st < kStages && st < issued; ++st) {
+            const int last = st + ((issued - 1 - st) / kStages) * kStages;
+            (void)mbar_wait(&full[st], (last / kStages) & 1);
+        }
+        set_status(a.status, KVQ_DEV_TIMEOUT);
+    }
+    if (warp >= Hkv) return;
+
+    // ------------------------------------------------------------------ epilogue
+    const bool dead = poison || timed_out;
+#pragma unroll
+    for (int x = 4; x < 32; x <<= 1) {
+        l_a += __shfl_xor_sync(kFull, l_a, x);
+        l_b += __shfl_xor_sync(kFull, l_b, x);
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) o[t][k] += __shfl_xor_sync(kFull, o[t][k], 2);
+    // lane (g, c) writes dims 16g..16g+15 of one head: c < 2 -> head 2c, else head 2(c-2)+1
+    const int h = warp;
+    const bool first = c < 2;
+    const int head = first ? 2 * c : 2 * (c - 2) + 1;
+    if (head >= a.G) return;
+    float r[16];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+        r[2 * t] = first ? o[t][0] : o[t][1];
+        r[2 * t + 1] = first ? o[t][2] : o[t][3];
+    }
+    const float l = first ? l_a : l_b;
+    const float m = first ? m_a : m_b;
+    const int hq = h * a.G + head;
+    if (a.splits == 1) {
+        const float sc = (dead || l == 0.0f) ? 0.0f : __ldg(a.gv + li) / l;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) r[k] *= sc;
+        store16(reinterpret_cast<TO*>(a.out) + (((size_t)li * a.batch + b) * a.Hq + hq) * kD + 16 * g, r);
+    } else {
+        float* part = a.partials + ((((size_t)li * a.batch + b) * a.Hq + hq) * a.splits + split) * kPartialStride;
+        if (g == 0) {
+            part[0] = dead ? INFINITY : m;
+            part[1] = l;
+        }
+        store16(part + 4 + 16 * g, r);
+    }
+}
+
+// ------------------------------------------------------------------ launcher
+size_t decode_tc_smem(int Hkv) { return (size_t)kStages * Hkv * kTile + 2 * kStages * sizeof(uint64_t); }
+
+template <typename TQ, typename TO>
+static cudaError_t launch_one(const AttnArgs& a, dim3 grid, cudaStream_t st) {
+    const size_t smem = decode_tc_smem(a.Hkv);
+    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<TQ, TO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    decode_tc_kernel<TQ, TO><<<grid, 32 * (a.Hkv + 1), smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_tc(const AttnArgs& a, int nlayers, bool q_bf16, bool out_bf16, cudaStream_t st) {
+    dim3 grid(a.splits, a.batch, nlayers);
+    if (q_bf16 && out_bf16) return launch_one<__nv_bfloat16, __nv_bfloat16>(a, grid, st);
+    if (q_bf16) return launch_one<__nv_bfloat16, float>(a, grid, st);
+    if (out_bf16) return launch_one<float, __nv_bfloat16>(a, grid, st);
+    return launch_one<float, float>(a, grid, st);
+}
+
+}  // namespace kvq

@@ -31,7 +31,8 @@
  *     offending unit and ORs a KVQ_DEV_* bit into `*dev_status`, an int32 in
  *     device memory that the caller zeroes and reads back.  dev_status may be
  *     NULL, in which case such faults are skipped silently.
- *   - head_dim must be 128 and page_size 16 (KVQ_EUNSUPPORTED otherwise).
+ *   - head_dim must be 128, page_size 16, num_kv_heads <= 8 and the GQA
+ *     group num_q_heads / num_kv_heads <= 4 (KVQ_EUNSUPPORTED otherwise).
  *   - dtype arguments take KVQ_F32 or KVQ_BF16.
  *
  * Cache layout (owned by the caller, `kvq_page_bytes` bytes per page and
@@ -82,8 +83,8 @@ enum { KVQ_F32 = 0, KVQ_BF16 = 1 };
 
 typedef struct {
     int32_t num_layers;     /* L                                           */
-    int32_t num_q_heads;    /* Hq, a multiple of num_kv_heads              */
-    int32_t num_kv_heads;   /* Hkv, 1..16                                   */
+    int32_t num_q_heads;    /* Hq = G * Hkv with GQA group G in 1..4        */
+    int32_t num_kv_heads;   /* Hkv, 1..8 (even when use_hadamard)           */
     int32_t head_dim;       /* must be 128                                  */
     int32_t page_size;      /* must be 16                                   */
     int32_t use_hadamard;   /* 1: keys rotated by normalised Hadamard-128   */
