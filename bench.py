@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--layers", type=int, default=36,
+                    help="layers of the ragged workload (36; fewer only for profiling captures)")
     return ap.parse_args()
 
 
@@ -149,9 +151,10 @@ def ncu_traffic(kernel_file: str):
 class Ragged:
     """Device-resident ragged decode workload (one replica)."""
 
-    def __init__(self, kvq, synth):
+    def __init__(self, kvq, synth, layers=36):
         self.kvq = kvq
-        w = synth.WORKLOADS["ragged"]
+        import dataclasses
+        w = dataclasses.replace(synth.WORKLOADS["ragged"], num_layers=layers)
         self.w = w
         L, B, S = w.num_layers, w.batch, w.decode_steps
         self.L, self.B, self.S = L, B, S
@@ -235,34 +238,66 @@ def time_device(wl: Ragged, warmup: int, steps: int, world: int):
 
 
 def time_e2e(wl: Ragged, steps: int, world: int):
-    """Same steps through the public API from pinned host buffers, copies inside."""
+    """Same steps through the public API from pinned host buffers, copies inside.
+
+    Every step copies its own query, new K/V and slots in and its output out.
+    The copies run on a second stream into double-buffered device buffers, so
+    step i+1's inputs move while step i computes (as a serving loop would).
+    """
     st = torch.cuda.current_stream()
+    cp = torch.cuda.Stream()
     S = wl.S
-    hq = wl.q[:min(S, steps)].cpu().pin_memory()
-    hk = wl.k_new[:min(S, steps)].cpu().pin_memory()
-    hv = wl.v_new[:min(S, steps)].cpu().pin_memory()
+    n_host = min(S, steps)
+    hq = wl.q[:n_host].cpu().pin_memory()
+    hk = wl.k_new[:n_host].cpu().pin_memory()
+    hv = wl.v_new[:n_host].cpu().pin_memory()
     hslots = wl.slots.cpu().pin_memory()
     hlens = wl.seq_lens.cpu().pin_memory()
-    hout = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
-    dq, dk, dv = torch.empty_like(wl.q[0]), torch.empty_like(wl.k_new[0]), torch.empty_like(wl.v_new[0])
-    dslots, dlens = torch.empty_like(wl.slots[0]), torch.empty_like(wl.seq_lens[0])
+    hout = [torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory() for _ in range(2)]
+    dq = [torch.empty_like(wl.q[0]) for _ in range(2)]
+    dk = [torch.empty_like(wl.k_new[0]) for _ in range(2)]
+    dv = [torch.empty_like(wl.v_new[0]) for _ in range(2)]
+    dslots = [torch.empty_like(wl.slots[0]) for _ in range(2)]
+    dlens = [torch.empty_like(wl.seq_lens[0]) for _ in range(2)]
+    dout = [torch.empty_like(wl.out) for _ in range(2)]
     h2d = hq[0].numel() * 2 + hk[0].numel() * 2 * 2 + hslots[0].numel() * 8 + hlens[0].numel() * 4
-    d2h = hout.numel() * 2
+    d2h = hout[0].numel() * 2
+    ready = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    freed = [torch.cuda.Event() for _ in range(2)]
     torch.cuda.synchronize()
     barrier(world)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(st)
+    cp.wait_stream(st)
+
+    def h2d_step(i):
+        j, s = i % 2, i % n_host
+        with torch.cuda.stream(cp):
+            if i >= 2:
+                cp.wait_event(freed[j])
+            dq[j].copy_(hq[s], non_blocking=True)
+            dk[j].copy_(hk[s], non_blocking=True)
+            dv[j].copy_(hv[s], non_blocking=True)
+            dslots[j].copy_(hslots[s], non_blocking=True)
+            dlens[j].copy_(hlens[s], non_blocking=True)
+            ready[j].record(cp)
+
+    h2d_step(0)
     for i in range(steps):
-        s = i % hq.shape[0]
-        dq.copy_(hq[s], non_blocking=True)
-        dk.copy_(hk[s], non_blocking=True)
-        dv.copy_(hv[s], non_blocking=True)
-        dslots.copy_(hslots[s], non_blocking=True)
-        dlens.copy_(hlens[s], non_blocking=True)
-        wl.kvq.quantize_append(wl.shape, wl.calib, wl.cache, dk, dv, dslots)
-        wl.kvq.decode_attention(wl.shape, wl.calib, wl.cache, dq, wl.page_table_dev, dlens, out=wl.out,
+        j = i % 2
+        if i + 1 < steps:
+            h2d_step(i + 1)
+        st.wait_event(ready[j])
+        wl.kvq.quantize_append(wl.shape, wl.calib, wl.cache, dk[j], dv[j], dslots[j])
+        wl.kvq.decode_attention(wl.shape, wl.calib, wl.cache, dq[j], wl.page_table_dev, dlens[j], out=dout[j],
                                 workspace=wl.ws)
-        hout.copy_(wl.out, non_blocking=True)
+        freed[j].record(st)
+        done[j].record(st)
+        with torch.cuda.stream(cp):
+            cp.wait_event(done[j])
+            hout[j].copy_(dout[j], non_blocking=True)
+    st.wait_stream(cp)
     t1.record(st)
     torch.cuda.synchronize()
     barrier(world)
@@ -316,9 +351,10 @@ def cores():
 
 # ------------------------------------------------------------------ main
 def config_block(wl=None):
-    return {"workload": "ragged decode: 36 layers, 32 q / 8 kv heads, head_dim 128, batch 64, "
+    layers = wl.L if wl is not None else 36
+    return {"workload": f"ragged decode: {layers} layers, 32 q / 8 kv heads, head_dim 128, batch 64, "
                         "lengths U[1024,8192], 16-token pages in shuffled order, 64 append+decode steps cycled",
-            "batch": 64, "layers": 36, "kv_cache": "nvfp4 (e2m1 codes, e4m3 per-16 scales, fp32 tensor scale)",
+            "batch": 64, "layers": layers, "kv_cache": "nvfp4 (e2m1 codes, e4m3 per-16 scales, fp32 tensor scale)",
             "l2": "inputs larger than L2 (about 12.4 GB of cache read per step)",
             "parallelism": "replicas (independent sequences per GPU)"}
 
@@ -352,7 +388,7 @@ def main():
     import synth
     assert torch.cuda.is_available(), "bench needs a CUDA device"
     t_setup = time.time()
-    wl = Ragged(kvq, synth)
+    wl = Ragged(kvq, synth, args.layers)
     sys.stderr.write(f"[bench] setup {time.time() - t_setup:.1f} s, {wl.num_pages} pages, "
                      f"cache {wl.cache.data.numel() / 1e9:.2f} GB\n")
     clock = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
