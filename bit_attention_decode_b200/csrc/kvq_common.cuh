@@ -94,17 +94,12 @@ __device__ __forceinline__ void load16(const __nv_bfloat16* p, float* x) {
 }
 
 // ---------------------------------------------------------------- key transform
-// One thread holds block `blk` (16 elements) of a 128-element key row; the 8
-// threads of a row are 8 consecutive lanes (lane & 7 == blk).  Applies the
-// smoothing multiply y = k * inv_s and, with `hadamard`, the normalised
-// Hadamard-128: butterflies h = 1, 2, 4, 8 inside the thread, h = 16, 32, 64
-// across lanes, then one multiply by fp32(1/sqrt(128)).  Every operation is a
-// single fp32 rounding, in the order the stages are listed.
-__device__ __forceinline__ void transform_key_block(float* y, const float* __restrict__ inv_s_row,
-                                                    int blk, bool hadamard) {
-#pragma unroll
-    for (int i = 0; i < kBlk; ++i) y[i] = __fmul_rn(y[i], __ldg(inv_s_row + blk * kBlk + i));
-    if (!hadamard) return;
+// Normalised Hadamard-128 of a key row held as 8 blocks of 16 in 8
+// consecutive lanes (lane & 7 == blk): butterflies h = 1, 2, 4, 8 inside the
+// thread, h = 16, 32, 64 across lanes, then one multiply by fp32(1/sqrt(128)).
+// Every operation is a single fp32 rounding, in the order listed; every lane
+// of the warp must call it.
+__device__ __forceinline__ void hadamard_block(float* y, int blk) {
 #pragma unroll
     for (int h = 1; h < kBlk; h <<= 1) {
 #pragma unroll
@@ -127,6 +122,15 @@ __device__ __forceinline__ void transform_key_block(float* y, const float* __res
     }
 #pragma unroll
     for (int i = 0; i < kBlk; ++i) y[i] = __fmul_rn(y[i], kInvSqrt128);
+}
+
+// Key pre-transform of one block: smoothing multiply y = k * inv_s, then the
+// optional rotation (see hadamard_block).
+__device__ __forceinline__ void transform_key_block(float* y, const float* __restrict__ inv_s_row,
+                                                    int blk, bool hadamard) {
+#pragma unroll
+    for (int i = 0; i < kBlk; ++i) y[i] = __fmul_rn(y[i], __ldg(inv_s_row + blk * kBlk + i));
+    if (hadamard) hadamard_block(y, blk);
 }
 
 __device__ __forceinline__ void set_status(int32_t* status, int32_t bits) {

@@ -103,57 +103,193 @@ __device__ __forceinline__ void quantize_block(const float* y, float g, float en
     codes = make_uint2(w[0], w[1]);
 }
 
-// grid (num_tokens, nlayers); block Hkv * 16 threads: threads [0, 8 Hkv) own
-// the 8 key blocks of each head, the rest the value blocks.
+// Bulk-copy staging of the inputs.  A work item is a chunk of `tc`
+// consecutive tokens of one layer: its key rows and value rows are two
+// contiguous ranges (tc x Hkv x 128 elements each), streamed into a ring of
+// kAppendStages shared-memory stages with cp.async.bulk and an mbarrier
+// transaction count.  Thread 0 keeps kAppendStages - 1 chunks in flight.
+// Quantisation then reads the stage: a token takes Hkv * 16 threads, threads
+// [0, 8 Hkv) owning the 8 key blocks of each head and the rest the value
+// blocks; a CTA of 256 threads works on 256 / (16 Hkv) tokens at a time.
+// With the rotation Hkv is even, so every warp lies inside one token and the
+// cross-lane butterflies stay uniform.
+constexpr int kAppendStages = 3;
+constexpr int kAppendStageBytes = 32768;   // key + value rows of one chunk
+constexpr unsigned long long kAppendWaitNs = 2000000000ull;
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ bool append_wait(uint64_t* bar, uint32_t parity) {
+    auto try_wait = [&]() {
+        uint32_t ok;
+        asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+                     : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+        return ok != 0;
+    };
+    if (try_wait()) return true;
+    unsigned long long t0;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    for (;;) {
+        for (int i = 0; i < 64; ++i)
+            if (try_wait()) return true;
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        if (t - t0 > kAppendWaitNs) return false;
+    }
+}
+
 template <typename T>
-__global__ void __launch_bounds__(256)
-append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* __restrict__ slots,
-              int num_tokens, int Hkv, const float* __restrict__ inv_s, const float* __restrict__ gk,
-              const float* __restrict__ gv, uint8_t* __restrict__ cache, int64_t layer_stride,
-              int num_pages, int hadamard, int32_t* __restrict__ status) {
-    const int tok = blockIdx.x, li = blockIdx.y;
-    const int64_t slot = __ldg(slots + tok);
-    if (slot < 0) return;  // padding token
-    if (slot >= (int64_t)num_pages * kPage) {
-        if (threadIdx.x == 0) set_status(status, KVQ_DEV_BAD_SLOT);
-        return;
+__device__ __forceinline__ void load16_smem(const T* p, float* x);
+template <>
+__device__ __forceinline__ void load16_smem<float>(const float* p, float* x) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float4 t = reinterpret_cast<const float4*>(p)[i];
+        x[4 * i] = t.x; x[4 * i + 1] = t.y; x[4 * i + 2] = t.z; x[4 * i + 3] = t.w;
     }
-    const int t = threadIdx.x;
-    const bool is_v = t >= Hkv * 8;
-    const int h = (t >> 3) % Hkv;
-    const int blk = t & 7;
-    const size_t src = (((size_t)li * num_tokens + tok) * Hkv + h) * kD + blk * kBlk;
-    float y[kBlk];
-    load16(is_v ? v + src : k + src, y);
-    const float* inv_row = inv_s + ((size_t)li * Hkv + h) * kD;
-    if (hadamard) {
-        // every lane joins the cross-lane butterflies (groups of 8 lanes never
-        // mix keys and values); value lanes discard the result
-        float z[kBlk];
+}
+template <>
+__device__ __forceinline__ void load16_smem<__nv_bfloat16>(const __nv_bfloat16* p, float* x) {
 #pragma unroll
-        for (int i = 0; i < kBlk; ++i) z[i] = y[i];
-        transform_key_block(z, inv_row, blk, true);
-        if (!is_v) {
+    for (int i = 0; i < 2; ++i) {
+        uint4 t = reinterpret_cast<const uint4*>(p)[i];
+        uint32_t w[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
-            for (int i = 0; i < kBlk; ++i) y[i] = z[i];
+        for (int j = 0; j < 4; ++j) {
+            x[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+            x[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
         }
-    } else if (!is_v) {
-        transform_key_block(y, inv_row, blk, false);
     }
-    const float g = is_v ? __ldg(gv + li) : __ldg(gk + li);
-    const float enc = __frcp_rn(__fmul_rn(6.0f, g));
-    uint2 codes;
-    uint32_t sf;
-    quantize_block(y, g, enc, codes, sf);
-    const int64_t page = slot >> 4;
-    const int off = (int)(slot & 15);
-    uint8_t* tile = cache + (size_t)li * layer_stride + ((size_t)page * Hkv + h) * kTile;
-    if (!is_v) {
-        *reinterpret_cast<uint2*>(tile + kKCodes + off * 64 + blk * 8) = codes;
-        tile[kKScales + off * 8 + blk] = (uint8_t)sf;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(288, 2)
+append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* __restrict__ slots,
+              int num_tokens, int nlayers, int Hkv, int tc, const float* __restrict__ inv_s,
+              const float* __restrict__ gk, const float* __restrict__ gv, uint8_t* __restrict__ cache,
+              int64_t layer_stride, int num_pages, int hadamard, int32_t* __restrict__ status) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ uint64_t full[kAppendStages], empty[kAppendStages];
+    __shared__ int s_timeout, s_issued;
+    const int row = Hkv * kD;                                  // elements per token row
+    const uint32_t half_stage = kAppendStageBytes / 2;         // key rows, then value rows
+    const int chunks = (num_tokens + tc - 1) / tc;
+    const long items = (long)chunks * nlayers;
+    const int mine = items > blockIdx.x ? (int)((items - 1 - blockIdx.x) / gridDim.x + 1) : 0;
+    const int workers = 8;                                     // warps 0..7; warp 8 streams the inputs
+    const int warp = threadIdx.x >> 5;
+
+    if (threadIdx.x == 0) {
+        s_timeout = 0;
+        s_issued = 0;
+        for (int i = 0; i < kAppendStages; ++i) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&full[i])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(&empty[i])), "r"(workers));
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (warp == workers) {
+        // ---------------------------------------------------------- producer
+        if ((threadIdx.x & 31) == 0) {
+            int j = 0;
+            for (; j < mine; ++j) {
+                const int st = j % kAppendStages;
+                if (j >= kAppendStages && !append_wait(&empty[st], ((j / kAppendStages) - 1) & 1)) {
+                    atomicOr(&s_timeout, 1);
+                    break;
+                }
+                const long it = blockIdx.x + (long)j * gridDim.x;
+                const int li = (int)(it / chunks), t0 = (int)(it % chunks) * tc;
+                const int n = min(tc, num_tokens - t0);
+                const uint32_t bytes = (uint32_t)n * row * sizeof(T);
+                uint8_t* dst = smem + st * kAppendStageBytes;
+                const size_t off = ((size_t)li * num_tokens + t0) * row;
+                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(&full[st])),
+                             "r"(2 * bytes) : "memory");
+                asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                             ::"r"(smem_addr(dst)), "l"(k + off), "r"(bytes), "r"(smem_addr(&full[st])) : "memory");
+                asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                             ::"r"(smem_addr(dst + half_stage)), "l"(v + off), "r"(bytes), "r"(smem_addr(&full[st]))
+                             : "memory");
+            }
+            s_issued = j;
+        }
     } else {
-        *reinterpret_cast<uint2*>(tile + kVCodes + off * 64 + blk * 8) = codes;
-        tile[kVScales + blk * 16 + off] = (uint8_t)sf;
+        // ---------------------------------------------------------- workers
+        // a token takes 8 Hkv threads, thread (h, blk) owning block blk of
+        // head h for both the key and the value row
+        const int per_tok = Hkv * 8;
+        const int tpc = (workers * 32) / per_tok;              // tokens side by side
+        const int t = threadIdx.x % per_tok, sub = threadIdx.x / per_tok;
+        const int h = t >> 3, blk = t & 7;
+        const bool active = sub < tpc;
+        for (int j = 0; j < mine; ++j) {
+            const long it = blockIdx.x + (long)j * gridDim.x;
+            const int li = (int)(it / chunks), t0 = (int)(it % chunks) * tc;
+            const int n = min(tc, num_tokens - t0);
+            // per-chunk constants, loaded before waiting for the inputs
+            float inv[kBlk];
+            const float4* ip = reinterpret_cast<const float4*>(inv_s + ((size_t)li * Hkv + h) * kD + blk * kBlk);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 q4 = __ldg(ip + i);
+                inv[4 * i] = q4.x; inv[4 * i + 1] = q4.y; inv[4 * i + 2] = q4.z; inv[4 * i + 3] = q4.w;
+            }
+            const float g_k = __ldg(gk + li), g_v = __ldg(gv + li);
+            const float enc_k = __frcp_rn(__fmul_rn(6.0f, g_k)), enc_v = __frcp_rn(__fmul_rn(6.0f, g_v));
+            uint8_t* layer_cache = cache + (size_t)li * layer_stride;
+            const int st = j % kAppendStages;
+            if (!append_wait(&full[st], (j / kAppendStages) & 1)) {
+                atomicOr(&s_timeout, 1);
+                break;
+            }
+            const T* stage = reinterpret_cast<const T*>(smem + st * kAppendStageBytes);
+            if (active) {
+                for (int tt = sub; tt < n; tt += tpc) {
+                    const int64_t slot = __ldg(slots + t0 + tt);
+                    const bool ok = slot >= 0 && slot < (int64_t)num_pages * kPage;
+                    if (slot >= (int64_t)num_pages * kPage && t == 0) set_status(status, KVQ_DEV_BAD_SLOT);
+                    float y[kBlk];
+                    const size_t e = (size_t)tt * row + h * kD + blk * kBlk;
+                    load16_smem<T>(stage + e, y);
+                    // key: smoothing multiply, then the optional rotation (every
+                    // lane of the warp joins its butterflies)
+#pragma unroll
+                    for (int i = 0; i < kBlk; ++i) y[i] = __fmul_rn(y[i], inv[i]);
+                    if (hadamard) hadamard_block(y, blk);
+                    uint2 codes;
+                    uint32_t sf;
+                    quantize_block(y, g_k, enc_k, codes, sf);
+                    const int64_t page = slot >> 4;
+                    const int off = (int)(slot & 15);
+                    uint8_t* tile = layer_cache + ((size_t)page * Hkv + h) * kTile;
+                    if (ok) {
+                        *reinterpret_cast<uint2*>(tile + kKCodes + off * 64 + blk * 8) = codes;
+                        tile[kKScales + off * 8 + blk] = (uint8_t)sf;
+                    }
+                    load16_smem<T>(stage + half_stage / sizeof(T) + e, y);
+                    quantize_block(y, g_v, enc_v, codes, sf);
+                    if (ok) {
+                        *reinterpret_cast<uint2*>(tile + kVCodes + off * 64 + blk * 8) = codes;
+                        tile[kVScales + blk * 16 + off] = (uint8_t)sf;
+                    }
+                }
+            }
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(
+                                                          smem_addr(&empty[st])) : "memory");
+        }
+    }
+    __syncthreads();
+    if (s_timeout && threadIdx.x == 32 * workers) {
+        // wait (bounded) for the copies still in flight before leaving
+        const int issued = s_issued;
+        for (int j = max(0, issued - kAppendStages); j < issued; ++j)
+            (void)append_wait(&full[j % kAppendStages], (j / kAppendStages) & 1);
+        set_status(status, KVQ_DEV_TIMEOUT);
     }
 }
 
@@ -207,14 +343,33 @@ kvq_status quantize_append(const kvq_shape& s, const kvq_calib& c, const kvq_cac
     const float* gk = c.k_gscale + layer0;
     const float* gv = c.v_gscale + layer0;
     uint8_t* base = cache.data + (size_t)layer0 * cache.layer_stride_bytes;
-    dim3 grid(num_tokens, nlayers);
+    // tokens per chunk: key rows of one chunk fill half a stage
+    const int row_bytes = H * kD * (dtype == KVQ_F32 ? 4 : 2);
+    const int tc = max(1, (kAppendStageBytes / 2) / row_bytes);
+    const long items = (long)((num_tokens + tc - 1) / tc) * nlayers;
+    const int threads = 288;
+    const size_t smem = (size_t)kAppendStages * kAppendStageBytes;
+    int dev = 0, sms = 148, per_sm = 2;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e;
+    if (dtype == KVQ_F32) {
+        e = cudaFuncSetAttribute(append_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, append_kernel<float>, threads, smem);
+    } else {
+        e = cudaFuncSetAttribute(append_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, append_kernel<__nv_bfloat16>, threads, smem);
+    }
+    if (e != cudaSuccess) return KVQ_ECUDA;
+    const long wave = (long)sms * max(per_sm, 1);
+    const int grid = (int)(items < wave ? items : wave);
     if (dtype == KVQ_F32)
-        append_kernel<float><<<grid, H * 16, 0, st>>>((const float*)k, (const float*)v, slots, num_tokens, H,
-                                                     inv_s, gk, gv, base, cache.layer_stride_bytes,
-                                                     cache.num_pages, s.use_hadamard, status);
+        append_kernel<float><<<grid, threads, smem, st>>>((const float*)k, (const float*)v, slots, num_tokens,
+                                                        nlayers, H, tc, inv_s, gk, gv, base, cache.layer_stride_bytes,
+                                                        cache.num_pages, s.use_hadamard, status);
     else
-        append_kernel<__nv_bfloat16><<<grid, H * 16, 0, st>>>(
-            (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, slots, num_tokens, H, inv_s, gk, gv, base,
+        append_kernel<__nv_bfloat16><<<grid, threads, smem, st>>>(
+            (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, slots, num_tokens, nlayers, H, tc, inv_s, gk, gv, base,
             cache.layer_stride_bytes, cache.num_pages, s.use_hadamard, status);
     return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ECUDA;
 }
