@@ -86,35 +86,63 @@ class Problem:
 
 
 def build_problem(kvq, w: synth.Workload, lens, layers=None, extra_tokens: int = 0, shuffle: bool = True,
-                  keep_host=True, device="cuda", gen_device="cpu"):
-    """Calibrate, then append each sequence's first lens[b] tokens, one layer at a time."""
+                  keep_host=True, device="cuda", gen_device="cpu", keep=None, all_layers_one_call=False,
+                  keep_tails=False):
+    """Calibrate, then append each sequence's first lens[b] tokens.
+
+    keep:      optional set of (layer index, sequence) whose host copies are kept
+               (all when None and keep_host).
+    all_layers_one_call: append every layer with one quantize_append call
+               (K/V [nl][T][Hkv][D]) instead of one call per layer.
+    keep_tails: also return the extra_tokens tail of every sequence on the
+               device, as tails_k/v [extra][nl][B][Hkv][D].
+    """
     layers = list(range(w.num_layers)) if layers is None else list(layers)
     lens = torch.as_tensor(lens, dtype=torch.int32)
-    nl = len(layers)
+    nl, B = len(layers), len(lens)
     shape = kvq.Shape(num_layers=nl, num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads,
                       use_hadamard=w.hadamard)
-    kc = torch.stack([synth.calibration_windows(w, l, gen_device)[0] for l in layers])
-    vc = torch.stack([synth.calibration_windows(w, l, gen_device)[1] for l in layers])
+    wins = [synth.calibration_windows(w, l, gen_device) for l in layers]
+    kc = torch.stack([x[0] for x in wins])
+    vc = torch.stack([x[1] for x in wins])
+    del wins
     calib = kvq.calibrate_smoothing(shape, kc.to(device).contiguous(), vc.to(device).contiguous())
     page_table, num_pages = synth.build_page_table(w, lens + extra_tokens, shuffle=shuffle)
     cache = kvq.new_cache(shape, num_pages, device)
     seqs = {}
+    tails = None
+    if keep_tails and extra_tokens:
+        tails = (torch.empty(extra_tokens, nl, B, w.num_kv_heads, w.head_dim, dtype=w.dtype, device=device),
+                 torch.empty(extra_tokens, nl, B, w.num_kv_heads, w.head_dim, dtype=w.dtype, device=device))
+    slots = torch.cat([synth.slot_mapping(page_table, torch.full((int(n),), b), torch.arange(int(n)))
+                       for b, n in enumerate(lens.tolist())]).to(device)
+    layer_k, layer_v = [], []
     for li, l in enumerate(layers):
-        ks, vs, slots = [], [], []
-        for b in range(len(lens)):
+        ks, vs = [], []
+        for b in range(B):
             n = int(lens[b])
             k, v = synth.sequence_kv(w, l, b, n + extra_tokens, gen_device)
-            if keep_host:
+            if keep_host and (keep is None or (li, b) in keep):
                 seqs[(li, b)] = (k.float().cpu().numpy(), v.float().cpu().numpy())
+            if tails is not None:
+                tails[0][:, li, b] = k[n:].to(device)
+                tails[1][:, li, b] = v[n:].to(device)
             ks.append(k[:n])
             vs.append(v[:n])
-            slots.append(synth.slot_mapping(page_table, torch.full((n,), b), torch.arange(n)))
         k = torch.cat(ks).to(device)
         v = torch.cat(vs).to(device)
-        sm = torch.cat(slots).to(device)
-        kvq.quantize_append(shape, calib, cache, k.contiguous(), v.contiguous(), sm, layer0=li)
-    return Problem(w, layers, lens, page_table, num_pages, shape, calib, cache,
-                   kc.float().cpu().numpy(), vc.float().cpu().numpy(), seqs)
+        del ks, vs
+        if all_layers_one_call:
+            layer_k.append(k)
+            layer_v.append(v)
+        else:
+            kvq.quantize_append(shape, calib, cache, k.contiguous(), v.contiguous(), slots, layer0=li)
+    if all_layers_one_call:
+        kvq.quantize_append(shape, calib, cache, torch.stack(layer_k), torch.stack(layer_v), slots, layer0=0)
+    p = Problem(w, layers, lens, page_table, num_pages, shape, calib, cache,
+                kc.float().cpu().numpy(), vc.float().cpu().numpy(), seqs)
+    p.tails = tails
+    return p
 
 
 def oracle_calibration(p: Problem):
