@@ -30,5 +30,7 @@ struct AttnArgs {
 // tensor-core split-K decode (kvq_decode_tc.cu)
 cudaError_t launch_decode_tc(const AttnArgs& a, int nlayers, bool q_bf16, bool out_bf16, cudaStream_t st);
 size_t decode_tc_smem(int Hkv);
+// tensor-core (tcgen05) chunked causal prefill (kvq_prefill_tc.cu)
+cudaError_t launch_prefill_tc(const AttnArgs& a, int nlayers, bool q_bf16, bool out_bf16, cudaStream_t st);
 
 }  // namespace kvq

@@ -1,0 +1,664 @@
+// kvq_prefill_tc.cu -- chunked causal prefill over the packed NVFP4 cache on
+// the 5th-generation tensor cores (tcgen05.mma, accumulators in TMEM).
+//
+// The chunk's own keys and values are appended to the cache first; query i
+// of sequence b (absolute position q_start + i) then attends cached
+// positions j <= q_start + i ("chunked causal prefill", with the smoothing
+// and rotation folded into the query as in "NVFP4 attention cache on W4A4
+// Qwen3-8B" (rstation.ai), observation 2).
+//
+// One CTA: one layer, one sequence, one kv head, a tile of 32 query tokens.
+// The tile's 128 MMA rows are the G <= 4 query heads of the kv head times
+// the 32 tokens (row = head * 32 + token), so each dequantised key/value
+// block feeds 4 heads at once.  Per 64-token key block (4 pages):
+//   dequant warps (4): bulk-copy the 4 packed page tiles into a staging
+//     ring, dequantise to fp16 (E2M1 x E4M3 is exact in fp16) into a K tile
+//     (K-major) and a V tile (MN-major), both in the 128-byte-swizzled
+//     canonical layouts the MMA reads; rows past the sequence are zeros.
+//   MMA warp (1 elected thread): S = Q_hi K^T + Q_lo K^T (M=128, N=64, K=16
+//     steps; the query is split into fp16 hi + lo parts so its rounding does
+//     not reach the scores) into one of two TMEM score buffers, then
+//     O += P V (M=128, N=128) into the TMEM output accumulator.
+//   softmax warps (4, one TMEM lane = one row per thread): causal mask,
+//     running max with lazy rescaling (the output in TMEM is rescaled only
+//     when the max grows by more than 2^8), probabilities rounded once to
+//     fp16 into a swizzled P tile.
+// All hand-offs are mbarriers with bounded waits; a wait that runs out sets
+// KVQ_DEV_TIMEOUT, the CTA writes zeros and frees its TMEM.
+#include "kvq_attn.cuh"
+#include "kvq_common.cuh"
+#include "kvq_internal.h"
+
+namespace kvq {
+namespace {
+
+constexpr int kRows = 128;          // MMA M: 4 heads x 32 query tokens
+constexpr int kQTok = 32;           // query tokens per tile
+constexpr int kBlkTok = 64;         // key tokens per block (4 pages)
+constexpr int kStageN = 3;          // packed-page staging stages
+constexpr uint32_t kTmemCols = 256; // O [0,128), S0 [128,192), S1 [192,256)
+constexpr unsigned long long kWaitNs = 2000000000ull;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+// shared memory map (offsets from a 1024-aligned base)
+constexpr int kQBytes = kRows * kD * 2;           // 32 KB per fp16 query tile (hi or lo)
+constexpr int kKBytes = kBlkTok * kD * 2;         // 16 KB per fp16 key tile
+constexpr int kVBytes = kBlkTok * kD * 2;         // 16 KB per fp16 value tile
+constexpr int kPBytes = kRows * kBlkTok * 2;      // 16 KB per fp16 probability tile
+constexpr int kStageBytes = 4 * kTile;            // 4 packed page tiles of one head
+constexpr int kOffQhi = 0;
+constexpr int kOffQlo = kOffQhi + kQBytes;
+constexpr int kOffK = kOffQlo + kQBytes;          // 2 buffers
+constexpr int kOffV = kOffK + 2 * kKBytes;        // 2 buffers
+constexpr int kOffP = kOffV + 2 * kVBytes;        // 2 buffers
+constexpr int kOffStage = kOffP + 2 * kPBytes;    // kStageN stages
+constexpr int kSmemBytes = kOffStage + kStageN * kStageBytes;
+constexpr int kSmemAlloc = kSmemBytes + 1024;     // room to align the base
+
+enum { kWarpsSoftmax = 4, kWarpsDequant = 4 };
+constexpr int kMmaWarp = kWarpsSoftmax + kWarpsDequant;   // warp 8
+constexpr int kThreads = 32 * (kMmaWarp + 1);
+
+// ------------------------------------------------------------------ primitives
+__device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void bar_init(uint64_t* b, uint32_t n) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(n));
+}
+__device__ __forceinline__ void bar_arrive(uint64_t* b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+__device__ __forceinline__ void bar_expect(uint64_t* b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool bar_try(uint64_t* b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+                 : "=r"(ok) : "r"(su32(b)), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ unsigned long long now_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// bounded wait; false when it ran out
+__device__ __forceinline__ bool bar_wait(uint64_t* b, uint32_t parity) {
+    if (bar_try(b, parity)) return true;
+    const unsigned long long t0 = now_ns();
+    for (;;) {
+        for (int i = 0; i < 64; ++i)
+            if (bar_try(b, parity)) return true;
+        if (now_ns() - t0 > kWaitNs) return false;
+    }
+}
+// every lane of the warp waits; the outcome is made uniform across the warp
+__device__ __forceinline__ bool bar_wait_warp(uint64_t* b, uint32_t parity) {
+    return __all_sync(0xFFFFFFFFu, bar_wait(b, parity));
+}
+__device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, uint64_t* b) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(su32(dst)), "l"(src), "r"(bytes), "r"(su32(b)) : "memory");
+}
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 128-byte-swizzle smem matrix descriptor (sm_100 UMMA): start address,
+// leading / stride byte offsets, descriptor version 1, layout SWIZZLE_128B.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+// kind::f16 instruction descriptor: fp16 A and B, fp32 accumulate
+__host__ __device__ constexpr uint32_t f16_idesc(int M, int N, bool b_mn_major) {
+    return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile("{ .reg .pred p; setp.ne.b32 p, %4, 0;\n"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }"
+                 ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* b) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(b))
+                 : "memory");
+}
+// 32 consecutive fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+                   "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+                   "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+                   "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+    uint32_t r[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+                 "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                   "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+                   "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]),
+                   "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]),
+                   "r"(r[31])
+                 : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t h2(float lo, float hi) {
+    __half2 r = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t hmul2u(uint32_t a, uint32_t b) {
+    __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ void e2m1x8(uint32_t w, uint32_t* r) {
+    asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %4;\n"
+        "  cvt.rn.f16x2.e2m1x2 %0, b0; cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+        "  cvt.rn.f16x2.e2m1x2 %2, b2; cvt.rn.f16x2.e2m1x2 %3, b3; }"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(w));
+}
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// byte offset of 16-byte chunk `ch` of row `row` in a 128-byte-swizzled tile
+// of 128-byte rows (8-row atoms of 1024 bytes)
+__device__ __forceinline__ uint32_t sw128(int row, int ch) {
+    return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((ch ^ (row & 7)) << 4));
+}
+__device__ __forceinline__ void sts128(uint8_t* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    *reinterpret_cast<uint4*>(p) = make_uint4(a, b, c, d);
+}
+
+template <typename T>
+__device__ __forceinline__ void load_row128(const T* p, float* x);
+template <>
+__device__ __forceinline__ void load_row128<float>(const float* p, float* x) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        float4 t = __ldg(reinterpret_cast<const float4*>(p) + i);
+        x[4 * i] = t.x; x[4 * i + 1] = t.y; x[4 * i + 2] = t.z; x[4 * i + 3] = t.w;
+    }
+}
+template <>
+__device__ __forceinline__ void load_row128<__nv_bfloat16>(const __nv_bfloat16* p, float* x) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        uint4 t = __ldg(reinterpret_cast<const uint4*>(p) + i);
+        uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            x[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+            x[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+    }
+}
+
+struct PrefillBars {
+    uint64_t q_ready;                 // softmax warps wrote the query tiles (count 4)
+    uint64_t stage_full[kStageN];     // packed pages landed (tx bytes)
+    uint64_t stage_empty[kStageN];    // dequant warps read the stage (count 4)
+    uint64_t kv_full[2];              // K/V tile j%2 written (count 4)
+    uint64_t s_full[2];               // QK(j) done (commit)
+    uint64_t p_full[2];               // P tile j%2 written, O rescaled (count 4)
+    uint64_t pv_done[2];              // PV(j) done (commit)
+    uint64_t drain;                   // last commit before TMEM is freed after a timeout
+    uint32_t tmem_base;
+    int flags;                        // 1: a bounded wait ran out
+    int issued;                       // packed-page stages issued
+};
+
+// ------------------------------------------------------------------ kernel
+// grid (q tiles, batch * Hkv, nlayers), block 288.
+template <typename TQ, typename TO>
+__global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ PrefillBars bars;
+
+    const int tile = blockIdx.x, b = blockIdx.y / a.Hkv, h = blockIdx.y % a.Hkv, li = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int len = __ldg(a.seq_lens + b);
+    const int qs = __ldg(a.q_start + b);
+    const int q0 = tile * kQTok;
+    const int qn = min(kQTok, a.q_len - q0);                 // query tokens in this tile
+    const bool bad_len = len < 0 || len > a.max_pages * kPage;
+    // keys needed by the tile: positions < min(len, q_start + q0 + qn)
+    int kv_end = bad_len ? 0 : min(len, qs + q0 + qn);
+    if (kv_end < 0) kv_end = 0;
+    const int nb = (kv_end + kBlkTok - 1) / kBlkTok;          // 64-token blocks
+    const int npg = (kv_end + kPage - 1) / kPage;             // pages touched
+    const int32_t* pt = a.page_table + (size_t)b * a.max_pages;
+    const uint8_t* layer_base = a.cache + (size_t)li * a.layer_stride;
+
+    if (threadIdx.x == 0) {
+        bars.flags = 0;
+        bars.issued = 0;
+        bar_init(&bars.q_ready, kWarpsSoftmax);
+        for (int i = 0; i < kStageN; ++i) {
+            bar_init(&bars.stage_full[i], 1);
+            bar_init(&bars.stage_empty[i], kWarpsDequant);
+        }
+        for (int i = 0; i < 2; ++i) {
+            bar_init(&bars.kv_full[i], kWarpsDequant);
+            bar_init(&bars.s_full[i], 1);
+            bar_init(&bars.p_full[i], kWarpsSoftmax);
+            bar_init(&bars.pv_done[i], 1);
+        }
+        bar_init(&bars.drain, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    int badp = 0;
+    for (int i = threadIdx.x; i < npg; i += blockDim.x) {
+        const int pg = __ldg(pt + i);
+        badp |= (pg < 0 || pg >= a.num_pages);
+    }
+    badp = __syncthreads_or(badp);
+    if (threadIdx.x == 0) {
+        if (bad_len && tile == 0 && h == 0) set_status(a.status, KVQ_DEV_BAD_LEN);
+        if (badp) set_status(a.status, KVQ_DEV_BAD_PAGE);
+    }
+    const bool poison = bad_len || badp;
+
+    // TMEM: one warp allocates 256 columns for the CTA
+    if (warp == kMmaWarp) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&bars.tmem_base)),
+                     "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars.tmem_base;
+    const uint32_t tO = tmem, tS0 = tmem + 128;
+
+    // per-row state of the softmax warps, kept to the epilogue
+    float m_run = -INFINITY, l_run = 0.0f, isig = 1.0f;
+    bool row_ok = false;
+
+    if (!poison && nb > 0) {
+        if (warp < kWarpsSoftmax) {
+            // ------------------------------------------------------ softmax warps
+            const int r = threadIdx.x;                 // TMEM lane = MMA row
+            const int head = r >> 5, tok = r & 31;     // row = head * 32 + token
+            const int qi = q0 + tok;
+            row_ok = head < a.G && tok < qn;
+            const int qpos = qs + qi;                  // absolute position of this query
+            // query prologue: q~ = q * s (+ rotation) * g_K log2(e) / sqrt(128),
+            // per-row power-of-two normalisation, fp16 hi + lo tiles
+            {
+                float x[kD];
+                if (row_ok) {
+                    const TQ* src = reinterpret_cast<const TQ*>(a.q) +
+                                    ((((size_t)li * a.batch + b) * a.q_len + qi) * a.Hq + h * a.G + head) * kD;
+                    load_row128<TQ>(src, x);
+                    const float* srow = a.smooth + ((size_t)li * a.Hkv + h) * kD;
+#pragma unroll
+                    for (int i = 0; i < kD; ++i) x[i] *= __ldg(srow + i);
+                    float scale = __ldg(a.gk + li) * kLog2e * kInvSqrt128;
+                    if (a.hadamard) {
+#pragma unroll
+                        for (int hh = 1; hh < kD; hh <<= 1)
+#pragma unroll
+                            for (int j = 0; j < kD; ++j)
+                                if ((j & hh) == 0) {
+                                    const float u = x[j], v = x[j + hh];
+                                    x[j] = u + v;
+                                    x[j + hh] = u - v;
+                                }
+                        scale *= kInvSqrt128;
+                    }
+#pragma unroll
+                    for (int i = 0; i < kD; ++i) x[i] *= scale;
+                } else {
+#pragma unroll
+                    for (int i = 0; i < kD; ++i) x[i] = 0.0f;
+                }
+                float mx = 0.0f;
+#pragma unroll
+                for (int i = 0; i < kD; ++i) mx = fmaxf(mx, fabsf(x[i]));
+                int ex = 0;
+                if (mx > 0.0f) {
+                    frexpf(mx, &ex);
+                    ex = max(ex - 1, -100);
+                }
+                const float sig = ldexpf(1.0f, 14 - ex);
+                isig = ldexpf(1.0f, ex - 14);
+                // K-major 128B-swizzled tiles: dims 0..63 in atom plane 0, 64..127 in plane 1
+#pragma unroll
+                for (int ch = 0; ch < 16; ++ch) {
+                    uint32_t hi[4], lo[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float u = x[8 * ch + 2 * e] * sig, v = x[8 * ch + 2 * e + 1] * sig;
+                        hi[e] = h2(u, v);
+                        const float2 f = __half22float2(*reinterpret_cast<__half2*>(&hi[e]));
+                        lo[e] = h2(u - f.x, v - f.y);
+                    }
+                    const uint32_t off = (ch >> 3) * (kRows * 128) + sw128(r, ch & 7);
+                    sts128(smem + kOffQhi + off, hi[0], hi[1], hi[2], hi[3]);
+                    sts128(smem + kOffQlo + off, lo[0], lo[1], lo[2], lo[3]);
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) bar_arrive(&bars.q_ready);
+            }
+            const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+            for (int j = 0; j < nb; ++j) {
+                const int buf = j & 1;
+                if (!bar_wait_warp(&bars.s_full[buf], (j >> 1) & 1)) { atomicOr(&bars.flags, 1); break; }
+                tc_fence_after();
+                float s[kBlkTok];
+                tmem_ld32(tS0 + buf * 64 + lane_addr, s);
+                tmem_ld32(tS0 + buf * 64 + 32 + lane_addr, s + 32);
+                const int kp0 = j * kBlkTok;
+                float bm = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < kBlkTok; ++c) {
+                    const int kp = kp0 + c;
+                    s[c] = (kp <= qpos && kp < kv_end) ? s[c] * isig : -INFINITY;
+                    bm = fmaxf(bm, s[c]);
+                }
+                // lazy rescale: move the reference max only when it grows by > 2^8
+                const bool grow = bm > m_run + kRescaleThreshold || (m_run == -INFINITY && bm > -INFINITY);
+                bool stop = false;
+                if (__any_sync(0xFFFFFFFFu, grow)) {
+                    const float mn = grow ? bm : m_run;
+                    const float al = (m_run == -INFINITY) ? 0.0f : ex2(m_run - mn);
+                    if (j > 0) {
+                        // the previous P.V must have landed before O is rescaled
+                        if (!bar_wait_warp(&bars.pv_done[buf ^ 1], ((j - 1) >> 1) & 1)) {
+                            atomicOr(&bars.flags, 1);
+                            stop = true;
+                        }
+                        if (!stop) {
+                            tc_fence_after();
+#pragma unroll 1
+                            for (int cc = 0; cc < 4; ++cc) {
+                                float o[32];
+                                tmem_ld32(tO + cc * 32 + lane_addr, o);
+#pragma unroll
+                                for (int i = 0; i < 32; ++i) o[i] *= al;
+                                tmem_st32(tO + cc * 32 + lane_addr, o);
+                            }
+                        }
+                    }
+                    l_run *= al;
+                    m_run = mn;
+                }
+                if (stop) break;
+                // P tile buffer must be free: P.V(j-2) done
+                if (j >= 2 && !bar_wait_warp(&bars.pv_done[buf], ((j - 2) >> 1) & 1)) {
+                    atomicOr(&bars.flags, 1);
+                    break;
+                }
+                uint8_t* P = smem + kOffP + buf * kPBytes;
+                float lsum = 0.0f;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float p0 = ex2(s[8 * ch + 2 * e] - m_run), p1 = ex2(s[8 * ch + 2 * e + 1] - m_run);
+                        lsum += p0 + p1;
+                        w[e] = h2(p0, p1);
+                    }
+                    sts128(P + sw128(r, ch), w[0], w[1], w[2], w[3]);
+                }
+                l_run += lsum;
+                fence_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) bar_arrive(&bars.p_full[buf]);
+            }
+        } else if (warp < kMmaWarp) {
+            // ------------------------------------------------------ dequant warps
+            const int dt = threadIdx.x - 32 * kWarpsSoftmax;   // 0..127
+            const int tkn = dt >> 1, half = dt & 1;            // token of the block, half of head_dim
+            const bool issuer = (dt == 0);
+            int issued = 0;
+            auto issue = [&](int j) {   // stage j % kStageN <- the pages of block j
+                const int st = j % kStageN;
+                const int p_lo = j * 4, p_hi = min(npg, p_lo + 4);
+                bar_expect(&bars.stage_full[st], (uint32_t)(p_hi - p_lo) * kTile);
+                for (int p = p_lo; p < p_hi; ++p) {
+                    const int pg = __ldg(pt + p);
+                    bulk_copy(smem + kOffStage + st * kStageBytes + (p - p_lo) * kTile,
+                              layer_base + ((size_t)pg * a.Hkv + h) * kTile, kTile, &bars.stage_full[st]);
+                }
+            };
+            if (issuer)
+                for (; issued < kStageN - 1 && issued < nb; ++issued) issue(issued);
+            for (int j = 0; j < nb; ++j) {
+                const int buf = j & 1, st = j % kStageN;
+                int issue_ok = 1;
+                if (issuer && issued < nb) {
+                    if (issued >= kStageN &&
+                        !bar_wait(&bars.stage_empty[issued % kStageN], ((issued / kStageN) - 1) & 1)) {
+                        issue_ok = 0;
+                    } else {
+                        issue(issued);
+                        ++issued;
+                    }
+                }
+                if (!__shfl_sync(0xFFFFFFFFu, issue_ok, 0)) { atomicOr(&bars.flags, 1); break; }
+                if (!bar_wait_warp(&bars.stage_full[st], (j / kStageN) & 1)) { atomicOr(&bars.flags, 1); break; }
+                // read this thread's token row (64 dims of keys and values) from the stage
+                const int kp = j * kBlkTok + tkn;
+                const bool valid = kp < kv_end;
+                const uint8_t* T = smem + kOffStage + st * kStageBytes + (tkn >> 4) * kTile;
+                const int trow = tkn & 15;
+                uint4 kc[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+                uint4 vc[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+                uint32_t ks = 0, vs[4] = {0, 0, 0, 0};
+                if (valid) {
+                    kc[0] = *reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32);
+                    kc[1] = *reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32 + 16);
+                    ks = *reinterpret_cast<const uint32_t*>(T + kKScales + trow * 8 + half * 4);
+                    vc[0] = *reinterpret_cast<const uint4*>(T + kVCodes + trow * 64 + half * 32);
+                    vc[1] = *reinterpret_cast<const uint4*>(T + kVCodes + trow * 64 + half * 32 + 16);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) vs[q] = T[kVScales + (half * 4 + q) * 16 + trow];
+                }
+                __syncwarp();
+                if ((dt & 31) == 0) bar_arrive(&bars.stage_empty[st]);
+                // K/V tile buffer must be free: P.V(j-2) done
+                if (j >= 2 && !bar_wait_warp(&bars.pv_done[buf], ((j - 2) >> 1) & 1)) {
+                    atomicOr(&bars.flags, 1);
+                    break;
+                }
+                uint8_t* Kt = smem + kOffK + buf * kKBytes;
+                uint8_t* Vt = smem + kOffV + buf * kVBytes;
+                // 4 blocks of 16 dims: 8 code bytes and one scale each
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t kw0 = (q < 2) ? (q == 0 ? kc[0].x : kc[0].z) : (q == 2 ? kc[1].x : kc[1].z);
+                    const uint32_t kw1 = (q < 2) ? (q == 0 ? kc[0].y : kc[0].w) : (q == 2 ? kc[1].y : kc[1].w);
+                    const uint32_t vw0 = (q < 2) ? (q == 0 ? vc[0].x : vc[0].z) : (q == 2 ? vc[1].x : vc[1].z);
+                    const uint32_t vw1 = (q < 2) ? (q == 0 ? vc[0].y : vc[0].w) : (q == 2 ? vc[1].y : vc[1].w);
+                    uint32_t ka[4], kb[4], va[4], vb[4];
+                    e2m1x8(kw0, ka);
+                    e2m1x8(kw1, kb);
+                    e2m1x8(vw0, va);
+                    e2m1x8(vw1, vb);
+                    const uint32_t ksh = e4m3x2_to_f16x2((ks >> (8 * q)) & 0xFFu) & 0xFFFFu;
+                    const uint32_t vsh = e4m3x2_to_f16x2(vs[q]) & 0xFFFFu;
+                    const uint32_t ksc = valid ? (ksh | (ksh << 16)) : 0u;
+                    const uint32_t vsc = valid ? (vsh | (vsh << 16)) : 0u;
+                    // chunk index along head_dim: 2 chunks (8 dims each) per block
+                    const int dim_chunk = half * 8 + 2 * q;          // 0..15
+                    const int plane = dim_chunk >> 3, ch = dim_chunk & 7;
+                    // keys: K-major, row = token, dims 0..63 / 64..127 in planes of 64 rows x 128 B
+                    sts128(Kt + plane * (kBlkTok * 128) + sw128(tkn, ch), hmul2u(ka[0], ksc), hmul2u(ka[1], ksc),
+                           hmul2u(ka[2], ksc), hmul2u(ka[3], ksc));
+                    sts128(Kt + plane * (kBlkTok * 128) + sw128(tkn, ch + 1), hmul2u(kb[0], ksc),
+                           hmul2u(kb[1], ksc), hmul2u(kb[2], ksc), hmul2u(kb[3], ksc));
+                    // values: MN-major, row = token (the K of P.V), 128-byte rows of 64 dims
+                    sts128(Vt + plane * (kBlkTok * 128) + sw128(tkn, ch), hmul2u(va[0], vsc), hmul2u(va[1], vsc),
+                           hmul2u(va[2], vsc), hmul2u(va[3], vsc));
+                    sts128(Vt + plane * (kBlkTok * 128) + sw128(tkn, ch + 1), hmul2u(vb[0], vsc),
+                           hmul2u(vb[1], vsc), hmul2u(vb[2], vsc), hmul2u(vb[3], vsc));
+                }
+                fence_async_smem();
+                __syncwarp();
+                if ((dt & 31) == 0) bar_arrive(&bars.kv_full[buf]);
+            }
+            if (issuer) bars.issued = issued;
+        } else if (lane == 0) {
+            // ------------------------------------------------------ MMA issuer
+            const uint32_t qk = f16_idesc(kRows, kBlkTok, false);
+            const uint32_t pv = f16_idesc(kRows, kD, true);
+            const uint32_t qhi = su32(smem + kOffQhi), qlo = su32(smem + kOffQlo);
+            bool ok = bar_wait(&bars.q_ready, 0);
+            for (int j = 0; ok && j <= nb; ++j) {
+                if (j < nb) {
+                    const int buf = j & 1;
+                    if (!bar_wait(&bars.kv_full[buf], (j >> 1) & 1)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t kt = su32(smem + kOffK + buf * kKBytes);
+                    const uint32_t sd = tS0 + buf * 64;
+#pragma unroll 1
+                    for (int part = 0; part < 2; ++part) {
+                        const uint32_t qb = part ? qlo : qhi;
+#pragma unroll
+                        for (int s = 0; s < 8; ++s) {
+                            const uint64_t ad = sw128_desc(qb + (s >> 2) * (kRows * 128) + (s & 3) * 32, 16, 1024);
+                            const uint64_t bd = sw128_desc(kt + (s >> 2) * (kBlkTok * 128) + (s & 3) * 32, 16, 1024);
+                            mma_f16(sd, ad, bd, qk, (part | s) ? 1u : 0u);
+                        }
+                    }
+                    mma_commit(&bars.s_full[buf]);
+                }
+                if (j >= 1) {
+                    const int jp = j - 1, buf = jp & 1;
+                    if (!bar_wait(&bars.p_full[buf], (jp >> 1) & 1)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t pt_ = su32(smem + kOffP + buf * kPBytes);
+                    const uint32_t vt = su32(smem + kOffV + buf * kVBytes);
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) {
+                        const uint64_t ad = sw128_desc(pt_ + s * 32, 16, 1024);
+                        // 16 tokens = two 8-row atoms (stride 1024); dims 64..127 one plane (64 x 128 B) away
+                        const uint64_t bd = sw128_desc(vt + s * 2048, kBlkTok * 128, 1024);
+                        mma_f16(tO, ad, bd, pv, (jp | s) ? 1u : 0u);
+                    }
+                    mma_commit(&bars.pv_done[buf]);
+                }
+            }
+            if (!ok) atomicOr(&bars.flags, 1);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const bool timed_out = bars.flags != 0;
+    if (timed_out && threadIdx.x == 32 * kWarpsSoftmax) {
+        // drain: the packed-page copies still in flight
+        const int issued = bars.issued;
+        for (int j = max(0, issued - kStageN); j < issued; ++j)
+            (void)bar_wait(&bars.stage_full[j % kStageN], (j / kStageN) & 1);
+        set_status(a.status, KVQ_DEV_TIMEOUT);
+    }
+    if (timed_out && threadIdx.x == 32 * kMmaWarp) {
+        // drain: every MMA issued by this thread completes before the commit
+        // arrives; TMEM is freed only after that
+        mma_commit(&bars.drain);
+        (void)bar_wait(&bars.drain, 0);
+    }
+
+    // ---------------------------------------------------------------- epilogue
+    // (dead is uniform across the CTA, so the warp-collective TMEM loads below
+    // run on every lane of a softmax warp or on none)
+    const bool dead = poison || timed_out || nb == 0;
+    if (warp < kWarpsSoftmax) {
+        const int r = threadIdx.x;
+        const int head = r >> 5, tok = r & 31;
+        const int qi = q0 + tok;
+        float res[kD];
+        if (!dead) {
+            // the last P.V has landed once pv_done of the last block completes
+            const int jl = nb - 1;
+            const bool ok = bar_wait_warp(&bars.pv_done[jl & 1], (jl >> 1) & 1);
+            tc_fence_after();
+            const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+            const float sc = (ok && l_run > 0.0f) ? __ldg(a.gv + li) / l_run : 0.0f;
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+                float o[32];
+                tmem_ld32(tO + cc * 32 + lane_addr, o);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) res[cc * 32 + i] = ok ? o[i] * sc : 0.0f;
+            }
+            if (!ok && lane == 0) set_status(a.status, KVQ_DEV_TIMEOUT);
+        } else {
+#pragma unroll
+            for (int i = 0; i < kD; ++i) res[i] = 0.0f;
+        }
+        if (head < a.G && tok < qn) {
+            TO* dst = reinterpret_cast<TO*>(a.out) +
+                      ((((size_t)li * a.batch + b) * a.q_len + qi) * a.Hq + h * a.G + head) * kD;
+            if constexpr (sizeof(TO) == 4) {
+#pragma unroll
+                for (int i = 0; i < kD / 4; ++i)
+                    reinterpret_cast<float4*>(dst)[i] = make_float4(res[4 * i], res[4 * i + 1], res[4 * i + 2],
+                                                                    res[4 * i + 3]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < kD / 8; ++i) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        __nv_bfloat162 t2 = __floats2bfloat162_rn(res[8 * i + 2 * e], res[8 * i + 2 * e + 1]);
+                        w[e] = *reinterpret_cast<uint32_t*>(&t2);
+                    }
+                    reinterpret_cast<uint4*>(dst)[i] = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ launcher
+static cudaError_t launch_prefill(const AttnArgs& a, dim3 grid, bool qb, bool ob, cudaStream_t st) {
+    cudaError_t e;
+#define KVQ_LAUNCH(TQ, TO)                                                                                     \
+    e = cudaFuncSetAttribute(prefill_tc_kernel<TQ, TO>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc); \
+    if (e != cudaSuccess) return e;                                                                            \
+    prefill_tc_kernel<TQ, TO><<<grid, kThreads, kSmemAlloc, st>>>(a);
+    if (qb && ob) { KVQ_LAUNCH(__nv_bfloat16, __nv_bfloat16) }
+    else if (qb) { KVQ_LAUNCH(__nv_bfloat16, float) }
+    else if (ob) { KVQ_LAUNCH(float, __nv_bfloat16) }
+    else { KVQ_LAUNCH(float, float) }
+#undef KVQ_LAUNCH
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_tc(const AttnArgs& a, int nlayers, bool q_bf16, bool out_bf16, cudaStream_t st) {
+    dim3 grid((a.q_len + kQTok - 1) / kQTok, a.batch * a.Hkv, nlayers);
+    return launch_prefill(a, grid, q_bf16, out_bf16, st);
+}
+
+}  // namespace kvq
