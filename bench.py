@@ -42,7 +42,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
-    ap.add_argument("--workload", default="ragged", choices=["ragged"])
+    ap.add_argument("--workload", default="ragged", choices=["ragged", "prefill", "qwen3_8b", "hadamard"],
+                    help="ragged (default, the decode-throughput workload); prefill, qwen3_8b, hadamard: "
+                         "the chunked-prefill and prefix workloads, for their own kernel numbers")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -225,6 +227,133 @@ class Ragged:
                                   self.seq_lens[s], out=self.out, workspace=self.ws)
 
 
+class Prefill:
+    """Chunked causal prefill: 36 layers, batch 8, 8192 cached tokens + a
+    512-token chunk.  One step = append the chunk's K/V into every layer, then
+    prefill attention of every layer (tcgen05)."""
+
+    def __init__(self, kvq, synth, layers=36):
+        import dataclasses
+        w = dataclasses.replace(synth.WORKLOADS["prefill"], num_layers=layers)
+        self.kvq, self.w = kvq, w
+        L, B, P0, Tq = w.num_layers, w.batch, w.context, w.prefill_chunk
+        self.L, self.B, self.P0, self.Tq = L, B, P0, Tq
+        dev = "cuda"
+        total = P0 + Tq
+        lens = torch.full((B,), total, dtype=torch.int32)
+        self.page_table, self.num_pages = synth.build_page_table(w, lens)
+        self.shape = kvq.Shape(L, w.num_q_heads, w.num_kv_heads)
+        kc = torch.stack([synth.calibration_windows(w, l, dev)[0] for l in range(L)])
+        vc = torch.stack([synth.calibration_windows(w, l, dev)[1] for l in range(L)])
+        self.calib = kvq.calibrate_smoothing(self.shape, kc, vc, exclude_pos0=True)
+        del kc, vc
+        self.cache = kvq.new_cache(self.shape, self.num_pages, dev)
+        H, D = w.num_kv_heads, w.head_dim
+        pre_slots = torch.cat([synth.slot_mapping(self.page_table, torch.full((P0,), b), torch.arange(P0))
+                               for b in range(B)]).to(dev)
+        self.chunk_slots = torch.cat([synth.slot_mapping(self.page_table, torch.full((Tq,), b),
+                                                         torch.arange(P0, total)) for b in range(B)]).to(dev)
+        self.chunk_k = torch.empty(L, B * Tq, H, D, dtype=torch.bfloat16, device=dev)
+        self.chunk_v = torch.empty_like(self.chunk_k)
+        for l in range(L):
+            ks, vs = [], []
+            for b in range(B):
+                k, v = synth.sequence_kv(w, l, b, total, dev)
+                ks.append(k[:P0])
+                vs.append(v[:P0])
+                self.chunk_k[l, b * Tq:(b + 1) * Tq] = k[P0:]
+                self.chunk_v[l, b * Tq:(b + 1) * Tq] = v[P0:]
+            kvq.quantize_append(self.shape, self.calib, self.cache, torch.cat(ks), torch.cat(vs), pre_slots, layer0=l)
+            del ks, vs
+        self.q = torch.stack([synth.prefill_queries(w, l, dev) for l in range(L)])   # [L][B][Tq][Hq][D]
+        self.q_start = torch.full((B,), P0, dtype=torch.int32, device=dev)
+        self.seq_lens = lens.to(dev)
+        self.pt = self.page_table.to(dev)
+        self.out = torch.empty_like(self.q)
+        # attended keys summed over the chunk's queries, per (layer, sequence, query head)
+        keys = Tq * P0 + Tq * (Tq + 1) // 2
+        self.flops = 4 * D * w.num_q_heads * L * B * keys
+        torch.cuda.synchronize()
+
+    def append(self):
+        self.kvq.quantize_append(self.shape, self.calib, self.cache, self.chunk_k, self.chunk_v, self.chunk_slots)
+
+    def attend(self):
+        self.kvq.prefill_attention(self.shape, self.calib, self.cache, self.q, self.q_start, self.pt, self.seq_lens,
+                                   out=self.out)
+
+
+class Prefix:
+    """Qwen3-8B-shaped (or Hadamard) prefix workload: one step = quantise-append
+    every layer's whole prefix (one launch), then one decode step of every layer."""
+
+    def __init__(self, kvq, synth, name, layers=36):
+        import dataclasses
+        w = dataclasses.replace(synth.WORKLOADS[name], num_layers=layers)
+        self.kvq, self.w = kvq, w
+        L, B, T = w.num_layers, w.batch, w.context
+        self.L, self.B, self.T = L, B, T
+        dev = "cuda"
+        lens = torch.full((B,), T, dtype=torch.int32)
+        self.page_table, self.num_pages = synth.build_page_table(w, lens)
+        self.shape = kvq.Shape(L, w.num_q_heads, w.num_kv_heads, use_hadamard=w.hadamard)
+        kc = torch.stack([synth.calibration_windows(w, l, dev)[0] for l in range(L)])
+        vc = torch.stack([synth.calibration_windows(w, l, dev)[1] for l in range(L)])
+        self.calib = kvq.calibrate_smoothing(self.shape, kc, vc, exclude_pos0=True)
+        del kc, vc
+        self.cache = kvq.new_cache(self.shape, self.num_pages, dev)
+        H, D = w.num_kv_heads, w.head_dim
+        self.slots = torch.cat([synth.slot_mapping(self.page_table, torch.full((T,), b), torch.arange(T))
+                                for b in range(B)]).to(dev)
+        self.k = torch.empty(L, B * T, H, D, dtype=torch.bfloat16, device=dev)
+        self.v = torch.empty_like(self.k)
+        for l in range(L):
+            for b in range(B):
+                k, v = synth.sequence_kv(w, l, b, T, dev)
+                self.k[l, b * T:(b + 1) * T] = k
+                self.v[l, b * T:(b + 1) * T] = v
+        self.q = torch.stack([synth.decode_queries(w, l, 0, dev) for l in range(L)])
+        self.seq_lens = lens.to(dev)
+        self.pt = self.page_table.to(dev)
+        self.out = torch.empty(L, B, w.num_q_heads, D, dtype=torch.bfloat16, device=dev)
+        need = kvq.decode_workspace_bytes(self.shape, L, B, self.page_table.shape[1])
+        self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        self.launches = 2 + (1 if need else 0)
+        self.append_bytes = L * B * T * (2 * H * D * 2 + TOKEN_LAYER_BYTES)
+        self.decode_bytes = L * B * T * TOKEN_LAYER_BYTES + L * B * QO_BYTES_PER_SEQ_LAYER
+        torch.cuda.synchronize()
+
+    def append(self):
+        self.kvq.quantize_append(self.shape, self.calib, self.cache, self.k, self.v, self.slots)
+
+    def decode(self):
+        self.kvq.decode_attention(self.shape, self.calib, self.cache, self.q, self.pt, self.seq_lens, out=self.out,
+                                  workspace=self.ws)
+
+
+def time_two_kernels(first, second, warmup: int, steps: int, world: int):
+    """Time steps of first() + second() with events around each call."""
+    st = torch.cuda.current_stream()
+    for _ in range(warmup):
+        first()
+        second()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(st)
+    for i in range(steps):
+        ev[i][0].record(st)
+        first()
+        ev[i][1].record(st)
+        second()
+        ev[i][2].record(st)
+    t1.record(st)
+    torch.cuda.synchronize()
+    barrier(world)
+    return (t0.elapsed_time(t1), [e[0].elapsed_time(e[1]) for e in ev], [e[1].elapsed_time(e[2]) for e in ev])
+
+
 def time_device(wl: Ragged, warmup: int, steps: int, world: int):
     st = torch.cuda.current_stream()
     for i in range(warmup):
@@ -375,6 +504,67 @@ def config_block(wl=None):
             "parallelism": "replicas (independent sequences per GPU)"}
 
 
+def other_workload(args, kvq, synth, rank, world):
+    """One JSON line for the chunked-prefill or prefix workloads."""
+    peak_hbm, hbm_kind = measured_peak()
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        peak_tf, tf_kind = float(pk["bf16_tflops"]), "measured (cuBLAS bf16 burst; fp16 runs at the same rate)"
+        peak_tf_sus = float(pk.get("bf16_tflops_sustained", peak_tf))
+    except (OSError, KeyError, ValueError):
+        peak_tf, tf_kind, peak_tf_sus = 1590.0, "fallback", 1400.0
+    warm = max(3, args.warmup)
+    clock = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if args.workload == "prefill":
+        wl = Prefill(kvq, synth, args.layers)
+        total, app_ms, pre_ms = time_two_kernels(wl.append, wl.attend, warm, args.steps, world)
+        clocks = clock.stop() if clock else None
+        total = max_over_ranks(total, world)
+        tokens = world * wl.B * wl.Tq * args.steps
+        pre = statistics.mean(pre_ms)
+        achieved = wl.flops / (pre / 1e3) / 1e12
+        line = {"metric": "NVFP4-KV chunked causal prefill tokens/s; achieved tensor TFLOP/s vs B200 peak",
+                "value": tokens / (total / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": warm, "ms_per_step": total / args.steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f16 mma (q split hi+lo), f32 accumulate", "data": "synthetic",
+                "config": {"workload": f"chunked prefill: {wl.L} layers, batch 8, 8192 cached + 512-token causal "
+                                       "chunk, 32 q / 8 kv heads, head_dim 128", "layers": wl.L},
+                "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                             "frac": achieved / peak_tf, "frac_of_sustained": achieved / peak_tf_sus,
+                             "traffic": None, "peak_source": tf_kind,
+                             "kernel": "kvq prefill (tcgen05)", "alg_flops_per_launch": wl.flops,
+                             "note": "algorithmic flops count 4 per attended (query head, key, dim); the kernel "
+                                     "issues 1.5x that on the tensor pipe (query hi + lo)"},
+                "append_ms": statistics.mean(app_ms), "prefill_ms": pre, "gpu_launches": 2 * args.steps,
+                "clocks": clocks}
+    else:
+        wl = Prefix(kvq, synth, args.workload, args.layers)
+        total, app_ms, dec_ms = time_two_kernels(wl.append, wl.decode, warm, args.steps, world)
+        clocks = clock.stop() if clock else None
+        total = max_over_ranks(total, world)
+        app, dec = statistics.mean(app_ms), statistics.mean(dec_ms)
+        line = {"metric": METRIC, "value": world * wl.B * args.steps / (total / 1e3), "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": warm, "ms_per_step": total / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic",
+                "config": {"workload": f"{args.workload}: {wl.L} layers, batch {wl.B} x {wl.T} tokens; one step = "
+                                       "quantise-append of the whole prefix + one decode step",
+                           "hadamard": wl.w.hadamard},
+                "roofline": {"bound": "hbm", "achieved": wl.decode_bytes / (dec / 1e3) / 1e9, "peak": peak_hbm,
+                             "unit": "GB/s", "frac": wl.decode_bytes / (dec / 1e3) / 1e9 / peak_hbm, "traffic": None,
+                             "peak_source": hbm_kind, "kernel": "kvq decode", "alg_bytes_per_launch": wl.decode_bytes},
+                "append": {"achieved": wl.append_bytes / (app / 1e3) / 1e9, "unit": "GB/s",
+                           "frac": wl.append_bytes / (app / 1e3) / 1e9 / peak_hbm, "alg_bytes_per_launch":
+                           wl.append_bytes, "ms": app},
+                "decode_ms": dec, "gpu_launches": wl.launches * args.steps, "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     rank, world, local = dist_setup(args)
@@ -403,6 +593,8 @@ def main():
     import bit_attention_decode_b200 as kvq
     import synth
     assert torch.cuda.is_available(), "bench needs a CUDA device"
+    if args.workload != "ragged":
+        return other_workload(args, kvq, synth, rank, world)
     t_setup = time.time()
     wl = Ragged(kvq, synth, args.layers)
     sys.stderr.write(f"[bench] setup {time.time() - t_setup:.1f} s, {wl.num_pages} pages, "
