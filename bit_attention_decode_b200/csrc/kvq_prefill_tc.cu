@@ -7,22 +7,27 @@
 // and rotation folded into the query as in "NVFP4 attention cache on W4A4
 // Qwen3-8B" (rstation.ai), observation 2).
 //
-// One CTA: one layer, one sequence, one kv head, a tile of 32 query tokens.
-// The tile's 128 MMA rows are the G <= 4 query heads of the kv head times
-// the 32 tokens (row = head * 32 + token), so each dequantised key/value
-// block feeds 4 heads at once.  Per 64-token key block (4 pages):
+// One CTA: one layer, one sequence, one kv head, and two tiles (A, B) of 32
+// query tokens each.  A tile's 128 MMA rows are the G <= 4 query heads of
+// the kv head times its 32 tokens (row = head * 32 + token), so each
+// dequantised key/value block feeds 8 query heads x 32 tokens.  Per 64-token
+// key block (4 pages):
 //   dequant warps (4): bulk-copy the 4 packed page tiles into a staging
 //     ring, dequantise to fp16 (E2M1 x E4M3 is exact in fp16) into a K tile
 //     (K-major) and a V tile (MN-major), both in the 128-byte-swizzled
 //     canonical layouts the MMA reads; rows past the sequence are zeros.
-//   MMA warp (1 elected thread): S = Q_hi K^T + Q_lo K^T (M=128, N=64, K=16
-//     steps; the query is split into fp16 hi + lo parts so its rounding does
-//     not reach the scores) into one of two TMEM score buffers, then
-//     O += P V (M=128, N=128) into the TMEM output accumulator.
-//   softmax warps (4, one TMEM lane = one row per thread): causal mask,
-//     running max with lazy rescaling (the output in TMEM is rescaled only
-//     when the max grows by more than 2^8), probabilities rounded once to
-//     fp16 into a swizzled P tile.
+//   MMA warp (1 elected thread): for each tile, S = Q_hi K^T + Q_lo K^T
+//     (M=128, N=64, K=16 steps; the query is split into fp16 hi + lo parts
+//     so its rounding does not reach the scores) into one of the tile's two
+//     TMEM score buffers, then O += P V (M=128, N=128) with P read from TMEM.
+//   softmax warpgroups (one per tile; a thread owns one TMEM lane = row):
+//     causal mask on diagonal blocks only, running max with lazy rescaling
+//     (the output in TMEM is rescaled only when the max grows by more than
+//     2^8), probabilities rounded once to fp16 and stored back over the
+//     first 32 columns of their own score buffer as the A operand of P V.
+// The two tiles ping-pong: while one warpgroup works on its scores, the
+// tensor pipe runs the other tile's MMAs.  TMEM: O_A, O_B (128 columns each),
+// S_A[2], S_B[2] (64 each) = 512 columns.
 // All hand-offs are mbarriers with bounded waits; a wait that runs out sets
 // KVQ_DEV_TIMEOUT, the CTA writes zeros and frees its TMEM.
 #include "kvq_attn.cuh"
@@ -32,31 +37,30 @@
 namespace kvq {
 namespace {
 
-constexpr int kRows = 128;          // MMA M: 4 heads x 32 query tokens
+constexpr int kRows = 128;          // MMA M of one tile: 4 heads x 32 query tokens
 constexpr int kQTok = 32;           // query tokens per tile
+constexpr int kTiles = 2;           // query tiles per CTA (A, B)
 constexpr int kBlkTok = 64;         // key tokens per block (4 pages)
 constexpr int kStageN = 3;          // packed-page staging stages
-constexpr uint32_t kTmemCols = 256; // O [0,128), S0 [128,192), S1 [192,256)
+constexpr uint32_t kTmemCols = 512; // O_A, O_B [0,256), S_A[2] [256,384), S_B[2] [384,512)
 constexpr unsigned long long kWaitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 // shared memory map (offsets from a 1024-aligned base)
-constexpr int kQBytes = kRows * kD * 2;           // 32 KB per fp16 query tile (hi or lo)
+constexpr int kQBytes = kRows * kD * 2;           // 32 KB per fp16 query tile part (hi or lo)
 constexpr int kKBytes = kBlkTok * kD * 2;         // 16 KB per fp16 key tile
 constexpr int kVBytes = kBlkTok * kD * 2;         // 16 KB per fp16 value tile
-constexpr int kPBytes = kRows * kBlkTok * 2;      // 16 KB per fp16 probability tile
 constexpr int kStageBytes = 4 * kTile;            // 4 packed page tiles of one head
-constexpr int kOffQhi = 0;
-constexpr int kOffQlo = kOffQhi + kQBytes;
-constexpr int kOffK = kOffQlo + kQBytes;          // 2 buffers
+constexpr int kOffQ = 0;                          // [tile][hi, lo]
+constexpr int kOffK = kOffQ + kTiles * 2 * kQBytes;   // 2 buffers
 constexpr int kOffV = kOffK + 2 * kKBytes;        // 2 buffers
-constexpr int kOffP = kOffV + 2 * kVBytes;        // 2 buffers
-constexpr int kOffStage = kOffP + 2 * kPBytes;    // kStageN stages
+constexpr int kOffStage = kOffV + 2 * kVBytes;    // kStageN stages
 constexpr int kSmemBytes = kOffStage + kStageN * kStageBytes;
 constexpr int kSmemAlloc = kSmemBytes + 1024;     // room to align the base
 
-enum { kWarpsSoftmax = 4, kWarpsDequant = 4 };
-constexpr int kMmaWarp = kWarpsSoftmax + kWarpsDequant;   // warp 8
+enum { kWarpsSoftmax = 4 * kTiles, kWarpsDequant = 3 };
+constexpr int kDequantWarp0 = kWarpsSoftmax;                   // warps 8..10
+constexpr int kMmaWarp = kWarpsSoftmax + kWarpsDequant;        // warp 11
 constexpr int kThreads = 32 * (kMmaWarp + 1);
 
 // ------------------------------------------------------------------ primitives
@@ -123,6 +127,12 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b,
                  "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }"
                  ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
 }
+// same, with the A operand (M x K, two fp16 per 32-bit column) in TMEM
+__device__ __forceinline__ void mma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile("{ .reg .pred p; setp.ne.b32 p, %4, 0;\n"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }"
+                 ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
 __device__ __forceinline__ void mma_commit(uint64_t* b) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(b))
                  : "memory");
@@ -153,6 +163,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
                    "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]),
                    "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]),
                    "r"(r[31])
+                 : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+                 "%15,%16};"
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                   "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+                   "r"(r[15])
                  : "memory");
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -209,13 +228,13 @@ __device__ __forceinline__ void load_row128<__nv_bfloat16>(const __nv_bfloat16* 
 }
 
 struct PrefillBars {
-    uint64_t q_ready;                 // softmax warps wrote the query tiles (count 4)
+    uint64_t q_ready;                 // both softmax warpgroups wrote their query tiles (count 8)
     uint64_t stage_full[kStageN];     // packed pages landed (tx bytes)
-    uint64_t stage_empty[kStageN];    // dequant warps read the stage (count 4)
-    uint64_t kv_full[2];              // K/V tile j%2 written (count 4)
-    uint64_t s_full[2];               // QK(j) done (commit)
-    uint64_t p_full[2];               // P tile j%2 written, O rescaled (count 4)
-    uint64_t pv_done[2];              // PV(j) done (commit)
+    uint64_t stage_empty[kStageN];    // dequant warps read the stage (count 3)
+    uint64_t kv_full[2];              // K/V tile j%2 written (count 3)
+    uint64_t s_full[kTiles][2];       // QK(tile, j) done (commit)
+    uint64_t p_full[kTiles][2];       // P(tile, j) stored in TMEM, O rescaled (count 4)
+    uint64_t pv_done[kTiles][2];      // PV(tile, j) done (commit)
     uint64_t drain;                   // last commit before TMEM is freed after a timeout
     uint32_t tmem_base;
     int flags;                        // 1: a bounded wait ran out
@@ -223,21 +242,21 @@ struct PrefillBars {
 };
 
 // ------------------------------------------------------------------ kernel
-// grid (q tiles, batch * Hkv, nlayers), block 288.
+// grid (query-tile pairs, batch * Hkv, nlayers), block 384.
 template <typename TQ, typename TO>
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ PrefillBars bars;
 
-    const int tile = blockIdx.x, b = blockIdx.y / a.Hkv, h = blockIdx.y % a.Hkv, li = blockIdx.z;
+    const int pair = blockIdx.x, b = blockIdx.y / a.Hkv, h = blockIdx.y % a.Hkv, li = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int len = __ldg(a.seq_lens + b);
     const int qs = __ldg(a.q_start + b);
-    const int q0 = tile * kQTok;
-    const int qn = min(kQTok, a.q_len - q0);                 // query tokens in this tile
+    const int q0 = pair * (kTiles * kQTok);
+    const int qn = min(kTiles * kQTok, a.q_len - q0);        // query tokens of the pair
     const bool bad_len = len < 0 || len > a.max_pages * kPage;
-    // keys needed by the tile: positions < min(len, q_start + q0 + qn)
+    // keys needed by the pair: positions < min(len, q_start + q0 + qn)
     int kv_end = bad_len ? 0 : min(len, qs + q0 + qn);
     if (kv_end < 0) kv_end = 0;
     const int nb = (kv_end + kBlkTok - 1) / kBlkTok;          // 64-token blocks
@@ -255,9 +274,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
         }
         for (int i = 0; i < 2; ++i) {
             bar_init(&bars.kv_full[i], kWarpsDequant);
-            bar_init(&bars.s_full[i], 1);
-            bar_init(&bars.p_full[i], kWarpsSoftmax);
-            bar_init(&bars.pv_done[i], 1);
+            for (int t = 0; t < kTiles; ++t) {
+                bar_init(&bars.s_full[t][i], 1);
+                bar_init(&bars.p_full[t][i], 4);
+                bar_init(&bars.pv_done[t][i], 1);
+            }
         }
         bar_init(&bars.drain, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -269,12 +290,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
     }
     badp = __syncthreads_or(badp);
     if (threadIdx.x == 0) {
-        if (bad_len && tile == 0 && h == 0) set_status(a.status, KVQ_DEV_BAD_LEN);
+        if (bad_len && pair == 0 && h == 0) set_status(a.status, KVQ_DEV_BAD_LEN);
         if (badp) set_status(a.status, KVQ_DEV_BAD_PAGE);
     }
     const bool poison = bad_len || badp;
 
-    // TMEM: one warp allocates 256 columns for the CTA
+    // TMEM: one warp allocates all 512 columns for the CTA (one CTA per SM)
     if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&bars.tmem_base)),
                      "r"(kTmemCols) : "memory");
@@ -284,19 +305,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars.tmem_base;
-    const uint32_t tO = tmem, tS0 = tmem + 128;
+    // per tile t: O at tmem + 128 t; S buffer u at tmem + 256 + 128 t + 64 u
+    auto tO = [&](int t) { return tmem + 128u * t; };
+    auto tS = [&](int t, int u) { return tmem + 256u + 128u * t + 64u * u; };
 
     // per-row state of the softmax warps, kept to the epilogue
     float m_run = -INFINITY, l_run = 0.0f, isig = 1.0f;
-    bool row_ok = false;
 
     if (!poison && nb > 0) {
         if (warp < kWarpsSoftmax) {
-            // ------------------------------------------------------ softmax warps
-            const int r = threadIdx.x;                 // TMEM lane = MMA row
+            // ------------------------------------------------------ softmax warpgroups
+            const int t = warp >> 2;                   // tile of this warpgroup
+            const int r = threadIdx.x & 127;           // TMEM lane = MMA row
             const int head = r >> 5, tok = r & 31;     // row = head * 32 + token
-            const int qi = q0 + tok;
-            row_ok = head < a.G && tok < qn;
+            const int qi = q0 + t * kQTok + tok;
+            const bool row_ok = head < a.G && (t * kQTok + tok) < qn;
             const int qpos = qs + qi;                  // absolute position of this query
             // query prologue: q~ = q * s (+ rotation) * g_K log2(e) / sqrt(128),
             // per-row power-of-two normalisation, fp16 hi + lo tiles
@@ -338,6 +361,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                 }
                 const float sig = ldexpf(1.0f, 14 - ex);
                 isig = ldexpf(1.0f, ex - 14);
+                uint8_t* qhi = smem + kOffQ + (2 * t) * kQBytes;
+                uint8_t* qlo = qhi + kQBytes;
                 // K-major 128B-swizzled tiles: dims 0..63 in atom plane 0, 64..127 in plane 1
 #pragma unroll
                 for (int ch = 0; ch < 16; ++ch) {
@@ -350,29 +375,34 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                         lo[e] = h2(u - f.x, v - f.y);
                     }
                     const uint32_t off = (ch >> 3) * (kRows * 128) + sw128(r, ch & 7);
-                    sts128(smem + kOffQhi + off, hi[0], hi[1], hi[2], hi[3]);
-                    sts128(smem + kOffQlo + off, lo[0], lo[1], lo[2], lo[3]);
+                    sts128(qhi + off, hi[0], hi[1], hi[2], hi[3]);
+                    sts128(qlo + off, lo[0], lo[1], lo[2], lo[3]);
                 }
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) bar_arrive(&bars.q_ready);
             }
-            const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+            const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
             for (int j = 0; j < nb; ++j) {
-                const int buf = j & 1;
-                if (!bar_wait_warp(&bars.s_full[buf], (j >> 1) & 1)) { atomicOr(&bars.flags, 1); break; }
+                const int u = j & 1;
+                if (!bar_wait_warp(&bars.s_full[t][u], (j >> 1) & 1)) { atomicOr(&bars.flags, 1); break; }
                 tc_fence_after();
                 float s[kBlkTok];
-                tmem_ld32(tS0 + buf * 64 + lane_addr, s);
-                tmem_ld32(tS0 + buf * 64 + 32 + lane_addr, s + 32);
+                tmem_ld32(tS(t, u) + lane_addr, s);
+                tmem_ld32(tS(t, u) + 32 + lane_addr, s + 32);
                 const int kp0 = j * kBlkTok;
+                // interior blocks (every key visible to this row) skip the mask
+                if (kp0 + kBlkTok - 1 > qpos || kp0 + kBlkTok > kv_end) {
+#pragma unroll
+                    for (int c = 0; c < kBlkTok; ++c) {
+                        const int kp = kp0 + c;
+                        s[c] = (kp <= qpos && kp < kv_end) ? s[c] : -INFINITY;
+                    }
+                }
                 float bm = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < kBlkTok; ++c) {
-                    const int kp = kp0 + c;
-                    s[c] = (kp <= qpos && kp < kv_end) ? s[c] * isig : -INFINITY;
-                    bm = fmaxf(bm, s[c]);
-                }
+                for (int c = 0; c < kBlkTok; ++c) bm = fmaxf(bm, s[c]);
+                bm *= isig;
                 // lazy rescale: move the reference max only when it grows by > 2^8
                 const bool grow = bm > m_run + kRescaleThreshold || (m_run == -INFINITY && bm > -INFINITY);
                 bool stop = false;
@@ -381,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                     const float al = (m_run == -INFINITY) ? 0.0f : ex2(m_run - mn);
                     if (j > 0) {
                         // the previous P.V must have landed before O is rescaled
-                        if (!bar_wait_warp(&bars.pv_done[buf ^ 1], ((j - 1) >> 1) & 1)) {
+                        if (!bar_wait_warp(&bars.pv_done[t][u ^ 1], ((j - 1) >> 1) & 1)) {
                             atomicOr(&bars.flags, 1);
                             stop = true;
                         }
@@ -390,10 +420,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
 #pragma unroll 1
                             for (int cc = 0; cc < 4; ++cc) {
                                 float o[32];
-                                tmem_ld32(tO + cc * 32 + lane_addr, o);
+                                tmem_ld32(tO(t) + cc * 32 + lane_addr, o);
 #pragma unroll
                                 for (int i = 0; i < 32; ++i) o[i] *= al;
-                                tmem_st32(tO + cc * 32 + lane_addr, o);
+                                tmem_st32(tO(t) + cc * 32 + lane_addr, o);
                             }
                         }
                     }
@@ -401,34 +431,29 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                     m_run = mn;
                 }
                 if (stop) break;
-                // P tile buffer must be free: P.V(j-2) done
-                if (j >= 2 && !bar_wait_warp(&bars.pv_done[buf], ((j - 2) >> 1) & 1)) {
-                    atomicOr(&bars.flags, 1);
-                    break;
-                }
-                uint8_t* P = smem + kOffP + buf * kPBytes;
+                // probabilities, fp16, stored over the first 32 columns of the score buffer
+                const float nm = -m_run;
                 float lsum = 0.0f;
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t w[4];
+                for (int hv = 0; hv < 2; ++hv) {
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float p0 = ex2(s[8 * ch + 2 * e] - m_run), p1 = ex2(s[8 * ch + 2 * e + 1] - m_run);
+                    for (int c = 0; c < 16; ++c) {
+                        const float p0 = ex2(fmaf(s[32 * hv + 2 * c], isig, nm));
+                        const float p1 = ex2(fmaf(s[32 * hv + 2 * c + 1], isig, nm));
                         lsum += p0 + p1;
-                        w[e] = h2(p0, p1);
+                        pk[c] = h2(p0, p1);
                     }
-                    sts128(P + sw128(r, ch), w[0], w[1], w[2], w[3]);
+                    tmem_st16u(tS(t, u) + 16 * hv + lane_addr, pk);
                 }
                 l_run += lsum;
-                fence_async_smem();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) bar_arrive(&bars.p_full[buf]);
+                if (lane == 0) bar_arrive(&bars.p_full[t][u]);
             }
         } else if (warp < kMmaWarp) {
             // ------------------------------------------------------ dequant warps
-            const int dt = threadIdx.x - 32 * kWarpsSoftmax;   // 0..127
-            const int tkn = dt >> 1, half = dt & 1;            // token of the block, half of head_dim
+            const int dt = threadIdx.x - 32 * kDequantWarp0;   // 0..95
             const bool issuer = (dt == 0);
             int issued = 0;
             auto issue = [&](int j) {   // stage j % kStageN <- the pages of block j
@@ -457,61 +482,76 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                 }
                 if (!__shfl_sync(0xFFFFFFFFu, issue_ok, 0)) { atomicOr(&bars.flags, 1); break; }
                 if (!bar_wait_warp(&bars.stage_full[st], (j / kStageN) & 1)) { atomicOr(&bars.flags, 1); break; }
-                // read this thread's token row (64 dims of keys and values) from the stage
-                const int kp = j * kBlkTok + tkn;
-                const bool valid = kp < kv_end;
-                const uint8_t* T = smem + kOffStage + st * kStageBytes + (tkn >> 4) * kTile;
-                const int trow = tkn & 15;
-                uint4 kc[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-                uint4 vc[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-                uint32_t ks = 0, vs[4] = {0, 0, 0, 0};
-                if (valid) {
-                    kc[0] = *reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32);
-                    kc[1] = *reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32 + 16);
-                    ks = *reinterpret_cast<const uint32_t*>(T + kKScales + trow * 8 + half * 4);
-                    vc[0] = *reinterpret_cast<const uint4*>(T + kVCodes + trow * 64 + half * 32);
-                    vc[1] = *reinterpret_cast<const uint4*>(T + kVCodes + trow * 64 + half * 32 + 16);
+                // items (token, half of head_dim): 128 per block over 96 threads
+                constexpr int kItems = 2 * kBlkTok, kDqThreads = 32 * kWarpsDequant;
+                constexpr int kPer = (kItems + kDqThreads - 1) / kDqThreads;
+                uint4 kc[kPer][2], vc[kPer][2];
+                uint32_t ks[kPer], vs[kPer][4];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) vs[q] = T[kVScales + (half * 4 + q) * 16 + trow];
+                for (int e = 0; e < kPer; ++e) {
+                    const int it = dt + e * kDqThreads;
+                    const int tkn = it >> 1, half = it & 1;
+                    kc[e][0] = kc[e][1] = vc[e][0] = vc[e][1] = make_uint4(0, 0, 0, 0);
+                    ks[e] = 0;
+                    vs[e][0] = vs[e][1] = vs[e][2] = vs[e][3] = 0;
+                    if (it < kItems && j * kBlkTok + tkn < kv_end) {
+                        const uint8_t* T = smem + kOffStage + st * kStageBytes + (tkn >> 4) * kTile;
+                        const int trow = tkn & 15;
+                        kc[e][0] = *reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32);
+                        kc[e][1] = *reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32 + 16);
+                        ks[e] = *reinterpret_cast<const uint32_t*>(T + kKScales + trow * 8 + half * 4);
+                        vc[e][0] = *reinterpret_cast<const uint4*>(T + kVCodes + trow * 64 + half * 32);
+                        vc[e][1] = *reinterpret_cast<const uint4*>(T + kVCodes + trow * 64 + half * 32 + 16);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) vs[e][q] = T[kVScales + (half * 4 + q) * 16 + trow];
+                    }
                 }
                 __syncwarp();
                 if ((dt & 31) == 0) bar_arrive(&bars.stage_empty[st]);
-                // K/V tile buffer must be free: P.V(j-2) done
-                if (j >= 2 && !bar_wait_warp(&bars.pv_done[buf], ((j - 2) >> 1) & 1)) {
+                // K/V tile buffer must be free: both tiles' P.V(j-2) done (the commit
+                // after tile B's covers every earlier MMA)
+                if (j >= 2 && !bar_wait_warp(&bars.pv_done[kTiles - 1][buf], ((j - 2) >> 1) & 1)) {
                     atomicOr(&bars.flags, 1);
                     break;
                 }
                 uint8_t* Kt = smem + kOffK + buf * kKBytes;
                 uint8_t* Vt = smem + kOffV + buf * kVBytes;
-                // 4 blocks of 16 dims: 8 code bytes and one scale each
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t kw0 = (q < 2) ? (q == 0 ? kc[0].x : kc[0].z) : (q == 2 ? kc[1].x : kc[1].z);
-                    const uint32_t kw1 = (q < 2) ? (q == 0 ? kc[0].y : kc[0].w) : (q == 2 ? kc[1].y : kc[1].w);
-                    const uint32_t vw0 = (q < 2) ? (q == 0 ? vc[0].x : vc[0].z) : (q == 2 ? vc[1].x : vc[1].z);
-                    const uint32_t vw1 = (q < 2) ? (q == 0 ? vc[0].y : vc[0].w) : (q == 2 ? vc[1].y : vc[1].w);
-                    uint32_t ka[4], kb[4], va[4], vb[4];
-                    e2m1x8(kw0, ka);
-                    e2m1x8(kw1, kb);
-                    e2m1x8(vw0, va);
-                    e2m1x8(vw1, vb);
-                    const uint32_t ksh = e4m3x2_to_f16x2((ks >> (8 * q)) & 0xFFu) & 0xFFFFu;
-                    const uint32_t vsh = e4m3x2_to_f16x2(vs[q]) & 0xFFFFu;
-                    const uint32_t ksc = valid ? (ksh | (ksh << 16)) : 0u;
-                    const uint32_t vsc = valid ? (vsh | (vsh << 16)) : 0u;
-                    // chunk index along head_dim: 2 chunks (8 dims each) per block
-                    const int dim_chunk = half * 8 + 2 * q;          // 0..15
-                    const int plane = dim_chunk >> 3, ch = dim_chunk & 7;
-                    // keys: K-major, row = token, dims 0..63 / 64..127 in planes of 64 rows x 128 B
-                    sts128(Kt + plane * (kBlkTok * 128) + sw128(tkn, ch), hmul2u(ka[0], ksc), hmul2u(ka[1], ksc),
-                           hmul2u(ka[2], ksc), hmul2u(ka[3], ksc));
-                    sts128(Kt + plane * (kBlkTok * 128) + sw128(tkn, ch + 1), hmul2u(kb[0], ksc),
-                           hmul2u(kb[1], ksc), hmul2u(kb[2], ksc), hmul2u(kb[3], ksc));
-                    // values: MN-major, row = token (the K of P.V), 128-byte rows of 64 dims
-                    sts128(Vt + plane * (kBlkTok * 128) + sw128(tkn, ch), hmul2u(va[0], vsc), hmul2u(va[1], vsc),
-                           hmul2u(va[2], vsc), hmul2u(va[3], vsc));
-                    sts128(Vt + plane * (kBlkTok * 128) + sw128(tkn, ch + 1), hmul2u(vb[0], vsc),
-                           hmul2u(vb[1], vsc), hmul2u(vb[2], vsc), hmul2u(vb[3], vsc));
+                for (int e = 0; e < kPer; ++e) {
+                    const int it = dt + e * kDqThreads;
+                    if (it >= kItems) break;
+                    const int tkn = it >> 1, half = it & 1;
+                    const bool valid = j * kBlkTok + tkn < kv_end;
+                    // 4 blocks of 16 dims: 8 code bytes and one scale each
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4& c0 = kc[e][q >> 1];
+                        const uint4& c1 = vc[e][q >> 1];
+                        const uint32_t kw0 = (q & 1) ? c0.z : c0.x, kw1 = (q & 1) ? c0.w : c0.y;
+                        const uint32_t vw0 = (q & 1) ? c1.z : c1.x, vw1 = (q & 1) ? c1.w : c1.y;
+                        uint32_t ka[4], kb[4], va[4], vb[4];
+                        e2m1x8(kw0, ka);
+                        e2m1x8(kw1, kb);
+                        e2m1x8(vw0, va);
+                        e2m1x8(vw1, vb);
+                        const uint32_t ksh = e4m3x2_to_f16x2((ks[e] >> (8 * q)) & 0xFFu) & 0xFFFFu;
+                        const uint32_t vsh = e4m3x2_to_f16x2(vs[e][q]) & 0xFFFFu;
+                        const uint32_t ksc = valid ? (ksh | (ksh << 16)) : 0u;
+                        const uint32_t vsc = valid ? (vsh | (vsh << 16)) : 0u;
+                        // chunk index along head_dim: 2 chunks (8 dims each) per block
+                        const int dim_chunk = half * 8 + 2 * q;          // 0..15
+                        const int plane = dim_chunk >> 3, ch = dim_chunk & 7;
+                        // keys: K-major, row = token, dims 0..63 / 64..127 in planes of 64 rows x 128 B
+                        sts128(Kt + plane * (kBlkTok * 128) + sw128(tkn, ch), hmul2u(ka[0], ksc),
+                               hmul2u(ka[1], ksc), hmul2u(ka[2], ksc), hmul2u(ka[3], ksc));
+                        sts128(Kt + plane * (kBlkTok * 128) + sw128(tkn, ch + 1), hmul2u(kb[0], ksc),
+                               hmul2u(kb[1], ksc), hmul2u(kb[2], ksc), hmul2u(kb[3], ksc));
+                        // values: MN-major, row = token (the K of P.V), 128-byte rows of 64 dims
+                        sts128(Vt + plane * (kBlkTok * 128) + sw128(tkn, ch), hmul2u(va[0], vsc),
+                               hmul2u(va[1], vsc), hmul2u(va[2], vsc), hmul2u(va[3], vsc));
+                        sts128(Vt + plane * (kBlkTok * 128) + sw128(tkn, ch + 1), hmul2u(vb[0], vsc),
+                               hmul2u(vb[1], vsc), hmul2u(vb[2], vsc), hmul2u(vb[3], vsc));
+                    }
                 }
                 fence_async_smem();
                 __syncwarp();
@@ -522,7 +562,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
             // ------------------------------------------------------ MMA issuer
             const uint32_t qk = f16_idesc(kRows, kBlkTok, false);
             const uint32_t pv = f16_idesc(kRows, kD, true);
-            const uint32_t qhi = su32(smem + kOffQhi), qlo = su32(smem + kOffQlo);
             bool ok = bar_wait(&bars.q_ready, 0);
             for (int j = 0; ok && j <= nb; ++j) {
                 if (j < nb) {
@@ -530,33 +569,39 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                     if (!bar_wait(&bars.kv_full[buf], (j >> 1) & 1)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t kt = su32(smem + kOffK + buf * kKBytes);
-                    const uint32_t sd = tS0 + buf * 64;
 #pragma unroll 1
-                    for (int part = 0; part < 2; ++part) {
-                        const uint32_t qb = part ? qlo : qhi;
+                    for (int t = 0; t < kTiles; ++t) {
+                        const uint32_t sd = tS(t, buf);
+#pragma unroll 1
+                        for (int part = 0; part < 2; ++part) {
+                            const uint32_t qb = su32(smem + kOffQ + (2 * t + part) * kQBytes);
 #pragma unroll
-                        for (int s = 0; s < 8; ++s) {
-                            const uint64_t ad = sw128_desc(qb + (s >> 2) * (kRows * 128) + (s & 3) * 32, 16, 1024);
-                            const uint64_t bd = sw128_desc(kt + (s >> 2) * (kBlkTok * 128) + (s & 3) * 32, 16, 1024);
-                            mma_f16(sd, ad, bd, qk, (part | s) ? 1u : 0u);
+                            for (int s = 0; s < 8; ++s) {
+                                const uint64_t ad = sw128_desc(qb + (s >> 2) * (kRows * 128) + (s & 3) * 32, 16, 1024);
+                                const uint64_t bd = sw128_desc(kt + (s >> 2) * (kBlkTok * 128) + (s & 3) * 32, 16, 1024);
+                                mma_f16(sd, ad, bd, qk, (part | s) ? 1u : 0u);
+                            }
                         }
+                        mma_commit(&bars.s_full[t][buf]);
                     }
-                    mma_commit(&bars.s_full[buf]);
                 }
                 if (j >= 1) {
                     const int jp = j - 1, buf = jp & 1;
-                    if (!bar_wait(&bars.p_full[buf], (jp >> 1) & 1)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t pt_ = su32(smem + kOffP + buf * kPBytes);
                     const uint32_t vt = su32(smem + kOffV + buf * kVBytes);
+#pragma unroll 1
+                    for (int t = 0; t < kTiles; ++t) {
+                        if (!bar_wait(&bars.p_full[t][buf], (jp >> 1) & 1)) { ok = false; break; }
+                        tc_fence_after();
 #pragma unroll
-                    for (int s = 0; s < 4; ++s) {
-                        const uint64_t ad = sw128_desc(pt_ + s * 32, 16, 1024);
-                        // 16 tokens = two 8-row atoms (stride 1024); dims 64..127 one plane (64 x 128 B) away
-                        const uint64_t bd = sw128_desc(vt + s * 2048, kBlkTok * 128, 1024);
-                        mma_f16(tO, ad, bd, pv, (jp | s) ? 1u : 0u);
+                        for (int s = 0; s < 4; ++s) {
+                            // P: 16 tokens = 8 packed columns of the score buffer
+                            // V: 16 tokens = two 8-row atoms (stride 1024); dims 64..127 one plane away
+                            const uint64_t bd = sw128_desc(vt + s * 2048, kBlkTok * 128, 1024);
+                            mma_f16_ta(tO(t), tS(t, buf) + 8 * s, bd, pv, (jp | s) ? 1u : 0u);
+                        }
+                        mma_commit(&bars.pv_done[t][buf]);
                     }
-                    mma_commit(&bars.pv_done[buf]);
+                    if (!ok) break;
                 }
             }
             if (!ok) atomicOr(&bars.flags, 1);
@@ -567,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
     __syncthreads();
     tc_fence_after();
     const bool timed_out = bars.flags != 0;
-    if (timed_out && threadIdx.x == 32 * kWarpsSoftmax) {
+    if (timed_out && threadIdx.x == 32 * kDequantWarp0) {
         // drain: the packed-page copies still in flight
         const int issued = bars.issued;
         for (int j = max(0, issued - kStageN); j < issued; ++j)
@@ -586,21 +631,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
     // run on every lane of a softmax warp or on none)
     const bool dead = poison || timed_out || nb == 0;
     if (warp < kWarpsSoftmax) {
-        const int r = threadIdx.x;
+        const int t = warp >> 2;
+        const int r = threadIdx.x & 127;
         const int head = r >> 5, tok = r & 31;
-        const int qi = q0 + tok;
+        const int qi = q0 + t * kQTok + tok;
         float res[kD];
         if (!dead) {
-            // the last P.V has landed once pv_done of the last block completes
+            // the last P.V of this tile has landed once its pv_done completes
             const int jl = nb - 1;
-            const bool ok = bar_wait_warp(&bars.pv_done[jl & 1], (jl >> 1) & 1);
+            const bool ok = bar_wait_warp(&bars.pv_done[t][jl & 1], (jl >> 1) & 1);
             tc_fence_after();
-            const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+            const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
             const float sc = (ok && l_run > 0.0f) ? __ldg(a.gv + li) / l_run : 0.0f;
-#pragma unroll 1
+#pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
                 float o[32];
-                tmem_ld32(tO + cc * 32 + lane_addr, o);
+                tmem_ld32(tO(t) + cc * 32 + lane_addr, o);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) res[cc * 32 + i] = ok ? o[i] * sc : 0.0f;
             }
@@ -609,7 +655,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
 #pragma unroll
             for (int i = 0; i < kD; ++i) res[i] = 0.0f;
         }
-        if (head < a.G && tok < qn) {
+        if (head < a.G && (t * kQTok + tok) < qn) {
             TO* dst = reinterpret_cast<TO*>(a.out) +
                       ((((size_t)li * a.batch + b) * a.q_len + qi) * a.Hq + h * a.G + head) * kD;
             if constexpr (sizeof(TO) == 4) {
@@ -657,7 +703,7 @@ static cudaError_t launch_prefill(const AttnArgs& a, dim3 grid, bool qb, bool ob
 }
 
 cudaError_t launch_prefill_tc(const AttnArgs& a, int nlayers, bool q_bf16, bool out_bf16, cudaStream_t st) {
-    dim3 grid((a.q_len + kQTok - 1) / kQTok, a.batch * a.Hkv, nlayers);
+    dim3 grid((a.q_len + kTiles * kQTok - 1) / (kTiles * kQTok), a.batch * a.Hkv, nlayers);
     return launch_prefill(a, grid, q_bf16, out_bf16, st);
 }
 
