@@ -231,7 +231,8 @@ struct PrefillBars {
     uint64_t q_ready;                 // both softmax warpgroups wrote their query tiles (count 8)
     uint64_t stage_full[kStageN];     // packed pages landed (tx bytes)
     uint64_t stage_empty[kStageN];    // dequant warps read the stage (count 3)
-    uint64_t kv_full[2];              // K/V tile j%2 written (count 3)
+    uint64_t k_full[2];               // K tile j%2 written (count 3)
+    uint64_t v_full[2];               // V tile j%2 written (count 3)
     uint64_t s_full[kTiles][2];       // QK(tile, j) done (commit)
     uint64_t p_full[kTiles][2];       // P(tile, j) stored in TMEM, O rescaled (count 4)
     uint64_t pv_done[kTiles][2];      // PV(tile, j) done (commit)
@@ -273,7 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
             bar_init(&bars.stage_empty[i], kWarpsDequant);
         }
         for (int i = 0; i < 2; ++i) {
-            bar_init(&bars.kv_full[i], kWarpsDequant);
+            bar_init(&bars.k_full[i], kWarpsDequant);
+            bar_init(&bars.v_full[i], kWarpsDequant);
             for (int t = 0; t < kTiles; ++t) {
                 bar_init(&bars.s_full[t][i], 1);
                 bar_init(&bars.p_full[t][i], 4);
@@ -508,14 +510,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                 }
                 __syncwarp();
                 if ((dt & 31) == 0) bar_arrive(&bars.stage_empty[st]);
-                // K/V tile buffer must be free: both tiles' P.V(j-2) done (the commit
-                // after tile B's covers every earlier MMA)
-                if (j >= 2 && !bar_wait_warp(&bars.pv_done[kTiles - 1][buf], ((j - 2) >> 1) & 1)) {
+                // K tile buffer: free once both tiles' Q.K(j-2) are done (the
+                // commit after tile B's covers every earlier MMA)
+                if (j >= 2 && !bar_wait_warp(&bars.s_full[kTiles - 1][buf], ((j - 2) >> 1) & 1)) {
                     atomicOr(&bars.flags, 1);
                     break;
                 }
                 uint8_t* Kt = smem + kOffK + buf * kKBytes;
                 uint8_t* Vt = smem + kOffV + buf * kVBytes;
+                uint32_t vsc[kPer][4];
 #pragma unroll
                 for (int e = 0; e < kPer; ++e) {
                     const int it = dt + e * kDqThreads;
@@ -526,18 +529,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const uint4& c0 = kc[e][q >> 1];
-                        const uint4& c1 = vc[e][q >> 1];
                         const uint32_t kw0 = (q & 1) ? c0.z : c0.x, kw1 = (q & 1) ? c0.w : c0.y;
-                        const uint32_t vw0 = (q & 1) ? c1.z : c1.x, vw1 = (q & 1) ? c1.w : c1.y;
-                        uint32_t ka[4], kb[4], va[4], vb[4];
+                        uint32_t ka[4], kb[4];
                         e2m1x8(kw0, ka);
                         e2m1x8(kw1, kb);
-                        e2m1x8(vw0, va);
-                        e2m1x8(vw1, vb);
                         const uint32_t ksh = e4m3x2_to_f16x2((ks[e] >> (8 * q)) & 0xFFu) & 0xFFFFu;
                         const uint32_t vsh = e4m3x2_to_f16x2(vs[e][q]) & 0xFFFFu;
                         const uint32_t ksc = valid ? (ksh | (ksh << 16)) : 0u;
-                        const uint32_t vsc = valid ? (vsh | (vsh << 16)) : 0u;
+                        vsc[e][q] = valid ? (vsh | (vsh << 16)) : 0u;
                         // chunk index along head_dim: 2 chunks (8 dims each) per block
                         const int dim_chunk = half * 8 + 2 * q;          // 0..15
                         const int plane = dim_chunk >> 3, ch = dim_chunk & 7;
@@ -546,59 +545,95 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                                hmul2u(ka[1], ksc), hmul2u(ka[2], ksc), hmul2u(ka[3], ksc));
                         sts128(Kt + plane * (kBlkTok * 128) + sw128(tkn, ch + 1), hmul2u(kb[0], ksc),
                                hmul2u(kb[1], ksc), hmul2u(kb[2], ksc), hmul2u(kb[3], ksc));
-                        // values: MN-major, row = token (the K of P.V), 128-byte rows of 64 dims
-                        sts128(Vt + plane * (kBlkTok * 128) + sw128(tkn, ch), hmul2u(va[0], vsc),
-                               hmul2u(va[1], vsc), hmul2u(va[2], vsc), hmul2u(va[3], vsc));
-                        sts128(Vt + plane * (kBlkTok * 128) + sw128(tkn, ch + 1), hmul2u(vb[0], vsc),
-                               hmul2u(vb[1], vsc), hmul2u(vb[2], vsc), hmul2u(vb[3], vsc));
                     }
                 }
                 fence_async_smem();
                 __syncwarp();
-                if ((dt & 31) == 0) bar_arrive(&bars.kv_full[buf]);
+                if ((dt & 31) == 0) bar_arrive(&bars.k_full[buf]);
+                // V tile buffer: free once both tiles' P.V(j-2) are done
+                if (j >= 2 && !bar_wait_warp(&bars.pv_done[kTiles - 1][buf], ((j - 2) >> 1) & 1)) {
+                    atomicOr(&bars.flags, 1);
+                    break;
+                }
+#pragma unroll
+                for (int e = 0; e < kPer; ++e) {
+                    const int it = dt + e * kDqThreads;
+                    if (it >= kItems) break;
+                    const int tkn = it >> 1, half = it & 1;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4& c1 = vc[e][q >> 1];
+                        const uint32_t vw0 = (q & 1) ? c1.z : c1.x, vw1 = (q & 1) ? c1.w : c1.y;
+                        uint32_t va[4], vb[4];
+                        e2m1x8(vw0, va);
+                        e2m1x8(vw1, vb);
+                        const uint32_t sc = vsc[e][q];
+                        const int dim_chunk = half * 8 + 2 * q;
+                        const int plane = dim_chunk >> 3, ch = dim_chunk & 7;
+                        // values: MN-major, row = token (the K of P.V), 128-byte rows of 64 dims
+                        sts128(Vt + plane * (kBlkTok * 128) + sw128(tkn, ch), hmul2u(va[0], sc), hmul2u(va[1], sc),
+                               hmul2u(va[2], sc), hmul2u(va[3], sc));
+                        sts128(Vt + plane * (kBlkTok * 128) + sw128(tkn, ch + 1), hmul2u(vb[0], sc),
+                               hmul2u(vb[1], sc), hmul2u(vb[2], sc), hmul2u(vb[3], sc));
+                    }
+                }
+                fence_async_smem();
+                __syncwarp();
+                if ((dt & 31) == 0) bar_arrive(&bars.v_full[buf]);
             }
             if (issuer) bars.issued = issued;
         } else if (lane == 0) {
             // ------------------------------------------------------ MMA issuer
+            // Descriptors are built once; a k-step only advances the 14-bit
+            // start-address field (16-byte units) by a constant, which never
+            // carries out of the field for shared-memory addresses.
             const uint32_t qk = f16_idesc(kRows, kBlkTok, false);
             const uint32_t pv = f16_idesc(kRows, kD, true);
+            uint64_t qd[kTiles][2], kd[2], vd[2];
+#pragma unroll
+            for (int t = 0; t < kTiles; ++t)
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+                    qd[t][part] = sw128_desc(su32(smem + kOffQ + (2 * t + part) * kQBytes), 16, 1024);
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                kd[u] = sw128_desc(su32(smem + kOffK + u * kKBytes), 16, 1024);
+                vd[u] = sw128_desc(su32(smem + kOffV + u * kVBytes), kBlkTok * 128, 1024);
+            }
             bool ok = bar_wait(&bars.q_ready, 0);
             for (int j = 0; ok && j <= nb; ++j) {
                 if (j < nb) {
                     const int buf = j & 1;
-                    if (!bar_wait(&bars.kv_full[buf], (j >> 1) & 1)) { ok = false; break; }
+                    if (!bar_wait(&bars.k_full[buf], (j >> 1) & 1)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t kt = su32(smem + kOffK + buf * kKBytes);
-#pragma unroll 1
+                    const uint64_t kb = kd[buf];
+#pragma unroll
                     for (int t = 0; t < kTiles; ++t) {
                         const uint32_t sd = tS(t, buf);
-#pragma unroll 1
-                        for (int part = 0; part < 2; ++part) {
-                            const uint32_t qb = su32(smem + kOffQ + (2 * t + part) * kQBytes);
 #pragma unroll
-                            for (int s = 0; s < 8; ++s) {
-                                const uint64_t ad = sw128_desc(qb + (s >> 2) * (kRows * 128) + (s & 3) * 32, 16, 1024);
-                                const uint64_t bd = sw128_desc(kt + (s >> 2) * (kBlkTok * 128) + (s & 3) * 32, 16, 1024);
-                                mma_f16(sd, ad, bd, qk, (part | s) ? 1u : 0u);
-                            }
-                        }
+                        for (int part = 0; part < 2; ++part)
+#pragma unroll
+                            for (int s = 0; s < 8; ++s)
+                                mma_f16(sd, qd[t][part] + (uint64_t)(((s >> 2) * (kRows * 128) + (s & 3) * 32) >> 4),
+                                        kb + (uint64_t)(((s >> 2) * (kBlkTok * 128) + (s & 3) * 32) >> 4), qk,
+                                        (part | s) ? 1u : 0u);
                         mma_commit(&bars.s_full[t][buf]);
                     }
                 }
                 if (j >= 1) {
                     const int jp = j - 1, buf = jp & 1;
-                    const uint32_t vt = su32(smem + kOffV + buf * kVBytes);
-#pragma unroll 1
+                    const uint64_t vb = vd[buf];
+                    if (!bar_wait(&bars.v_full[buf], (jp >> 1) & 1)) { ok = false; break; }
+#pragma unroll
                     for (int t = 0; t < kTiles; ++t) {
                         if (!bar_wait(&bars.p_full[t][buf], (jp >> 1) & 1)) { ok = false; break; }
                         tc_fence_after();
+                        // P: 16 tokens = 8 packed columns of the score buffer;
+                        // V: 16 tokens = two 8-row atoms (2048 bytes)
 #pragma unroll
-                        for (int s = 0; s < 4; ++s) {
-                            // P: 16 tokens = 8 packed columns of the score buffer
-                            // V: 16 tokens = two 8-row atoms (stride 1024); dims 64..127 one plane away
-                            const uint64_t bd = sw128_desc(vt + s * 2048, kBlkTok * 128, 1024);
-                            mma_f16_ta(tO(t), tS(t, buf) + 8 * s, bd, pv, (jp | s) ? 1u : 0u);
-                        }
+                        for (int s = 0; s < 4; ++s)
+                            mma_f16_ta(tO(t), tS(t, buf) + 8 * s, vb + (uint64_t)((s * 2048) >> 4), pv,
+                                       (jp | s) ? 1u : 0u);
                         mma_commit(&bars.pv_done[t][buf]);
                     }
                     if (!ok) break;
