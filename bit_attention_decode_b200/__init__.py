@@ -76,6 +76,8 @@ _lib.kvq_prefill_attention.argtypes = [_SHP, _CAL, _CCH, _I32, _I32, _P, _I32, _
 _lib.kvq_decode_attention_noalloc.restype = _I32
 _lib.kvq_decode_attention_noalloc.argtypes = [_SHP, _CAL, _CCH, _I32, _I32, _P, _I32, _P, _I32, _P, _I32, _P,
                                               _I32, _P, _P]
+_lib.kvq_selftest_wait_timeout.restype = _I32
+_lib.kvq_selftest_wait_timeout.argtypes = [_P, ctypes.c_int64, _P]
 _lib.kvq_round_e2m1.restype = _I32
 _lib.kvq_round_e2m1.argtypes = [_P, _P, ctypes.c_int64, _P]
 _lib.kvq_round_e4m3.restype = _I32
@@ -84,7 +86,7 @@ _lib.kvq_round_e4m3.argtypes = [_P, _P, ctypes.c_int64, _P]
 EXPORTED = ("kvq_page_bytes", "kvq_status_string", "kvq_version", "kvq_calibrate_smoothing",
             "kvq_quantize_append", "kvq_decode_workspace_bytes", "kvq_decode_attention",
             "kvq_prefill_workspace_bytes", "kvq_prefill_attention", "kvq_decode_attention_noalloc",
-            "kvq_round_e2m1", "kvq_round_e4m3")
+            "kvq_round_e2m1", "kvq_round_e4m3", "kvq_selftest_wait_timeout")
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -283,6 +285,12 @@ def prefill_attention(shape: Shape, calib: Calibration, cache: PagedCache, q: to
                                       _dtype_code(out), _ptr(workspace), ws_bytes, _ptr(status), _stream()),
            "kvq_prefill_attention")
     return out
+
+
+def selftest_wait_timeout(status: torch.Tensor, limit_ns: int = 20_000_000):
+    """Run the bounded-wait self-test: ORs DEV_TIMEOUT into ``status`` (int32, device)."""
+    _need_cuda(status)
+    _check(_lib.kvq_selftest_wait_timeout(status.data_ptr(), int(limit_ns), _stream()), "kvq_selftest_wait_timeout")
 
 
 def round_e2m1(x: torch.Tensor) -> torch.Tensor:

@@ -163,6 +163,12 @@ kvq_status kvq_prefill_attention(const kvq_shape* shape, const kvq_calib* calib,
                         dev_status, (cudaStream_t)stream);
 }
 
+kvq_status kvq_selftest_wait_timeout(int32_t* dev_status, int64_t limit_ns, void* stream) {
+    if (!dev_status || limit_ns < 1000 || limit_ns > 10000000000LL) return KVQ_EINVAL;
+    KVQ_TRY(check_device());
+    return kvq::selftest_wait_timeout(dev_status, (long long)limit_ns, (cudaStream_t)stream);
+}
+
 kvq_status kvq_round_e2m1(const float* x, uint8_t* codes, int64_t n, void* stream) {
     if (n < 0 || (n > 0 && (!x || !codes))) return KVQ_EINVAL;
     if (n == 0) return KVQ_OK;

@@ -33,6 +33,7 @@
 #include "kvq_attn.cuh"
 #include "kvq_common.cuh"
 #include "kvq_internal.h"
+#include "kvq_sync.cuh"
 
 namespace kvq {
 namespace {
@@ -43,7 +44,6 @@ constexpr int kTiles = 2;           // query tiles per CTA (A, B)
 constexpr int kBlkTok = 64;         // key tokens per block (4 pages)
 constexpr int kStageN = 3;          // packed-page staging stages
 constexpr uint32_t kTmemCols = 512; // O_A, O_B [0,256), S_A[2] [256,384), S_B[2] [384,512)
-constexpr unsigned long long kWaitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 // shared memory map (offsets from a 1024-aligned base)
@@ -64,45 +64,6 @@ constexpr int kMmaWarp = kWarpsSoftmax + kWarpsDequant;        // warp 11
 constexpr int kThreads = 32 * (kMmaWarp + 1);
 
 // ------------------------------------------------------------------ primitives
-__device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-__device__ __forceinline__ void bar_init(uint64_t* b, uint32_t n) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(n));
-}
-__device__ __forceinline__ void bar_arrive(uint64_t* b) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
-}
-__device__ __forceinline__ void bar_expect(uint64_t* b, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool bar_try(uint64_t* b, uint32_t parity) {
-    uint32_t ok;
-    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-                 : "=r"(ok) : "r"(su32(b)), "r"(parity) : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ unsigned long long now_ns() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-// bounded wait; false when it ran out
-__device__ __forceinline__ bool bar_wait(uint64_t* b, uint32_t parity) {
-    if (bar_try(b, parity)) return true;
-    const unsigned long long t0 = now_ns();
-    for (;;) {
-        for (int i = 0; i < 64; ++i)
-            if (bar_try(b, parity)) return true;
-        if (now_ns() - t0 > kWaitNs) return false;
-    }
-}
-// every lane of the warp waits; the outcome is made uniform across the warp
-__device__ __forceinline__ bool bar_wait_warp(uint64_t* b, uint32_t parity) {
-    return __all_sync(0xFFFFFFFFu, bar_wait(b, parity));
-}
-__device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, uint64_t* b) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(su32(dst)), "l"(src), "r"(bytes), "r"(su32(b)) : "memory");
-}
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -134,7 +95,7 @@ __device__ __forceinline__ void mma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uin
                  ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc) : "memory");
 }
 __device__ __forceinline__ void mma_commit(uint64_t* b) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(b))
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(b))
                  : "memory");
 }
 // 32 consecutive fp32 columns of this thread's TMEM lane
@@ -268,21 +229,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
     if (threadIdx.x == 0) {
         bars.flags = 0;
         bars.issued = 0;
-        bar_init(&bars.q_ready, kWarpsSoftmax);
+        mbar_init(&bars.q_ready, kWarpsSoftmax);
         for (int i = 0; i < kStageN; ++i) {
-            bar_init(&bars.stage_full[i], 1);
-            bar_init(&bars.stage_empty[i], kWarpsDequant);
+            mbar_init(&bars.stage_full[i], 1);
+            mbar_init(&bars.stage_empty[i], kWarpsDequant);
         }
         for (int i = 0; i < 2; ++i) {
-            bar_init(&bars.k_full[i], kWarpsDequant);
-            bar_init(&bars.v_full[i], kWarpsDequant);
+            mbar_init(&bars.k_full[i], kWarpsDequant);
+            mbar_init(&bars.v_full[i], kWarpsDequant);
             for (int t = 0; t < kTiles; ++t) {
-                bar_init(&bars.s_full[t][i], 1);
-                bar_init(&bars.p_full[t][i], 4);
-                bar_init(&bars.pv_done[t][i], 1);
+                mbar_init(&bars.s_full[t][i], 1);
+                mbar_init(&bars.p_full[t][i], 4);
+                mbar_init(&bars.pv_done[t][i], 1);
             }
         }
-        bar_init(&bars.drain, 1);
+        mbar_init(&bars.drain, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     int badp = 0;
@@ -299,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
 
     // TMEM: one warp allocates all 512 columns for the CTA (one CTA per SM)
     if (warp == kMmaWarp) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&bars.tmem_base)),
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&bars.tmem_base)),
                      "r"(kTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -382,12 +343,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                 }
                 fence_async_smem();
                 __syncwarp();
-                if (lane == 0) bar_arrive(&bars.q_ready);
+                if (lane == 0) mbar_arrive(&bars.q_ready);
             }
             const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
             for (int j = 0; j < nb; ++j) {
                 const int u = j & 1;
-                if (!bar_wait_warp(&bars.s_full[t][u], (j >> 1) & 1)) { atomicOr(&bars.flags, 1); break; }
+                if (!mbar_wait_warp(&bars.s_full[t][u], (j >> 1) & 1)) { atomicOr(&bars.flags, 1); break; }
                 tc_fence_after();
                 float s[kBlkTok];
                 tmem_ld32(tS(t, u) + lane_addr, s);
@@ -413,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                     const float al = (m_run == -INFINITY) ? 0.0f : ex2(m_run - mn);
                     if (j > 0) {
                         // the previous P.V must have landed before O is rescaled
-                        if (!bar_wait_warp(&bars.pv_done[t][u ^ 1], ((j - 1) >> 1) & 1)) {
+                        if (!mbar_wait_warp(&bars.pv_done[t][u ^ 1], ((j - 1) >> 1) & 1)) {
                             atomicOr(&bars.flags, 1);
                             stop = true;
                         }
@@ -451,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                 l_run += lsum;
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) bar_arrive(&bars.p_full[t][u]);
+                if (lane == 0) mbar_arrive(&bars.p_full[t][u]);
             }
         } else if (warp < kMmaWarp) {
             // ------------------------------------------------------ dequant warps
@@ -461,10 +422,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
             auto issue = [&](int j) {   // stage j % kStageN <- the pages of block j
                 const int st = j % kStageN;
                 const int p_lo = j * 4, p_hi = min(npg, p_lo + 4);
-                bar_expect(&bars.stage_full[st], (uint32_t)(p_hi - p_lo) * kTile);
+                mbar_arrive_expect_tx(&bars.stage_full[st], (uint32_t)(p_hi - p_lo) * kTile);
                 for (int p = p_lo; p < p_hi; ++p) {
                     const int pg = __ldg(pt + p);
-                    bulk_copy(smem + kOffStage + st * kStageBytes + (p - p_lo) * kTile,
+                    bulk_g2s(smem + kOffStage + st * kStageBytes + (p - p_lo) * kTile,
                               layer_base + ((size_t)pg * a.Hkv + h) * kTile, kTile, &bars.stage_full[st]);
                 }
             };
@@ -475,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                 int issue_ok = 1;
                 if (issuer && issued < nb) {
                     if (issued >= kStageN &&
-                        !bar_wait(&bars.stage_empty[issued % kStageN], ((issued / kStageN) - 1) & 1)) {
+                        !mbar_wait(&bars.stage_empty[issued % kStageN], ((issued / kStageN) - 1) & 1)) {
                         issue_ok = 0;
                     } else {
                         issue(issued);
@@ -483,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                     }
                 }
                 if (!__shfl_sync(0xFFFFFFFFu, issue_ok, 0)) { atomicOr(&bars.flags, 1); break; }
-                if (!bar_wait_warp(&bars.stage_full[st], (j / kStageN) & 1)) { atomicOr(&bars.flags, 1); break; }
+                if (!mbar_wait_warp(&bars.stage_full[st], (j / kStageN) & 1)) { atomicOr(&bars.flags, 1); break; }
                 // items (token, half of head_dim): 128 per block over 96 threads
                 constexpr int kItems = 2 * kBlkTok, kDqThreads = 32 * kWarpsDequant;
                 constexpr int kPer = (kItems + kDqThreads - 1) / kDqThreads;
@@ -509,10 +470,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                     }
                 }
                 __syncwarp();
-                if ((dt & 31) == 0) bar_arrive(&bars.stage_empty[st]);
+                if ((dt & 31) == 0) mbar_arrive(&bars.stage_empty[st]);
                 // K tile buffer: free once both tiles' Q.K(j-2) are done (the
                 // commit after tile B's covers every earlier MMA)
-                if (j >= 2 && !bar_wait_warp(&bars.s_full[kTiles - 1][buf], ((j - 2) >> 1) & 1)) {
+                if (j >= 2 && !mbar_wait_warp(&bars.s_full[kTiles - 1][buf], ((j - 2) >> 1) & 1)) {
                     atomicOr(&bars.flags, 1);
                     break;
                 }
@@ -549,9 +510,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                 }
                 fence_async_smem();
                 __syncwarp();
-                if ((dt & 31) == 0) bar_arrive(&bars.k_full[buf]);
+                if ((dt & 31) == 0) mbar_arrive(&bars.k_full[buf]);
                 // V tile buffer: free once both tiles' P.V(j-2) are done
-                if (j >= 2 && !bar_wait_warp(&bars.pv_done[kTiles - 1][buf], ((j - 2) >> 1) & 1)) {
+                if (j >= 2 && !mbar_wait_warp(&bars.pv_done[kTiles - 1][buf], ((j - 2) >> 1) & 1)) {
                     atomicOr(&bars.flags, 1);
                     break;
                 }
@@ -579,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                 }
                 fence_async_smem();
                 __syncwarp();
-                if ((dt & 31) == 0) bar_arrive(&bars.v_full[buf]);
+                if ((dt & 31) == 0) mbar_arrive(&bars.v_full[buf]);
             }
             if (issuer) bars.issued = issued;
         } else if (lane == 0) {
@@ -594,17 +555,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
             for (int t = 0; t < kTiles; ++t)
 #pragma unroll
                 for (int part = 0; part < 2; ++part)
-                    qd[t][part] = sw128_desc(su32(smem + kOffQ + (2 * t + part) * kQBytes), 16, 1024);
+                    qd[t][part] = sw128_desc(smem_u32(smem + kOffQ + (2 * t + part) * kQBytes), 16, 1024);
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
-                kd[u] = sw128_desc(su32(smem + kOffK + u * kKBytes), 16, 1024);
-                vd[u] = sw128_desc(su32(smem + kOffV + u * kVBytes), kBlkTok * 128, 1024);
+                kd[u] = sw128_desc(smem_u32(smem + kOffK + u * kKBytes), 16, 1024);
+                vd[u] = sw128_desc(smem_u32(smem + kOffV + u * kVBytes), kBlkTok * 128, 1024);
             }
-            bool ok = bar_wait(&bars.q_ready, 0);
+            bool ok = mbar_wait(&bars.q_ready, 0);
             for (int j = 0; ok && j <= nb; ++j) {
                 if (j < nb) {
                     const int buf = j & 1;
-                    if (!bar_wait(&bars.k_full[buf], (j >> 1) & 1)) { ok = false; break; }
+                    if (!mbar_wait(&bars.k_full[buf], (j >> 1) & 1)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t kb = kd[buf];
 #pragma unroll
@@ -623,10 +584,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                 if (j >= 1) {
                     const int jp = j - 1, buf = jp & 1;
                     const uint64_t vb = vd[buf];
-                    if (!bar_wait(&bars.v_full[buf], (jp >> 1) & 1)) { ok = false; break; }
+                    if (!mbar_wait(&bars.v_full[buf], (jp >> 1) & 1)) { ok = false; break; }
 #pragma unroll
                     for (int t = 0; t < kTiles; ++t) {
-                        if (!bar_wait(&bars.p_full[t][buf], (jp >> 1) & 1)) { ok = false; break; }
+                        if (!mbar_wait(&bars.p_full[t][buf], (jp >> 1) & 1)) { ok = false; break; }
                         tc_fence_after();
                         // P: 16 tokens = 8 packed columns of the score buffer;
                         // V: 16 tokens = two 8-row atoms (2048 bytes)
@@ -651,14 +612,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
         // drain: the packed-page copies still in flight
         const int issued = bars.issued;
         for (int j = max(0, issued - kStageN); j < issued; ++j)
-            (void)bar_wait(&bars.stage_full[j % kStageN], (j / kStageN) & 1);
+            (void)mbar_wait(&bars.stage_full[j % kStageN], (j / kStageN) & 1);
         set_status(a.status, KVQ_DEV_TIMEOUT);
     }
     if (timed_out && threadIdx.x == 32 * kMmaWarp) {
         // drain: every MMA issued by this thread completes before the commit
         // arrives; TMEM is freed only after that
         mma_commit(&bars.drain);
-        (void)bar_wait(&bars.drain, 0);
+        (void)mbar_wait(&bars.drain, 0);
     }
 
     // ---------------------------------------------------------------- epilogue
@@ -674,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
         if (!dead) {
             // the last P.V of this tile has landed once its pv_done completes
             const int jl = nb - 1;
-            const bool ok = bar_wait_warp(&bars.pv_done[t][jl & 1], (jl >> 1) & 1);
+            const bool ok = mbar_wait_warp(&bars.pv_done[t][jl & 1], (jl >> 1) & 1);
             tc_fence_after();
             const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
             const float sc = (ok && l_run > 0.0f) ? __ldg(a.gv + li) / l_run : 0.0f;

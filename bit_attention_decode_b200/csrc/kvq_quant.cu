@@ -10,6 +10,7 @@
 // E4M3 scale per 16, FP32 tensor scale).
 #include "kvq_common.cuh"
 #include "kvq_internal.h"
+#include "kvq_sync.cuh"
 
 namespace kvq {
 
@@ -115,29 +116,6 @@ __device__ __forceinline__ void quantize_block(const float* y, float g, float en
 // cross-lane butterflies stay uniform.
 constexpr int kAppendStages = 3;
 constexpr int kAppendStageBytes = 32768;   // key + value rows of one chunk
-constexpr unsigned long long kAppendWaitNs = 2000000000ull;
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ bool append_wait(uint64_t* bar, uint32_t parity) {
-    auto try_wait = [&]() {
-        uint32_t ok;
-        asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-                     : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
-        return ok != 0;
-    };
-    if (try_wait()) return true;
-    unsigned long long t0;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
-    for (;;) {
-        for (int i = 0; i < 64; ++i)
-            if (try_wait()) return true;
-        unsigned long long t;
-        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-        if (t - t0 > kAppendWaitNs) return false;
-    }
-}
 
 template <typename T>
 __device__ __forceinline__ void load16_smem(const T* p, float* x);
@@ -184,8 +162,8 @@ append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* _
         s_timeout = 0;
         s_issued = 0;
         for (int i = 0; i < kAppendStages; ++i) {
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&full[i])));
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(&empty[i])), "r"(workers));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&full[i])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&empty[i])), "r"(workers));
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -197,7 +175,7 @@ append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* _
             int j = 0;
             for (; j < mine; ++j) {
                 const int st = j % kAppendStages;
-                if (j >= kAppendStages && !append_wait(&empty[st], ((j / kAppendStages) - 1) & 1)) {
+                if (j >= kAppendStages && !mbar_wait(&empty[st], ((j / kAppendStages) - 1) & 1)) {
                     atomicOr(&s_timeout, 1);
                     break;
                 }
@@ -207,12 +185,12 @@ append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* _
                 const uint32_t bytes = (uint32_t)n * row * sizeof(T);
                 uint8_t* dst = smem + st * kAppendStageBytes;
                 const size_t off = ((size_t)li * num_tokens + t0) * row;
-                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(&full[st])),
+                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&full[st])),
                              "r"(2 * bytes) : "memory");
                 asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                             ::"r"(smem_addr(dst)), "l"(k + off), "r"(bytes), "r"(smem_addr(&full[st])) : "memory");
+                             ::"r"(smem_u32(dst)), "l"(k + off), "r"(bytes), "r"(smem_u32(&full[st])) : "memory");
                 asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                             ::"r"(smem_addr(dst + half_stage)), "l"(v + off), "r"(bytes), "r"(smem_addr(&full[st]))
+                             ::"r"(smem_u32(dst + half_stage)), "l"(v + off), "r"(bytes), "r"(smem_u32(&full[st]))
                              : "memory");
             }
             s_issued = j;
@@ -242,7 +220,7 @@ append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* _
             const float enc_k = __frcp_rn(__fmul_rn(6.0f, g_k)), enc_v = __frcp_rn(__fmul_rn(6.0f, g_v));
             uint8_t* layer_cache = cache + (size_t)li * layer_stride;
             const int st = j % kAppendStages;
-            if (!append_wait(&full[st], (j / kAppendStages) & 1)) {
+            if (!mbar_wait(&full[st], (j / kAppendStages) & 1)) {
                 atomicOr(&s_timeout, 1);
                 break;
             }
@@ -280,7 +258,7 @@ append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* _
             }
             __syncwarp();
             if ((threadIdx.x & 31) == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(
-                                                          smem_addr(&empty[st])) : "memory");
+                                                          smem_u32(&empty[st])) : "memory");
         }
     }
     __syncthreads();
@@ -288,7 +266,7 @@ append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* _
         // wait (bounded) for the copies still in flight before leaving
         const int issued = s_issued;
         for (int j = max(0, issued - kAppendStages); j < issued; ++j)
-            (void)append_wait(&full[j % kAppendStages], (j / kAppendStages) & 1);
+            (void)mbar_wait(&full[j % kAppendStages], (j / kAppendStages) & 1);
         set_status(status, KVQ_DEV_TIMEOUT);
     }
 }

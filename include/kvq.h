@@ -259,6 +259,17 @@ kvq_status kvq_decode_attention_noalloc(const kvq_shape* shape, const kvq_calib*
 kvq_status kvq_round_e2m1(const float* x, uint8_t* codes, int64_t n, void* stream);
 kvq_status kvq_round_e4m3(const float* x, uint8_t* codes, int64_t n, void* stream);
 
+/*
+ * kvq_selftest_wait_timeout -- failure-detection self-test.  Launches one
+ * small kernel that runs the library's bounded shared-memory-barrier wait
+ * (the one every copy hand-off in the attention and append kernels uses) on
+ * a barrier nothing ever arrives at.  The wait gives up after limit_ns
+ * nanoseconds (1 us .. 10 s) and ORs KVQ_DEV_TIMEOUT into *dev_status; no
+ * fault is raised and the context stays usable.
+ * Errors: KVQ_EINVAL for a null status or a limit out of range.
+ */
+kvq_status kvq_selftest_wait_timeout(int32_t* dev_status, int64_t limit_ns, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

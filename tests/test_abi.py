@@ -83,6 +83,14 @@ def test_host_validation_rejects_before_launch(kvq_lib):
     assert _call_decode(kvq, s, ws_bytes=need - 1) == kvq.KVQ_EWORKSPACE
 
 
+def test_selftest_validation(kvq_lib):
+    kvq = kvq_lib
+    f = kvq._lib.kvq_selftest_wait_timeout
+    assert f(None, 1_000_000, None) == kvq.KVQ_EINVAL
+    assert f(256, 10, None) == kvq.KVQ_EINVAL                   # limit below 1 us
+    assert f(256, 10 ** 12, None) == kvq.KVQ_EINVAL             # limit above 10 s
+
+
 def test_append_validation(kvq_lib):
     kvq = kvq_lib
     s = kvq.Shape(1, 32, 8)

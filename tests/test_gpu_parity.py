@@ -162,3 +162,22 @@ def test_device_faults_are_flagged_not_trapped(kvq):
     assert status.item() & kvq.DEV_BAD_SLOT
     changed = (p.cache.data != before).nonzero()
     assert changed.numel() > 0 and torch.all(changed[:, 1] == 0)           # only page 0 (slot 5) touched
+
+
+def test_bounded_wait_gives_up_and_context_survives(kvq):
+    """A wait on a barrier nothing arrives at runs out and reports DEV_TIMEOUT."""
+    import time
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.perf_counter()
+    kvq.selftest_wait_timeout(status, limit_ns=20_000_000)   # 20 ms
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    assert status.item() == kvq.DEV_TIMEOUT
+    assert dt < 5.0
+    # the context is still usable: a normal decode afterwards is correct
+    w = small(num_layers=1, batch=1, calib_windows=1, calib_len=32)
+    p = harness.build_problem(kvq, w, lens=[50])
+    cal = harness.oracle_calibration(p)
+    q, out = decode_all(kvq, p)
+    want = harness.oracle_attend(p, 0, 0, q[0, 0][None], 49, 50, cal)
+    harness.check_attention(out[0, 0], want[0], "decode after a timed-out wait f32")
