@@ -150,6 +150,39 @@ __device__ __forceinline__ void e2m1x8(uint32_t w, uint32_t* r) {
         "  cvt.rn.f16x2.e2m1x2 %2, b2; cvt.rn.f16x2.e2m1x2 %3, b3; }"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(w));
 }
+// 2^x on the FMA pipe, for the share of the softmax exponentials taken off
+// the MUFU unit.  x = n + f with n = floor(x) (a round-down add of 1.5 * 2^23
+// leaves n in the low mantissa bits), 2^f from a cubic fitted to 2^f on
+// [0, 1] by iteratively reweighted least squares in relative error (maximum
+// relative error 7.6e-5, below the fp16 rounding the probabilities get
+// next), and n added to the exponent field.  Valid for -126 <= x < 128.
+__device__ __forceinline__ float poly_exp2(float x) {
+    constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+    x = fmaxf(x, -126.0f);
+    const float t = __fadd_rd(x, kMagic);
+    const float f = x - (t - kMagic);
+    const float p = fmaf(fmaf(fmaf(0.07802344113588333f, f, 0.22606651484966278f), f, 0.6958349347114563f), f,
+                         0.9999249577522278f);
+    const int n = __float_as_int(t) - __float_as_int(kMagic);
+    return __int_as_float(__float_as_int(p) + (n << 23));
+}
+// packed fp32 pair arithmetic (one instruction for two lanes of data)
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{ .reg .b64 ra, rb, rc, rd; mov.b64 ra, {%2, %3}; mov.b64 rb, {%4, %5}; mov.b64 rc, {%6, %7};\n"
+        "  fma.rn.f32x2 rd, ra, rb, rc; mov.b64 {%0, %1}, rd; }"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("{ .reg .b64 ra, rb, rd; mov.b64 ra, {%2, %3}; mov.b64 rb, {%4, %5};\n"
+        "  add.rn.f32x2 rd, ra, rb; mov.b64 {%0, %1}, rd; }"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -394,22 +427,30 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                     m_run = mn;
                 }
                 if (stop) break;
-                // probabilities, fp16, stored over the first 32 columns of the score buffer
-                const float nm = -m_run;
-                float lsum = 0.0f;
+                // probabilities, fp16, stored over the first 32 columns of the score
+                // buffer; one pair in four is exponentiated on the FMA pipe
+                const float2 sc2 = make_float2(isig, isig), nm2 = make_float2(-m_run, -m_run);
+                float2 lsum = make_float2(0.0f, 0.0f);
 #pragma unroll
                 for (int hv = 0; hv < 2; ++hv) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
-                        const float p0 = ex2(fmaf(s[32 * hv + 2 * c], isig, nm));
-                        const float p1 = ex2(fmaf(s[32 * hv + 2 * c + 1], isig, nm));
-                        lsum += p0 + p1;
-                        pk[c] = h2(p0, p1);
+                        const float2 x = ffma2(make_float2(s[32 * hv + 2 * c], s[32 * hv + 2 * c + 1]), sc2, nm2);
+                        float2 pp;
+                        if ((c & 3) == 3) {
+                            pp.x = poly_exp2(x.x);
+                            pp.y = poly_exp2(x.y);
+                        } else {
+                            pp.x = ex2(x.x);
+                            pp.y = ex2(x.y);
+                        }
+                        lsum = fadd2(lsum, pp);
+                        pk[c] = h2(pp.x, pp.y);
                     }
                     tmem_st16u(tS(t, u) + 16 * hv + lane_addr, pk);
                 }
-                l_run += lsum;
+                l_run += lsum.x + lsum.y;
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars.p_full[t][u]);
