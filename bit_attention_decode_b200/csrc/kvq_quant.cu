@@ -199,7 +199,7 @@ append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* _
         // ---------------------------------------------------------- workers
         // a token takes 8 Hkv threads, thread (h, blk) owning block blk of
         // head h for both the key and the value row
-        const int per_tok = Hkv * 8;
+        const int per_tok = Hkv * 8;                           // a multiple of 8: lane & 7 == blk
         const int tpc = (workers * 32) / per_tok;              // tokens side by side
         const int t = threadIdx.x % per_tok, sub = threadIdx.x / per_tok;
         const int h = t >> 3, blk = t & 7;
@@ -220,40 +220,54 @@ append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* _
             const float enc_k = __frcp_rn(__fmul_rn(6.0f, g_k)), enc_v = __frcp_rn(__fmul_rn(6.0f, g_v));
             uint8_t* layer_cache = cache + (size_t)li * layer_stride;
             const int st = j % kAppendStages;
-            if (!mbar_wait(&full[st], (j / kAppendStages) & 1)) {
+            // warp-uniform outcome: a warp never splits before its shuffles
+            if (!mbar_wait_warp(&full[st], (j / kAppendStages) & 1)) {
                 atomicOr(&s_timeout, 1);
                 break;
             }
             const T* stage = reinterpret_cast<const T*>(smem + st * kAppendStageBytes);
-            if (active) {
-                for (int tt = sub; tt < n; tt += tpc) {
-                    const int64_t slot = __ldg(slots + t0 + tt);
-                    const bool ok = slot >= 0 && slot < (int64_t)num_pages * kPage;
-                    if (slot >= (int64_t)num_pages * kPage && t == 0) set_status(status, KVQ_DEV_BAD_SLOT);
-                    float y[kBlk];
-                    const size_t e = (size_t)tt * row + h * kD + blk * kBlk;
+            // Every lane runs the same number of iterations (the rotation's
+            // butterflies are full-warp shuffles, and a warp may hold the
+            // lanes of two tokens or idle lanes when 8 Hkv does not divide
+            // 256): lanes without a token compute on zeros and store nothing.
+            for (int base = 0; base < n; base += tpc) {
+                const int tt = base + sub;
+                const bool live = active && tt < n;
+                const int64_t slot = live ? __ldg(slots + t0 + tt) : -1;
+                const bool ok = slot >= 0 && slot < (int64_t)num_pages * kPage;
+                if (live && slot >= (int64_t)num_pages * kPage && t == 0) set_status(status, KVQ_DEV_BAD_SLOT);
+                float y[kBlk];
+                const size_t e = (size_t)(live ? tt : 0) * row + h * kD + blk * kBlk;
+                if (live) {
                     load16_smem<T>(stage + e, y);
-                    // key: smoothing multiply, then the optional rotation (every
-                    // lane of the warp joins its butterflies)
+                } else {
 #pragma unroll
-                    for (int i = 0; i < kBlk; ++i) y[i] = __fmul_rn(y[i], inv[i]);
-                    if (hadamard) hadamard_block(y, blk);
-                    uint2 codes;
-                    uint32_t sf;
-                    quantize_block(y, g_k, enc_k, codes, sf);
-                    const int64_t page = slot >> 4;
-                    const int off = (int)(slot & 15);
-                    uint8_t* tile = layer_cache + ((size_t)page * Hkv + h) * kTile;
-                    if (ok) {
-                        *reinterpret_cast<uint2*>(tile + kKCodes + off * 64 + blk * 8) = codes;
-                        tile[kKScales + off * 8 + blk] = (uint8_t)sf;
-                    }
+                    for (int i = 0; i < kBlk; ++i) y[i] = 0.0f;
+                }
+                // key: smoothing multiply, then the optional rotation
+#pragma unroll
+                for (int i = 0; i < kBlk; ++i) y[i] = __fmul_rn(y[i], inv[i]);
+                if (hadamard) hadamard_block(y, blk);
+                uint2 codes;
+                uint32_t sf;
+                quantize_block(y, g_k, enc_k, codes, sf);
+                const int64_t page = slot >> 4;
+                const int off = (int)(slot & 15);
+                uint8_t* tile = layer_cache + ((size_t)page * Hkv + h) * kTile;
+                if (ok) {
+                    *reinterpret_cast<uint2*>(tile + kKCodes + off * 64 + blk * 8) = codes;
+                    tile[kKScales + off * 8 + blk] = (uint8_t)sf;
+                }
+                if (live) {
                     load16_smem<T>(stage + half_stage / sizeof(T) + e, y);
-                    quantize_block(y, g_v, enc_v, codes, sf);
-                    if (ok) {
-                        *reinterpret_cast<uint2*>(tile + kVCodes + off * 64 + blk * 8) = codes;
-                        tile[kVScales + blk * 16 + off] = (uint8_t)sf;
-                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < kBlk; ++i) y[i] = 0.0f;
+                }
+                quantize_block(y, g_v, enc_v, codes, sf);
+                if (ok) {
+                    *reinterpret_cast<uint2*>(tile + kVCodes + off * 64 + blk * 8) = codes;
+                    tile[kVScales + blk * 16 + off] = (uint8_t)sf;
                 }
             }
             __syncwarp();

@@ -181,3 +181,29 @@ def test_bounded_wait_gives_up_and_context_survives(kvq):
     q, out = decode_all(kvq, p)
     want = harness.oracle_attend(p, 0, 0, q[0, 0][None], 49, 50, cal)
     harness.check_attention(out[0, 0], want[0], "decode after a timed-out wait f32")
+
+
+@pytest.mark.parametrize("hkv,group,hadamard", [(1, 1, False), (2, 4, True), (4, 2, False), (8, 3, False),
+                                                (6, 4, True)])
+def test_other_head_shapes(kvq, hkv, group, hadamard):
+    """kv heads 1..8 and GQA groups 1..4: append, decode and prefill."""
+    w = small(num_layers=1, batch=2, calib_windows=1, calib_len=48, hadamard=hadamard,
+              num_kv_heads=hkv, num_q_heads=hkv * group, prefill_chunk=40)
+    lens = [70, 143]
+    p = harness.build_problem(kvq, w, lens=lens)
+    cal = harness.oracle_calibration(p)
+    for got, want in zip(harness.calib_host(p), cal):
+        np.testing.assert_array_equal(got, want)
+    for b, n in enumerate(lens):
+        assert_codes_equal(p, 0, b, n, cal)
+    q, out = decode_all(kvq, p, out_dtype=torch.float32)
+    for b, n in enumerate(lens):
+        want = harness.oracle_attend(p, 0, b, q[0, b][None], n - 1, n, cal)
+        harness.check_attention(out[0, b], want[0], f"decode hkv {hkv} g {group} seq {b} f32")
+    qp = synth.prefill_queries(w, 0)[None]                       # [1][B][40][Hq][D]
+    q_start = torch.tensor([n - 40 for n in lens], dtype=torch.int32)
+    outp = kvq.prefill_attention(p.shape, p.calib, p.cache, qp.cuda(), q_start.cuda(), p.page_table.cuda(),
+                                 p.lens.cuda(), out_dtype=torch.float32).cpu().numpy()
+    for b, n in enumerate(lens):
+        want = harness.oracle_attend(p, 0, b, qp[0, b].float().numpy(), n - 40, n, cal)
+        harness.check_attention(outp[0, b], want, f"prefill hkv {hkv} g {group} seq {b} f32")
