@@ -46,20 +46,34 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
 
 // ------------------------------------------------------------------ host side
 DecodePlan decode_plan(const kvq_shape& s, int nlayers, int batch, int max_pages) {
-    // one CTA per (layer, sequence, split) covering all kv heads; aim for two
-    // waves at two resident CTAs per SM, splitting sequences only when the
-    // (layer, sequence) units alone cannot fill the GPU
+    // One CTA per (layer, sequence, split) covers all kv heads; two CTAs are
+    // resident per SM.  When the (layer, sequence) units fill at least one
+    // wave they are not split: the longest-first order balances the waves
+    // and no partials have to be merged.  Otherwise take the smallest split
+    // count that minimises  waves(units * splits) * (pages_per_split + 4), each
+    // larger count having to win by 10% (splits of under 8 pages are not
+    // considered).
     (void)s;
     const long units = (long)nlayers * batch;
-    const long target = 148L * 2 * 2;
-    int splits = 1;
-    if (units < target && max_pages > 8) {
-        splits = (int)((target + units - 1) / units);
-        splits = min(splits, (max_pages + 7) / 8);   // at least 8 pages per split
+    const long slots = 148L * 2;
+    int best_s = 1;
+    if (units < slots) {
+        long best = -1;
+        const int max_s = max(1, min(64, max_pages / 8));
+        for (int sp = 1; sp <= max_s; ++sp) {
+            const long pps = (max_pages + sp - 1) / sp;
+            const long waves = (units * sp + slots - 1) / slots;
+            const long cost = waves * (pps + 4);   // + fixed per-CTA work (prologue, partial)
+            // a larger split count must win by 10% to pay for its partials
+            if (best < 0 || cost * 10 < best * 9) {
+                best = cost;
+                best_s = sp;
+            }
+        }
     }
-    int pps = (max_pages + splits - 1) / splits;
+    int pps = (max_pages + best_s - 1) / best_s;
     if (pps < 1) pps = 1;
-    splits = (max_pages + pps - 1) / pps;
+    int splits = (max_pages + pps - 1) / pps;
     if (splits < 1) splits = 1;
     return {pps, splits};
 }

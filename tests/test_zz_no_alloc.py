@@ -57,10 +57,11 @@ def test_noalloc_matches_workspace_decode_on_consecutive_calls(kvq):
 
 def test_noalloc_rejects_problems_beyond_the_scratch(kvq):
     import ctypes
-    shape = kvq.Shape(36, 32, 8)
-    need = kvq.decode_workspace_bytes(shape, 36, 16, 64)
+    # few (layer, sequence) units over very long sequences: many splits
+    shape = kvq.Shape(8, 32, 8)
+    need = kvq.decode_workspace_bytes(shape, 8, 22, 16384)
     assert need > kvq.NOALLOC_SCRATCH_BYTES
     st = kvq._lib.kvq_decode_attention_noalloc(
-        ctypes.byref(shape.c()), ctypes.byref(kvq._Calib(16, 16, 16, 16)), ctypes.byref(kvq._Cache(4096, 1 << 24, 4)),
-        0, 36, 256, 1, 512, 64, 768, 16, 1024, 1, None, None)
+        ctypes.byref(shape.c()), ctypes.byref(kvq._Calib(16, 16, 16, 16)),
+        ctypes.byref(kvq._Cache(4096, 8 * 2304 * 4, 4)), 0, 8, 256, 1, 512, 16384, 768, 22, 1024, 1, None, None)
     assert st == kvq.KVQ_EWORKSPACE
