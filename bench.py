@@ -46,6 +46,8 @@ def parse():
                     help="ragged (default, the decode-throughput workload); prefill, qwen3_8b, hadamard: "
                          "the chunked-prefill and prefix workloads, for their own kernel numbers")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--source-sha", action="store_true",
+                    help="print the hash of the decode kernel's sources (the key of the committed ncu counters) and exit")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--layers", type=int, default=36,
@@ -87,12 +89,37 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
+    """SM clock and clock-event reasons of this process's GPU, sampled every
+    5 ms from a background thread through NVML (reads only) while the timed
+    region runs; nvidia-smi's own sampling loop where NVML is unavailable.
+    The device is found by its UUID, so a remapped CUDA_VISIBLE_DEVICES cannot
+    point the sampler at another GPU."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown"}
 
     def __init__(self, device_index: int):
+        import threading
         self.proc = None
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            self._nvml, self._h = pynvml, h
+            self._thread = threading.Thread(target=self._poll, daemon=True)
+            self._thread.start()
+            return
+        except Exception:
+            self._thread = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
@@ -100,7 +127,25 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def _poll(self):
+        nv, h = self._nvml, self._h
+        while not self._stop.is_set():
+            try:
+                self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                     int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))))
+            except Exception:
+                return
+            self._stop.wait(0.005)
+
     def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+            if not self.samples:
+                return None
+            reasons = sorted({name for _, bits in self.samples for bit, name in self.REASONS.items() if bits & bit})
+            return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                    "reasons": reasons, "samples": len(self.samples), "source": "nvml, 5 ms"}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -117,7 +162,7 @@ class ClockSampler:
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "source": "nvidia-smi, 200 ms"}
 
 
 def measured_peak():
@@ -128,14 +173,25 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def ncu_traffic(kernel_file: str):
+# every source of the decode kernel's translation unit: a change to any of
+# them invalidates the committed ncu counters
+DECODE_SOURCES = ("kvq_decode_tc.cu", "kvq_decode.cu", "kvq_attn.cuh", "kvq_common.cuh", "kvq_sync.cuh")
+
+
+def decode_source_sha() -> str:
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "bit_attention_decode_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic():
     """Per-launch DRAM bytes of the decode kernel from the committed ncu summary,
-    or None when the kernel source changed since that capture."""
+    or None when the kernel sources changed since that capture."""
     path = os.path.join(ROOT, "profiles", "decode_ragged_ncu.md")
-    src = os.path.join(ROOT, "bit_attention_decode_b200", "csrc", kernel_file)
     try:
-        with open(src, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        sha = decode_source_sha()
         vals = {}
         with open(path) as f:
             for line in f:
@@ -567,6 +623,9 @@ def other_workload(args, kvq, synth, rank, world):
 
 def main():
     args = parse()
+    if args.source_sha:
+        print(decode_source_sha())
+        return
     rank, world, local = dist_setup(args)
     if args.impl == "reference":
         if rank != 0:
@@ -607,7 +666,7 @@ def main():
     dec_avg_ms = statistics.mean(dec_ms)
     achieved = dec_bytes / (dec_avg_ms / 1e3) / 1e9
     peak, peak_kind = measured_peak()
-    traffic = ncu_traffic("kvq_decode.cu")
+    traffic = ncu_traffic()
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_block(wl),

@@ -70,69 +70,6 @@ __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
 __device__ __forceinline__ float load_elem(const float* p) { return *p; }
 __device__ __forceinline__ float load_elem(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
-// 16 consecutive elements starting at p (16-byte aligned for fp32, 32 B for bf16)
-__device__ __forceinline__ void load16(const float* p, float* x) {
-    const float4* q = reinterpret_cast<const float4*>(p);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float4 t = __ldg(q + i);
-        x[4 * i] = t.x; x[4 * i + 1] = t.y; x[4 * i + 2] = t.z; x[4 * i + 3] = t.w;
-    }
-}
-__device__ __forceinline__ void load16(const __nv_bfloat16* p, float* x) {
-    const uint4* q = reinterpret_cast<const uint4*>(p);
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        uint4 t = __ldg(q + i);
-        uint32_t w[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            x[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
-            x[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-        }
-    }
-}
-
-// ---------------------------------------------------------------- key transform
-// Normalised Hadamard-128 of a key row held as 8 blocks of 16 in 8
-// consecutive lanes (lane & 7 == blk): butterflies h = 1, 2, 4, 8 inside the
-// thread, h = 16, 32, 64 across lanes, then one multiply by fp32(1/sqrt(128)).
-// Every operation is a single fp32 rounding, in the order listed; every lane
-// of the warp must call it.
-__device__ __forceinline__ void hadamard_block(float* y, int blk) {
-#pragma unroll
-    for (int h = 1; h < kBlk; h <<= 1) {
-#pragma unroll
-        for (int j = 0; j < kBlk; ++j) {
-            if ((j & h) == 0) {
-                float a = y[j], b = y[j + h];
-                y[j] = __fadd_rn(a, b);
-                y[j + h] = __fsub_rn(a, b);
-            }
-        }
-    }
-#pragma unroll
-    for (int m = 1; m < 8; m <<= 1) {
-        const bool upper = (blk & m) != 0;
-#pragma unroll
-        for (int j = 0; j < kBlk; ++j) {
-            float other = __shfl_xor_sync(0xFFFFFFFFu, y[j], m);
-            y[j] = upper ? __fsub_rn(other, y[j]) : __fadd_rn(y[j], other);
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < kBlk; ++i) y[i] = __fmul_rn(y[i], kInvSqrt128);
-}
-
-// Key pre-transform of one block: smoothing multiply y = k * inv_s, then the
-// optional rotation (see hadamard_block).
-__device__ __forceinline__ void transform_key_block(float* y, const float* __restrict__ inv_s_row,
-                                                    int blk, bool hadamard) {
-#pragma unroll
-    for (int i = 0; i < kBlk; ++i) y[i] = __fmul_rn(y[i], __ldg(inv_s_row + blk * kBlk + i));
-    if (hadamard) hadamard_block(y, blk);
-}
-
 __device__ __forceinline__ void set_status(int32_t* status, int32_t bits) {
     if (status) atomicOr(status, bits);
 }

@@ -49,10 +49,13 @@ DecodePlan decode_plan(const kvq_shape& s, int nlayers, int batch, int max_pages
     // One CTA per (layer, sequence, split) covers all kv heads; two CTAs are
     // resident per SM.  When the (layer, sequence) units fill at least one
     // wave they are not split: the longest-first order balances the waves
-    // and no partials have to be merged.  Otherwise take the smallest split
-    // count that minimises  waves(units * splits) * (pages_per_split + 4), each
-    // larger count having to win by 10% (splits of under 8 pages are not
-    // considered).
+    // and no partials have to be merged.  Otherwise take the split count that
+    // minimises  waves(units * splits) * (pages_per_split + 4)  for sequences
+    // of max_pages (the + 4 stands for a CTA's fixed work: prologue and
+    // partial), the largest among equal costs: the lengths are not known on
+    // the host, and shorter pieces balance ragged lengths better.  Splits of
+    // under 8 pages are not considered; the partials stay below one wave of
+    // units x 64 splits.
     (void)s;
     const long units = (long)nlayers * batch;
     const long slots = 148L * 2;
@@ -63,9 +66,8 @@ DecodePlan decode_plan(const kvq_shape& s, int nlayers, int batch, int max_pages
         for (int sp = 1; sp <= max_s; ++sp) {
             const long pps = (max_pages + sp - 1) / sp;
             const long waves = (units * sp + slots - 1) / slots;
-            const long cost = waves * (pps + 4);   // + fixed per-CTA work (prologue, partial)
-            // a larger split count must win by 10% to pay for its partials
-            if (best < 0 || cost * 10 < best * 9) {
+            const long cost = waves * (pps + 4);
+            if (best < 0 || cost <= best) {
                 best = cost;
                 best_s = sp;
             }

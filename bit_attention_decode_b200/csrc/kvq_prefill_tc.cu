@@ -12,7 +12,7 @@
 // the kv head times its 32 tokens (row = head * 32 + token), so each
 // dequantised key/value block feeds 8 query heads x 32 tokens.  Per 64-token
 // key block (4 pages):
-//   dequant warps (4): bulk-copy the 4 packed page tiles into a staging
+//   dequant warps (3): bulk-copy the 4 packed page tiles into a staging
 //     ring, dequantise to fp16 (E2M1 x E4M3 is exact in fp16) into a K tile
 //     (K-major) and a V tile (MN-major), both in the 128-byte-swizzled
 //     canonical layouts the MMA reads; rows past the sequence are zeros.
@@ -33,6 +33,7 @@
 #include "kvq_attn.cuh"
 #include "kvq_common.cuh"
 #include "kvq_internal.h"
+#include "kvq_packed.cuh"
 #include "kvq_sync.cuh"
 
 namespace kvq {
@@ -165,23 +166,6 @@ __device__ __forceinline__ float poly_exp2(float x) {
                          0.9999249577522278f);
     const int n = __float_as_int(t) - __float_as_int(kMagic);
     return __int_as_float(__float_as_int(p) + (n << 23));
-}
-// packed fp32 pair arithmetic (one instruction for two lanes of data)
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-    float2 d;
-    asm("{ .reg .b64 ra, rb, rc, rd; mov.b64 ra, {%2, %3}; mov.b64 rb, {%4, %5}; mov.b64 rc, {%6, %7};\n"
-        "  fma.rn.f32x2 rd, ra, rb, rc; mov.b64 {%0, %1}, rd; }"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
-    float2 d;
-    asm("{ .reg .b64 ra, rb, rd; mov.b64 ra, {%2, %3}; mov.b64 rb, {%4, %5};\n"
-        "  add.rn.f32x2 rd, ra, rb; mov.b64 {%0, %1}, rd; }"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
 }
 __device__ __forceinline__ float ex2(float x) {
     float y;

@@ -11,6 +11,7 @@
 #include "kvq_common.cuh"
 #include "kvq_internal.h"
 #include "kvq_sync.cuh"
+#include "kvq_transform.cuh"
 
 namespace kvq {
 
@@ -57,13 +58,12 @@ calib_tensor_amax_kernel(const T* __restrict__ k, const T* __restrict__ v, int W
     const int r = live ? lane_row : rows - 1;   // dead lanes still join the shuffles
     const int h = r % Hkv;
     const size_t off = ((size_t)l * rows + r) * kD + blk * kBlk;
-    float y[kBlk], x[kBlk];
+    float2 y[kBlk / 2], x[kBlk / 2];
     load16(k + off, y);
     load16(v + off, x);
-    transform_key_block(y, inv_s + ((size_t)l * Hkv + h) * kD, blk, hadamard != 0);
-    float ak = 0.0f, av = 0.0f;
-#pragma unroll
-    for (int i = 0; i < kBlk; ++i) { ak = fmaxf(ak, fabsf(y[i])); av = fmaxf(av, fabsf(x[i])); }
+    smooth_block(y, inv_s + ((size_t)l * Hkv + h) * kD + blk * kBlk);
+    if (hadamard) hadamard_block(y, blk);
+    float ak = absmax16(y), av = absmax16(x);
     if (!live) { ak = 0.0f; av = 0.0f; }
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) {
@@ -85,61 +85,53 @@ __global__ void calib_finalize_gscale_kernel(float* __restrict__ gk, float* __re
 }
 
 // ------------------------------------------------------------------ quantise
+// Eight fp32 pairs -> four bytes of E2M1 codes: pair i -> byte i, its .x in
+// the low nibble.
+__device__ __forceinline__ uint32_t e2m1x8_rn(float2 a, float2 b, float2 c, float2 d) {
+    uint32_t w;
+    asm("{ .reg .b8 b0, b1, b2, b3;\n"
+        "  cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1; cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n"
+        "  cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5; cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n"
+        "  mov.b32 %0, {b0, b1, b2, b3}; }"
+        : "=r"(w)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
+    return w;
+}
+
 // One 16-element block: E4M3 block scale from the absmax, then E2M1 codes.
-// enc = 1/(6 g) is computed once per tensor by the caller.
-__device__ __forceinline__ void quantize_block(const float* y, float g, float enc, uint2& codes,
+// enc = 1/(6 g); rtab[c] = 1/(val(c) g) for every scale code c (0 where the
+// product is zero), both computed once per tensor.
+__device__ __forceinline__ void quantize_block(const float2* y, float enc, const float* rtab, uint2& codes,
                                                uint32_t& sf) {
-    float a = 0.0f;
+    sf = e4m3_rn(__fmul_rn(absmax16(y), enc));
+    const float r = rtab[sf & 0x7Fu];
+    const float2 r2 = make_float2(r, r);
+    float2 z[kBlk / 2];
 #pragma unroll
-    for (int i = 0; i < kBlk; ++i) a = fmaxf(a, fabsf(y[i]));
-    sf = e4m3_rn(__fmul_rn(a, enc));
-    const float d = __fmul_rn(e4m3_to_f32(sf), g);
-    const float r = (d == 0.0f) ? 0.0f : __frcp_rn(d);
-    uint32_t w[2] = {0u, 0u};
-#pragma unroll
-    for (int j = 0; j < kBlk / 2; ++j) {
-        uint32_t byte = e2m1x2_rn(__fmul_rn(y[2 * j + 1], r), __fmul_rn(y[2 * j], r));
-        w[j >> 2] |= byte << (8 * (j & 3));
-    }
-    codes = make_uint2(w[0], w[1]);
+    for (int i = 0; i < kBlk / 2; ++i) z[i] = fmul2(y[i], r2);
+    codes = make_uint2(e2m1x8_rn(z[0], z[1], z[2], z[3]), e2m1x8_rn(z[4], z[5], z[6], z[7]));
 }
 
 // Bulk-copy staging of the inputs.  A work item is a chunk of `tc`
 // consecutive tokens of one layer: its key rows and value rows are two
 // contiguous ranges (tc x Hkv x 128 elements each), streamed into a ring of
 // kAppendStages shared-memory stages with cp.async.bulk and an mbarrier
-// transaction count.  Thread 0 keeps kAppendStages - 1 chunks in flight.
-// Quantisation then reads the stage: a token takes Hkv * 16 threads, threads
-// [0, 8 Hkv) owning the 8 key blocks of each head and the rest the value
-// blocks; a CTA of 256 threads works on 256 / (16 Hkv) tokens at a time.
-// With the rotation Hkv is even, so every warp lies inside one token and the
+// transaction count.  The producer warp also copies the chunk's slots into
+// the stage's slot array, so that no worker waits on a global load per
+// token, and (when the stage last held another layer) writes the layer's
+// quantiser constants: enc = 1/(6 g) and the reciprocal 1/(val(c) g) of
+// every E4M3 scale code c, for the keys and for the values.  A block then
+// looks its reciprocal up instead of dividing.  A stage is full once the
+// copies have landed and the producer has arrived twice (before the copies,
+// and after its shared-memory stores).
+// Quantisation then reads the stage: a token takes Hkv * 8 threads, thread
+// (h, blk) owning block blk of head h for both the key and the value row; a
+// CTA of 256 worker threads works on 256 / (8 Hkv) tokens at a time.  With
+// the rotation Hkv is even, so every warp lies inside one token and the
 // cross-lane butterflies stay uniform.
 constexpr int kAppendStages = 3;
 constexpr int kAppendStageBytes = 32768;   // key + value rows of one chunk
-
-template <typename T>
-__device__ __forceinline__ void load16_smem(const T* p, float* x);
-template <>
-__device__ __forceinline__ void load16_smem<float>(const float* p, float* x) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float4 t = reinterpret_cast<const float4*>(p)[i];
-        x[4 * i] = t.x; x[4 * i + 1] = t.y; x[4 * i + 2] = t.z; x[4 * i + 3] = t.w;
-    }
-}
-template <>
-__device__ __forceinline__ void load16_smem<__nv_bfloat16>(const __nv_bfloat16* p, float* x) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        uint4 t = reinterpret_cast<const uint4*>(p)[i];
-        uint32_t w[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            x[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
-            x[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-        }
-    }
-}
+constexpr int kAppendMaxChunk = 64;        // tokens: bf16 rows of one kv head fill half a stage
 
 template <typename T>
 __global__ void __launch_bounds__(288, 2)
@@ -149,108 +141,130 @@ append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* _
               int64_t layer_stride, int num_pages, int hadamard, int32_t* __restrict__ status) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t full[kAppendStages], empty[kAppendStages];
+    __shared__ int64_t s_slot[kAppendStages][kAppendMaxChunk];
+    __shared__ float s_rtab[kAppendStages][2][128];           // [stage][key, value][scale code]
+    __shared__ float s_enc[kAppendStages][2];
+    __shared__ int s_layer[kAppendStages];                    // layer of the stage's constants
     __shared__ int s_timeout, s_issued;
     const int row = Hkv * kD;                                  // elements per token row
     const uint32_t half_stage = kAppendStageBytes / 2;         // key rows, then value rows
     const int chunks = (num_tokens + tc - 1) / tc;
     const long items = (long)chunks * nlayers;
-    const int mine = items > blockIdx.x ? (int)((items - 1 - blockIdx.x) / gridDim.x + 1) : 0;
+    // a contiguous run of items per CTA: its layer (and so the stage's
+    // constants) changes at most a few times
+    const long per = items / gridDim.x, extra = items % gridDim.x;
+    const long first = blockIdx.x * per + min((long)blockIdx.x, extra);
+    const int mine = (int)(per + ((long)blockIdx.x < extra ? 1 : 0));
     const int workers = 8;                                     // warps 0..7; warp 8 streams the inputs
-    const int warp = threadIdx.x >> 5;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t num_slots = (int64_t)num_pages * kPage;
 
     if (threadIdx.x == 0) {
         s_timeout = 0;
         s_issued = 0;
         for (int i = 0; i < kAppendStages; ++i) {
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&full[i])));
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&empty[i])), "r"(workers));
+            mbar_init(&full[i], 2);
+            mbar_init(&empty[i], workers);
+            s_layer[i] = -1;
         }
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_fence_init();
     }
     __syncthreads();
 
     if (warp == workers) {
         // ---------------------------------------------------------- producer
-        if ((threadIdx.x & 31) == 0) {
-            int j = 0;
-            for (; j < mine; ++j) {
-                const int st = j % kAppendStages;
-                if (j >= kAppendStages && !mbar_wait(&empty[st], ((j / kAppendStages) - 1) & 1)) {
-                    atomicOr(&s_timeout, 1);
-                    break;
-                }
-                const long it = blockIdx.x + (long)j * gridDim.x;
-                const int li = (int)(it / chunks), t0 = (int)(it % chunks) * tc;
-                const int n = min(tc, num_tokens - t0);
+        int j = 0;
+        for (; j < mine; ++j) {
+            const int st = j % kAppendStages;
+            if (j >= kAppendStages && !mbar_wait_warp(&empty[st], ((j / kAppendStages) - 1) & 1)) {
+                if (lane == 0) atomicOr(&s_timeout, 1);
+                break;
+            }
+            const long it = first + j;
+            const int li = (int)(it / chunks), t0 = (int)(it % chunks) * tc;
+            const int n = min(tc, num_tokens - t0);
+            if (lane == 0) {
                 const uint32_t bytes = (uint32_t)n * row * sizeof(T);
                 uint8_t* dst = smem + st * kAppendStageBytes;
                 const size_t off = ((size_t)li * num_tokens + t0) * row;
-                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&full[st])),
-                             "r"(2 * bytes) : "memory");
-                asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                             ::"r"(smem_u32(dst)), "l"(k + off), "r"(bytes), "r"(smem_u32(&full[st])) : "memory");
-                asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                             ::"r"(smem_u32(dst + half_stage)), "l"(v + off), "r"(bytes), "r"(smem_u32(&full[st]))
-                             : "memory");
+                mbar_arrive_expect_tx(&full[st], 2 * bytes);
+                bulk_g2s(dst, k + off, bytes, &full[st]);
+                bulk_g2s(dst + half_stage, v + off, bytes, &full[st]);
             }
-            s_issued = j;
+            for (int x = lane; x < n; x += 32) s_slot[st][x] = __ldg(slots + t0 + x);
+            if (s_layer[st] != li) {
+                // the same operations, in the same fp32 order, as a per-block
+                // d = val(sf) * g, r = (d == 0) ? 0 : 1/d
+                const float g_k = __ldg(gk + li), g_v = __ldg(gv + li);
+                for (int x = lane; x < 256; x += 32) {
+                    const float d = __fmul_rn(e4m3_to_f32(x & 127), (x < 128) ? g_k : g_v);
+                    s_rtab[st][x >> 7][x & 127] = (d == 0.0f) ? 0.0f : __frcp_rn(d);
+                }
+                if (lane < 2) s_enc[st][lane] = __frcp_rn(__fmul_rn(6.0f, lane ? g_v : g_k));
+                __syncwarp();
+                if (lane == 0) s_layer[st] = li;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full[st]);
         }
+        if (lane == 0) s_issued = j;
     } else {
         // ---------------------------------------------------------- workers
-        // a token takes 8 Hkv threads, thread (h, blk) owning block blk of
-        // head h for both the key and the value row
         const int per_tok = Hkv * 8;                           // a multiple of 8: lane & 7 == blk
         const int tpc = (workers * 32) / per_tok;              // tokens side by side
         const int t = threadIdx.x % per_tok, sub = threadIdx.x / per_tok;
         const int h = t >> 3, blk = t & 7;
         const bool active = sub < tpc;
+        float2 inv[kBlk / 2];                                  // smoothing factors of layer inv_layer
+        int inv_layer = -1;
         for (int j = 0; j < mine; ++j) {
-            const long it = blockIdx.x + (long)j * gridDim.x;
+            const long it = first + j;
             const int li = (int)(it / chunks), t0 = (int)(it % chunks) * tc;
             const int n = min(tc, num_tokens - t0);
-            // per-chunk constants, loaded before waiting for the inputs
-            float inv[kBlk];
-            const float4* ip = reinterpret_cast<const float4*>(inv_s + ((size_t)li * Hkv + h) * kD + blk * kBlk);
+            if (li != inv_layer) {
+                // loaded before waiting for the inputs
+                const float4* ip = reinterpret_cast<const float4*>(inv_s + ((size_t)li * Hkv + h) * kD + blk * kBlk);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float4 q4 = __ldg(ip + i);
-                inv[4 * i] = q4.x; inv[4 * i + 1] = q4.y; inv[4 * i + 2] = q4.z; inv[4 * i + 3] = q4.w;
+                for (int i = 0; i < 4; ++i) {
+                    const float4 f = __ldg(ip + i);
+                    inv[2 * i] = make_float2(f.x, f.y);
+                    inv[2 * i + 1] = make_float2(f.z, f.w);
+                }
+                inv_layer = li;
             }
-            const float g_k = __ldg(gk + li), g_v = __ldg(gv + li);
-            const float enc_k = __frcp_rn(__fmul_rn(6.0f, g_k)), enc_v = __frcp_rn(__fmul_rn(6.0f, g_v));
             uint8_t* layer_cache = cache + (size_t)li * layer_stride;
             const int st = j % kAppendStages;
             // warp-uniform outcome: a warp never splits before its shuffles
             if (!mbar_wait_warp(&full[st], (j / kAppendStages) & 1)) {
-                atomicOr(&s_timeout, 1);
+                if (lane == 0) atomicOr(&s_timeout, 1);
                 break;
             }
             const T* stage = reinterpret_cast<const T*>(smem + st * kAppendStageBytes);
+            const float enc_k = s_enc[st][0], enc_v = s_enc[st][1];
+            const float* rtab_k = s_rtab[st][0];
+            const float* rtab_v = s_rtab[st][1];
             // Every lane runs the same number of iterations (the rotation's
             // butterflies are full-warp shuffles, and a warp may hold the
             // lanes of two tokens or idle lanes when 8 Hkv does not divide
-            // 256): lanes without a token compute on zeros and store nothing.
+            // 256): lanes without a token compute on the chunk's first row
+            // and store nothing.  A token's 8 Hkv lanes are consecutive and
+            // share its liveness, so no live lane ever exchanges with them.
             for (int base = 0; base < n; base += tpc) {
                 const int tt = base + sub;
                 const bool live = active && tt < n;
-                const int64_t slot = live ? __ldg(slots + t0 + tt) : -1;
-                const bool ok = slot >= 0 && slot < (int64_t)num_pages * kPage;
-                if (live && slot >= (int64_t)num_pages * kPage && t == 0) set_status(status, KVQ_DEV_BAD_SLOT);
-                float y[kBlk];
+                const int64_t slot = live ? s_slot[st][tt] : -1;
+                const bool ok = slot >= 0 && slot < num_slots;
+                if (live && slot >= num_slots && t == 0) set_status(status, KVQ_DEV_BAD_SLOT);
                 const size_t e = (size_t)(live ? tt : 0) * row + h * kD + blk * kBlk;
-                if (live) {
-                    load16_smem<T>(stage + e, y);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < kBlk; ++i) y[i] = 0.0f;
-                }
+                float2 y[kBlk / 2];
+                load16(stage + e, y);
                 // key: smoothing multiply, then the optional rotation
 #pragma unroll
-                for (int i = 0; i < kBlk; ++i) y[i] = __fmul_rn(y[i], inv[i]);
+                for (int i = 0; i < kBlk / 2; ++i) y[i] = fmul2(y[i], inv[i]);
                 if (hadamard) hadamard_block(y, blk);
                 uint2 codes;
                 uint32_t sf;
-                quantize_block(y, g_k, enc_k, codes, sf);
+                quantize_block(y, enc_k, rtab_k, codes, sf);
                 const int64_t page = slot >> 4;
                 const int off = (int)(slot & 15);
                 uint8_t* tile = layer_cache + ((size_t)page * Hkv + h) * kTile;
@@ -258,21 +272,15 @@ append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* _
                     *reinterpret_cast<uint2*>(tile + kKCodes + off * 64 + blk * 8) = codes;
                     tile[kKScales + off * 8 + blk] = (uint8_t)sf;
                 }
-                if (live) {
-                    load16_smem<T>(stage + half_stage / sizeof(T) + e, y);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < kBlk; ++i) y[i] = 0.0f;
-                }
-                quantize_block(y, g_v, enc_v, codes, sf);
+                load16(stage + half_stage / sizeof(T) + e, y);
+                quantize_block(y, enc_v, rtab_v, codes, sf);
                 if (ok) {
                     *reinterpret_cast<uint2*>(tile + kVCodes + off * 64 + blk * 8) = codes;
                     tile[kVScales + blk * 16 + off] = (uint8_t)sf;
                 }
             }
             __syncwarp();
-            if ((threadIdx.x & 31) == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(
-                                                          smem_u32(&empty[st])) : "memory");
+            if (lane == 0) mbar_arrive(&empty[st]);
         }
     }
     __syncthreads();
