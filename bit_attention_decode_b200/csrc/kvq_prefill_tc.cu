@@ -379,9 +379,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                         s[c] = (kp <= qpos && kp < kv_end) ? s[c] : -INFINITY;
                     }
                 }
-                float bm = -INFINITY;
+                // block max as a tree of three-input maxima (depth 4, not 64)
+                float m21[22];
 #pragma unroll
-                for (int c = 0; c < kBlkTok; ++c) bm = fmaxf(bm, s[c]);
+                for (int c = 0; c < 21; ++c) m21[c] = fmax3(s[3 * c], s[3 * c + 1], s[3 * c + 2]);
+                m21[21] = s[63];
+                float m8[8];
+#pragma unroll
+                for (int c = 0; c < 7; ++c) m8[c] = fmax3(m21[3 * c], m21[3 * c + 1], m21[3 * c + 2]);
+                m8[7] = m21[21];
+                float bm = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], fmax3(m8[5], m8[6], m8[7])));
                 bm *= isig;
                 // lazy rescale: move the reference max only when it grows by > 2^8
                 const bool grow = bm > m_run + kRescaleThreshold || (m_run == -INFINITY && bm > -INFINITY);
@@ -414,7 +421,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                 // probabilities, fp16, stored over the first 32 columns of the score
                 // buffer; one pair in four is exponentiated on the FMA pipe
                 const float2 sc2 = make_float2(isig, isig), nm2 = make_float2(-m_run, -m_run);
-                float2 lsum = make_float2(0.0f, 0.0f);
+                // four independent partial sums (the row sum is a 32-deep chain otherwise)
+                float2 lsum[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
+                                  make_float2(0.0f, 0.0f)};
 #pragma unroll
                 for (int hv = 0; hv < 2; ++hv) {
                     uint32_t pk[16];
@@ -429,12 +438,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                             pp.x = ex2(x.x);
                             pp.y = ex2(x.y);
                         }
-                        lsum = fadd2(lsum, pp);
+                        lsum[c & 3] = fadd2(lsum[c & 3], pp);
                         pk[c] = h2(pp.x, pp.y);
                     }
                     tmem_st16u(tS(t, u) + 16 * hv + lane_addr, pk);
                 }
-                l_run += lsum.x + lsum.y;
+                const float2 l2 = fadd2(fadd2(lsum[0], lsum[1]), fadd2(lsum[2], lsum[3]));
+                l_run += l2.x + l2.y;
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars.p_full[t][u]);
@@ -442,69 +452,86 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
         } else if (warp < kMmaWarp) {
             // ------------------------------------------------------ dequant warps
             const int dt = threadIdx.x - 32 * kDequantWarp0;   // 0..95
-            const bool issuer = (dt == 0);
+            // The copies are issued by the last dequant warp, which has the
+            // fewest dequantisation items.  The page ids of a block are read one
+            // block ahead: a page-table load ahead of each copy would otherwise
+            // put four serial L2 round trips on every block.
+            const bool issuer = (dt == 32 * (kWarpsDequant - 1));
             int issued = 0;
+            int pgn[4] = {0, 0, 0, 0};   // page ids of block `issued`
+            auto fetch_ids = [&](int j) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) pgn[k] = (j * 4 + k < npg) ? __ldg(pt + j * 4 + k) : 0;
+            };
             auto issue = [&](int j) {   // stage j % kStageN <- the pages of block j
                 const int st = j % kStageN;
-                const int p_lo = j * 4, p_hi = min(npg, p_lo + 4);
-                mbar_arrive_expect_tx(&bars.stage_full[st], (uint32_t)(p_hi - p_lo) * kTile);
-                for (int p = p_lo; p < p_hi; ++p) {
-                    const int pg = __ldg(pt + p);
-                    bulk_g2s(smem + kOffStage + st * kStageBytes + (p - p_lo) * kTile,
-                              layer_base + ((size_t)pg * a.Hkv + h) * kTile, kTile, &bars.stage_full[st]);
-                }
+                const int p_lo = j * 4, n_p = min(npg, p_lo + 4) - p_lo;
+                int pg[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) pg[k] = pgn[k];
+                fetch_ids(j + 1);
+                mbar_arrive_expect_tx(&bars.stage_full[st], (uint32_t)n_p * kTile);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (k < n_p)
+                        bulk_g2s(smem + kOffStage + st * kStageBytes + k * kTile,
+                                 layer_base + ((size_t)pg[k] * a.Hkv + h) * kTile, kTile, &bars.stage_full[st]);
             };
+            if (issuer) fetch_ids(0);
+            // every stage is filled up front; a stage is refilled (block j +
+            // kStageN) as soon as the three warps have read block j out of it
             if (issuer)
-                for (; issued < kStageN - 1 && issued < nb; ++issued) issue(issued);
-            for (int j = 0; j < nb; ++j) {
-                const int buf = j & 1, st = j % kStageN;
+                for (; issued < kStageN && issued < nb; ++issued) issue(issued);
+            // items (token, half of head_dim): 128 per block over 96 threads
+            constexpr int kItems = 2 * kBlkTok, kDqThreads = 32 * kWarpsDequant;
+            constexpr int kPer = (kItems + kDqThreads - 1) / kDqThreads;
+            struct Staged {
+                uint4 kc[kPer][2], vc[kPer][2];
+                uint32_t ks[kPer], vs[kPer][4];
+            };
+            // read block j's codes and scales out of its stage, release the
+            // stage and (issuer) refill it with block j + kStageN
+            auto load_block = [&](int j, Staged& S) -> bool {
+                const int st = j % kStageN;
+                if (!mbar_wait_warp(&bars.stage_full[st], (j / kStageN) & 1)) return false;
+#pragma unroll
+                for (int e = 0; e < kPer; ++e) {
+                    const int it = dt + e * kDqThreads;
+                    const int tkn = it >> 1, half = it & 1;
+                    S.kc[e][0] = S.kc[e][1] = S.vc[e][0] = S.vc[e][1] = make_uint4(0, 0, 0, 0);
+                    S.ks[e] = 0;
+                    S.vs[e][0] = S.vs[e][1] = S.vs[e][2] = S.vs[e][3] = 0;
+                    if (it < kItems && j * kBlkTok + tkn < kv_end) {
+                        const uint8_t* T = smem + kOffStage + st * kStageBytes + (tkn >> 4) * kTile;
+                        const int trow = tkn & 15;
+                        S.kc[e][0] = *reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32);
+                        S.kc[e][1] = *reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32 + 16);
+                        S.ks[e] = *reinterpret_cast<const uint32_t*>(T + kKScales + trow * 8 + half * 4);
+                        S.vc[e][0] = *reinterpret_cast<const uint4*>(T + kVCodes + trow * 64 + half * 32);
+                        S.vc[e][1] = *reinterpret_cast<const uint4*>(T + kVCodes + trow * 64 + half * 32 + 16);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) S.vs[e][q] = T[kVScales + (half * 4 + q) * 16 + trow];
+                    }
+                }
+                __syncwarp();
+                if ((dt & 31) == 0) mbar_arrive(&bars.stage_empty[st]);
                 int issue_ok = 1;
-                if (issuer && issued < nb) {
-                    if (issued >= kStageN &&
-                        !mbar_wait(&bars.stage_empty[issued % kStageN], ((issued / kStageN) - 1) & 1)) {
+                if (issuer && issued < nb) {   // issued == j + kStageN
+                    if (!mbar_wait(&bars.stage_empty[st], (j / kStageN) & 1)) {
                         issue_ok = 0;
                     } else {
                         issue(issued);
                         ++issued;
                     }
                 }
-                if (!__shfl_sync(0xFFFFFFFFu, issue_ok, 0)) { atomicOr(&bars.flags, 1); break; }
-                if (!mbar_wait_warp(&bars.stage_full[st], (j / kStageN) & 1)) { atomicOr(&bars.flags, 1); break; }
-                // items (token, half of head_dim): 128 per block over 96 threads
-                constexpr int kItems = 2 * kBlkTok, kDqThreads = 32 * kWarpsDequant;
-                constexpr int kPer = (kItems + kDqThreads - 1) / kDqThreads;
-                uint4 kc[kPer][2], vc[kPer][2];
-                uint32_t ks[kPer], vs[kPer][4];
-#pragma unroll
-                for (int e = 0; e < kPer; ++e) {
-                    const int it = dt + e * kDqThreads;
-                    const int tkn = it >> 1, half = it & 1;
-                    kc[e][0] = kc[e][1] = vc[e][0] = vc[e][1] = make_uint4(0, 0, 0, 0);
-                    ks[e] = 0;
-                    vs[e][0] = vs[e][1] = vs[e][2] = vs[e][3] = 0;
-                    if (it < kItems && j * kBlkTok + tkn < kv_end) {
-                        const uint8_t* T = smem + kOffStage + st * kStageBytes + (tkn >> 4) * kTile;
-                        const int trow = tkn & 15;
-                        kc[e][0] = *reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32);
-                        kc[e][1] = *reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32 + 16);
-                        ks[e] = *reinterpret_cast<const uint32_t*>(T + kKScales + trow * 8 + half * 4);
-                        vc[e][0] = *reinterpret_cast<const uint4*>(T + kVCodes + trow * 64 + half * 32);
-                        vc[e][1] = *reinterpret_cast<const uint4*>(T + kVCodes + trow * 64 + half * 32 + 16);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) vs[e][q] = T[kVScales + (half * 4 + q) * 16 + trow];
-                    }
-                }
-                __syncwarp();
-                if ((dt & 31) == 0) mbar_arrive(&bars.stage_empty[st]);
-                // K tile buffer: free once both tiles' Q.K(j-2) are done (the
-                // commit after tile B's covers every earlier MMA)
-                if (j >= 2 && !mbar_wait_warp(&bars.s_full[kTiles - 1][buf], ((j - 2) >> 1) & 1)) {
-                    atomicOr(&bars.flags, 1);
-                    break;
-                }
+                return __shfl_sync(0xFFFFFFFFu, issue_ok, 0) != 0;
+            };
+            // keys of block j into K buffer j & 1, free once both tiles'
+            // Q.K(j - 2) are done (the commit after the last MMA covers all)
+            auto store_k = [&](int j, const Staged& S) -> bool {
+                const int buf = j & 1;
+                if (j >= 2 && !mbar_wait_warp(&bars.s_full[kTiles - 1][buf], ((j - 2) >> 1) & 1)) return false;
                 uint8_t* Kt = smem + kOffK + buf * kKBytes;
-                uint8_t* Vt = smem + kOffV + buf * kVBytes;
-                uint32_t vsc[kPer][4];
 #pragma unroll
                 for (int e = 0; e < kPer; ++e) {
                     const int it = dt + e * kDqThreads;
@@ -514,15 +541,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                     // 4 blocks of 16 dims: 8 code bytes and one scale each
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const uint4& c0 = kc[e][q >> 1];
+                        const uint4& c0 = S.kc[e][q >> 1];
                         const uint32_t kw0 = (q & 1) ? c0.z : c0.x, kw1 = (q & 1) ? c0.w : c0.y;
                         uint32_t ka[4], kb[4];
                         e2m1x8(kw0, ka);
                         e2m1x8(kw1, kb);
-                        const uint32_t ksh = e4m3x2_to_f16x2((ks[e] >> (8 * q)) & 0xFFu) & 0xFFFFu;
-                        const uint32_t vsh = e4m3x2_to_f16x2(vs[e][q]) & 0xFFFFu;
+                        const uint32_t ksh = e4m3x2_to_f16x2((S.ks[e] >> (8 * q)) & 0xFFu) & 0xFFFFu;
                         const uint32_t ksc = valid ? (ksh | (ksh << 16)) : 0u;
-                        vsc[e][q] = valid ? (vsh | (vsh << 16)) : 0u;
                         // chunk index along head_dim: 2 chunks (8 dims each) per block
                         const int dim_chunk = half * 8 + 2 * q;          // 0..15
                         const int plane = dim_chunk >> 3, ch = dim_chunk & 7;
@@ -536,24 +561,29 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                 fence_async_smem();
                 __syncwarp();
                 if ((dt & 31) == 0) mbar_arrive(&bars.k_full[buf]);
-                // V tile buffer: free once both tiles' P.V(j-2) are done
-                if (j >= 2 && !mbar_wait_warp(&bars.pv_done[kTiles - 1][buf], ((j - 2) >> 1) & 1)) {
-                    atomicOr(&bars.flags, 1);
-                    break;
-                }
+                return true;
+            };
+            // values of block j into V buffer j & 1, free once both tiles'
+            // P.V(j - 2) are done
+            auto store_v = [&](int j, const Staged& S) -> bool {
+                const int buf = j & 1;
+                if (j >= 2 && !mbar_wait_warp(&bars.pv_done[kTiles - 1][buf], ((j - 2) >> 1) & 1)) return false;
+                uint8_t* Vt = smem + kOffV + buf * kVBytes;
 #pragma unroll
                 for (int e = 0; e < kPer; ++e) {
                     const int it = dt + e * kDqThreads;
                     if (it >= kItems) break;
                     const int tkn = it >> 1, half = it & 1;
+                    const bool valid = j * kBlkTok + tkn < kv_end;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const uint4& c1 = vc[e][q >> 1];
+                        const uint4& c1 = S.vc[e][q >> 1];
                         const uint32_t vw0 = (q & 1) ? c1.z : c1.x, vw1 = (q & 1) ? c1.w : c1.y;
                         uint32_t va[4], vb[4];
                         e2m1x8(vw0, va);
                         e2m1x8(vw1, vb);
-                        const uint32_t sc = vsc[e][q];
+                        const uint32_t vsh = e4m3x2_to_f16x2(S.vs[e][q]) & 0xFFFFu;
+                        const uint32_t sc = valid ? (vsh | (vsh << 16)) : 0u;
                         const int dim_chunk = half * 8 + 2 * q;
                         const int plane = dim_chunk >> 3, ch = dim_chunk & 7;
                         // values: MN-major, row = token (the K of P.V), 128-byte rows of 64 dims
@@ -566,7 +596,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                 fence_async_smem();
                 __syncwarp();
                 if ((dt & 31) == 0) mbar_arrive(&bars.v_full[buf]);
+                return true;
+            };
+            // Software-pipelined: the keys of block j + 1 are written before
+            // the values of block j, because the MMA warp needs them first
+            // (Q.K(j + 1) is issued before P.V(j)).
+            Staged cur, nxt;
+            bool dq_ok = nb == 0 || (load_block(0, cur) && store_k(0, cur));
+            for (int j = 0; dq_ok && j < nb; ++j) {
+                if (j + 1 < nb) dq_ok = load_block(j + 1, nxt) && store_k(j + 1, nxt);
+                dq_ok = dq_ok && store_v(j, cur);
+                cur = nxt;
             }
+            if (!dq_ok) atomicOr(&bars.flags, 1);
             if (issuer) bars.issued = issued;
         } else if (lane == 0) {
             // ------------------------------------------------------ MMA issuer
@@ -593,6 +635,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                     if (!mbar_wait(&bars.k_full[buf], (j >> 1) & 1)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t kb = kd[buf];
+                    // tile by tile, so that tile A's softmax starts while the
+                    // tensor pipe works on tile B
 #pragma unroll
                     for (int t = 0; t < kTiles; ++t) {
                         const uint32_t sd = tS(t, buf);
