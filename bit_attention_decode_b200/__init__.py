@@ -4,7 +4,7 @@ Argument marshalling only: every step of calibration, quantise-append and
 attention runs in the CUDA kernels of ``libkvq.so`` (declared in
 ``include/kvq.h``).  PyTorch supplies device memory and the current stream.
 There is no CPU fallback: if the library is missing, importing this package
-raises ``ImportError``; build it with ``python -m bit_attention_decode_b200.build``.
+raises ``ImportError``; build it with ``python bit_attention_decode_b200/build.py``.
 """
 
 from __future__ import annotations
@@ -20,7 +20,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libkvq.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m bit_attention_decode_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python bit_attention_decode_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -61,6 +61,8 @@ _lib.kvq_version.restype = ctypes.c_char_p
 _lib.kvq_version.argtypes = []
 _lib.kvq_calibrate_smoothing.restype = _I32
 _lib.kvq_calibrate_smoothing.argtypes = [_SHP, _P, _P, _I32, _I32, _I32, _I32, _CAL, _P]
+_lib.kvq_calibrate_native.restype = _I32
+_lib.kvq_calibrate_native.argtypes = [_SHP, _P, _P, _I32, _I32, _I32, _CAL, _P]
 _lib.kvq_quantize_append.restype = _I32
 _lib.kvq_quantize_append.argtypes = [_SHP, _CAL, _CCH, _I32, _I32, _P, _P, _I32, _P, _I32, _P, _P]
 _lib.kvq_decode_workspace_bytes.restype = ctypes.c_size_t
@@ -83,7 +85,7 @@ _lib.kvq_round_e2m1.argtypes = [_P, _P, ctypes.c_int64, _P]
 _lib.kvq_round_e4m3.restype = _I32
 _lib.kvq_round_e4m3.argtypes = [_P, _P, ctypes.c_int64, _P]
 
-EXPORTED = ("kvq_page_bytes", "kvq_status_string", "kvq_version", "kvq_calibrate_smoothing",
+EXPORTED = ("kvq_page_bytes", "kvq_status_string", "kvq_version", "kvq_calibrate_smoothing", "kvq_calibrate_native",
             "kvq_quantize_append", "kvq_decode_workspace_bytes", "kvq_decode_attention",
             "kvq_prefill_workspace_bytes", "kvq_prefill_attention", "kvq_decode_attention_noalloc",
             "kvq_round_e2m1", "kvq_round_e4m3", "kvq_selftest_wait_timeout")
@@ -198,6 +200,21 @@ def calibrate_smoothing(shape: Shape, k_calib: torch.Tensor, v_calib: torch.Tens
     _check(_lib.kvq_calibrate_smoothing(ctypes.byref(shape.c()), k_calib.data_ptr(), v_calib.data_ptr(),
                                         _dtype_code(k_calib), W, T, int(bool(exclude_pos0)), ctypes.byref(c),
                                         _stream()), "kvq_calibrate_smoothing")
+    return out
+
+
+def calibrate_native(shape: Shape, k_calib: torch.Tensor, v_calib: torch.Tensor,
+                     out: Optional[Calibration] = None) -> Calibration:
+    """Keys in their native basis (s = 1) with calibrated tensor scales;
+    k/v_calib [L][W][T][Hkv][128]."""
+    _need_cuda(k_calib, v_calib)
+    L, W, T, H, D = k_calib.shape
+    if out is None:
+        out = new_calibration(shape, k_calib.device)
+    c = out.c()
+    _check(_lib.kvq_calibrate_native(ctypes.byref(shape.c()), k_calib.data_ptr(), v_calib.data_ptr(),
+                                     _dtype_code(k_calib), W, T, ctypes.byref(c), _stream()),
+           "kvq_calibrate_native")
     return out
 
 

@@ -93,6 +93,18 @@ kvq_status kvq_calibrate_smoothing(const kvq_shape* shape, const void* k_calib, 
                           (cudaStream_t)stream);
 }
 
+kvq_status kvq_calibrate_native(const kvq_shape* shape, const void* k_calib, const void* v_calib, int32_t dtype,
+                                int32_t num_windows, int32_t window_len, const kvq_calib* out, void* stream) {
+    KVQ_TRY(check_shape(shape));
+    KVQ_TRY(check_calib(out));
+    if (!k_calib || !v_calib || !good_dtype(dtype) || num_windows < 1 || window_len < 1) return KVQ_EINVAL;
+    if (!aligned(k_calib, 16) || !aligned(v_calib, 16)) return KVQ_EINVAL;
+    if (num_windows > 65535 || (long)num_windows * window_len * shape->num_kv_heads > (1L << 28)) return KVQ_EINVAL;
+    KVQ_TRY(check_device());
+    return kvq::calibrate_native(*shape, k_calib, v_calib, dtype, num_windows, window_len, *out,
+                                 (cudaStream_t)stream);
+}
+
 kvq_status kvq_quantize_append(const kvq_shape* shape, const kvq_calib* calib, const kvq_cache* cache,
                                int32_t layer0, int32_t nlayers, const void* k, const void* v, int32_t dtype,
                                const int64_t* slot_mapping, int32_t num_tokens, int32_t* dev_status,

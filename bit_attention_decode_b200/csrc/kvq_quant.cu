@@ -328,6 +328,39 @@ static kvq_status launch_calibrate(const kvq_shape& s, const T* k, const T* v, i
     return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ECUDA;
 }
 
+__global__ void fill_kernel(float* __restrict__ x, float value, int n) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) x[i] = value;
+}
+
+// Native basis: s = inv = 1, then the tensor scales of the unsmoothed keys
+// (the tensor-absmax kernel multiplies by inv = 1, which is exact).
+template <typename T>
+static kvq_status launch_calibrate_native(const kvq_shape& s, const T* k, const T* v, int W, int Tlen,
+                                          const kvq_calib& out, cudaStream_t st) {
+    const int L = s.num_layers, H = s.num_kv_heads;
+    const int n = L * H * kD;
+    if (cudaMemsetAsync(out.k_gscale, 0, L * sizeof(float), st) != cudaSuccess ||
+        cudaMemsetAsync(out.v_gscale, 0, L * sizeof(float), st) != cudaSuccess)
+        return KVQ_ECUDA;
+    fill_kernel<<<(n + 255) / 256, 256, 0, st>>>(out.k_smooth, 1.0f, n);
+    fill_kernel<<<(n + 255) / 256, 256, 0, st>>>(out.k_inv_smooth, 1.0f, n);
+    const long rows = (long)W * Tlen * H;
+    dim3 g3((unsigned)((rows * 8 + 255) / 256), L);
+    calib_tensor_amax_kernel<T><<<g3, 256, 0, st>>>(k, v, W, Tlen, H, out.k_inv_smooth, s.use_hadamard,
+                                                   reinterpret_cast<uint32_t*>(out.k_gscale),
+                                                   reinterpret_cast<uint32_t*>(out.v_gscale));
+    calib_finalize_gscale_kernel<<<(L + 63) / 64, 64, 0, st>>>(out.k_gscale, out.v_gscale, L);
+    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ECUDA;
+}
+
+kvq_status calibrate_native(const kvq_shape& s, const void* k, const void* v, int dtype, int W, int Tlen,
+                            const kvq_calib& out, cudaStream_t st) {
+    if (dtype == KVQ_F32)
+        return launch_calibrate_native(s, (const float*)k, (const float*)v, W, Tlen, out, st);
+    return launch_calibrate_native(s, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, W, Tlen, out, st);
+}
+
 kvq_status calibrate(const kvq_shape& s, const void* k, const void* v, int dtype, int W, int Tlen,
                      int exclude_pos0, const kvq_calib& out, cudaStream_t st) {
     if (dtype == KVQ_F32)

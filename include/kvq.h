@@ -141,6 +141,22 @@ kvq_status kvq_calibrate_smoothing(const kvq_shape* shape, const void* k_calib, 
                                    int32_t exclude_pos0, const kvq_calib* out, void* stream);
 
 /*
+ * kvq_calibrate_native -- tensor scales for keys kept in their native basis.
+ *
+ * [P1] results table, row "NVFP4 K only, native basis": the keys are
+ * quantised without smoothing.  Writes s = 1 and inv = 1 for every (layer,
+ * head, channel) -- so the append, the query pre-transform and attention
+ * run unchanged -- and the FP32 tensor scales of kvq_calibrate_smoothing
+ * over the unsmoothed keys: g_K = max |T(k)| / 2688 with T the optional
+ * rotation alone, g_V = max |v| / 2688, over every calibration token; a zero
+ * maximum gives 1.  Arguments and errors as kvq_calibrate_smoothing, without
+ * exclude_pos0 (there is no smoothing absmax to leave the sink out of).
+ */
+kvq_status kvq_calibrate_native(const kvq_shape* shape, const void* k_calib, const void* v_calib,
+                                int32_t dtype, int32_t num_windows, int32_t window_len,
+                                const kvq_calib* out, void* stream);
+
+/*
  * kvq_quantize_append -- transform, quantise and scatter tokens into the cache.
  *
  * [P1] setup paragraph: NVFP4 on post-RoPE cached keys and values, 16-blocks

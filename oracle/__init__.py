@@ -69,7 +69,7 @@ def _load():
         lib.oracle_e2m1_encode_n.argtypes = [P, P, i64]
         lib.oracle_e4m3_encode_n.argtypes = [P, P, i64]
         lib.oracle_transform_keys.argtypes = [P, P, i64, i32, i32, P]
-        lib.oracle_calibrate.argtypes = [P, P, i32, i32, i32, i32, i32, i32, P, P, P, P]
+        lib.oracle_calibrate.argtypes = [P, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, P]
         lib.oracle_quantize_rows.argtypes = [P, i64, f32, P, P]
         lib.oracle_dequantize_rows.argtypes = [P, P, i64, f32, P]
         lib.oracle_attention.argtypes = [P, i32, i32, i32, i32, P, i32, P, P, i32, P]
@@ -127,8 +127,9 @@ def e4m3_encode(x) -> np.ndarray:
 
 
 # ---------------------------------------------------------------- method steps
-def calibrate(k_calib, v_calib, exclude_pos0: bool = True, hadamard: bool = False):
-    """k/v_calib [L][W][T][H][D] -> (s, inv_s [L][H][D] fp32, g_K, g_V [L] fp32)."""
+def calibrate(k_calib, v_calib, exclude_pos0: bool = True, hadamard: bool = False, smooth: bool = True):
+    """k/v_calib [L][W][T][H][D] -> (s, inv_s [L][H][D] fp32, g_K, g_V [L] fp32).
+    smooth=False keeps the keys in their native basis (s = 1)."""
     k, pk = _c(_f32(k_calib), np.float32)
     v, pv = _c(_f32(v_calib), np.float32)
     L, W, T, H, D = k.shape
@@ -138,7 +139,7 @@ def calibrate(k_calib, v_calib, exclude_pos0: bool = True, hadamard: bool = Fals
     gk = np.empty(L, np.float32)
     gv = np.empty(L, np.float32)
     P = ctypes.c_void_p
-    _load().oracle_calibrate(pk, pv, L, W, T, H, int(bool(exclude_pos0)), int(bool(hadamard)),
+    _load().oracle_calibrate(pk, pv, L, W, T, H, int(bool(exclude_pos0)), int(bool(hadamard)), int(bool(smooth)),
                              s.ctypes.data_as(P), inv.ctypes.data_as(P),
                              gk.ctypes.data_as(P), gv.ctypes.data_as(P))
     return s, inv, gk, gv

@@ -162,8 +162,11 @@ void oracle_transform_keys(const float* k, const float* inv_s, int64_t n, int H,
  * for K (after the transform) and one for V.
  *
  * k, v: [L][W][T][H][D] fp32.  s, inv_s: [L][H][D].  gk, gv: [L]. */
+/* smooth = 0: keys kept in their native basis ([P1] results table, row
+ * "NVFP4 K only, native basis"): s = 1, and the tensor scale is taken over
+ * the unsmoothed (optionally rotated) keys. */
 void oracle_calibrate(const float* k, const float* v, int L, int W, int T, int H,
-                      int exclude_pos0, int hadamard,
+                      int exclude_pos0, int hadamard, int smooth,
                       float* s, float* inv_s, float* gk, float* gv)
 {
     const size_t per_tok = (size_t)H * HD, per_win = (size_t)T * per_tok,
@@ -181,7 +184,7 @@ void oracle_calibrate(const float* k, const float* v, int L, int W, int T, int H
                         float a = fabsf(kl[w * per_win + (size_t)t * per_tok + (size_t)h * HD + c]);
                         if (a > A) A = a;
                     }
-                float sc = (A > 0.0f) ? sqrtf(A) : 1.0f;
+                float sc = (smooth && A > 0.0f) ? sqrtf(A) : 1.0f;
                 sl[h * HD + c] = sc;
                 il[h * HD + c] = 1.0f / sc;
             }

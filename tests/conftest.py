@@ -29,7 +29,13 @@ def read_golden(name):
 @pytest.fixture(scope="session")
 def kvq_lib():
     """The binding module; builds libkvq.so in-tree first if it is missing."""
-    from bit_attention_decode_b200 import build as _build
+    # build.py by path: importing the package would load a stale library first
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "kvq_build", os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                                  "bit_attention_decode_b200", "build.py"))
+    _build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(_build)
     if not _build.up_to_date():
         _build.build()
     import bit_attention_decode_b200 as kvq

@@ -87,7 +87,7 @@ class Problem:
 
 def build_problem(kvq, w: synth.Workload, lens, layers=None, extra_tokens: int = 0, shuffle: bool = True,
                   keep_host=True, device="cuda", gen_device="cpu", keep=None, all_layers_one_call=False,
-                  keep_tails=False):
+                  keep_tails=False, native=False):
     """Calibrate, then append each sequence's first lens[b] tokens.
 
     keep:      optional set of (layer index, sequence) whose host copies are kept
@@ -96,6 +96,7 @@ def build_problem(kvq, w: synth.Workload, lens, layers=None, extra_tokens: int =
                (K/V [nl][T][Hkv][D]) instead of one call per layer.
     keep_tails: also return the extra_tokens tail of every sequence on the
                device, as tails_k/v [extra][nl][B][Hkv][D].
+    native:    calibrate the keys in their native basis (no smoothing).
     """
     layers = list(range(w.num_layers)) if layers is None else list(layers)
     lens = torch.as_tensor(lens, dtype=torch.int32)
@@ -106,7 +107,10 @@ def build_problem(kvq, w: synth.Workload, lens, layers=None, extra_tokens: int =
     kc = torch.stack([x[0] for x in wins])
     vc = torch.stack([x[1] for x in wins])
     del wins
-    calib = kvq.calibrate_smoothing(shape, kc.to(device).contiguous(), vc.to(device).contiguous())
+    if native:
+        calib = kvq.calibrate_native(shape, kc.to(device).contiguous(), vc.to(device).contiguous())
+    else:
+        calib = kvq.calibrate_smoothing(shape, kc.to(device).contiguous(), vc.to(device).contiguous())
     page_table, num_pages = synth.build_page_table(w, lens + extra_tokens, shuffle=shuffle)
     cache = kvq.new_cache(shape, num_pages, device)
     seqs = {}
@@ -142,11 +146,13 @@ def build_problem(kvq, w: synth.Workload, lens, layers=None, extra_tokens: int =
     p = Problem(w, layers, lens, page_table, num_pages, shape, calib, cache,
                 kc.float().cpu().numpy(), vc.float().cpu().numpy(), seqs)
     p.tails = tails
+    p.native = native
     return p
 
 
 def oracle_calibration(p: Problem):
-    return oracle.calibrate(p.k_calib, p.v_calib, exclude_pos0=True, hadamard=p.w.hadamard)
+    return oracle.calibrate(p.k_calib, p.v_calib, exclude_pos0=True, hadamard=p.w.hadamard,
+                            smooth=not getattr(p, "native", False))
 
 
 def calib_host(p: Problem):

@@ -72,6 +72,27 @@ def test_ragged_multilayer_bf16(kvq, hadamard):
                 harness.check_attention(out[li, b], want[0], f"layer {li} seq {b} len {n} {tag}")
 
 
+@pytest.mark.parametrize("hadamard", [False, True])
+def test_native_basis_keys(kvq, hadamard):
+    # "NVFP4 attention cache on W4A4 Qwen3-8B", results table row "NVFP4 K
+    # only, native basis": no smoothing
+    w = small(num_layers=2, batch=3, calib_windows=2, calib_len=64, hadamard=hadamard)
+    lens = [5, 140, 301]
+    p = harness.build_problem(kvq, w, lens=lens, native=True)
+    cal = harness.oracle_calibration(p)
+    assert np.all(cal[0] == 1)
+    for got, want, name in zip(harness.calib_host(p), cal, ("s", "inv_s", "g_K", "g_V")):
+        np.testing.assert_array_equal(got, want, err_msg=name)
+    for li in range(2):
+        for b, n in enumerate(lens):
+            assert_codes_equal(p, li, b, n, cal)
+    q, out = decode_all(kvq, p)
+    for li in range(2):
+        for b, n in enumerate(lens):
+            want = harness.oracle_attend(p, li, b, q[li, b][None], n - 1, n, cal)
+            harness.check_attention(out[li, b], want[0], f"native layer {li} seq {b} len {n}")
+
+
 def test_many_units_single_split(kvq):
     # enough (layer, sequence, head) units that the decode needs no split
     w = small(num_layers=10, batch=64, calib_windows=1, calib_len=32)

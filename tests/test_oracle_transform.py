@@ -80,3 +80,29 @@ def test_calibrate_all_zero_gives_unit_scales():
     z = np.zeros((1, 1, 4, 1, 128), np.float32)
     s, inv, gk, gv = oracle.calibrate(z, z)
     assert np.all(s == 1) and np.all(inv == 1) and gk[0] == 1 and gv[0] == 1
+
+
+def test_calibrate_native_basis_keeps_keys_unsmoothed():
+    # "NVFP4 attention cache on W4A4 Qwen3-8B", results table row "NVFP4 K
+    # only, native basis": no smoothing, so
+    # s = inv = 1 and the key tensor scale is the plain absmax over every
+    # calibration token (the sink of _windows at 50 included)
+    k, v, A = _windows()
+    s, inv, gk, gv = oracle.calibrate(k, v, hadamard=False, smooth=False)
+    assert np.all(s == 1) and np.all(inv == 1)
+    np.testing.assert_array_equal(gk, np.full(2, np.float32(50.0 / 2688.0)))
+    np.testing.assert_array_equal(gv, np.array([4.0 / 2688.0, 13.0 / 2688.0], np.float32))
+
+
+def test_calibrate_native_basis_with_rotation_against_scipy():
+    # with the rotation and no smoothing the key scale is max |H k| / sqrt(128)
+    # over all tokens / 2688; H from scipy (fp64), so compare to a few ulps
+    from scipy.linalg import hadamard
+    rng = np.random.default_rng(7)
+    k = rng.standard_normal((1, 2, 8, 2, 128)).astype(np.float32)
+    v = rng.standard_normal((1, 2, 8, 2, 128)).astype(np.float32)
+    s, inv, gk, gv = oracle.calibrate(k, v, hadamard=True, smooth=False)
+    assert np.all(s == 1)
+    rot = k.astype(np.float64) @ hadamard(128).T / np.sqrt(128.0)
+    np.testing.assert_allclose(gk[0], np.abs(rot).max() / 2688.0, rtol=4e-7)
+    assert gv[0] == np.float32(np.abs(v).max() / 2688.0)
