@@ -33,6 +33,7 @@ import torch  # noqa: E402
 METRIC = "NVFP4-KV decode attention tokens/s; achieved HBM GB/s vs B200 peak"
 FALLBACK_HBM_GBS = 6650.0
 TOKEN_LAYER_BYTES = 1152          # packed K+V codes and scales of 8 heads
+TOKEN_LAYER_BYTES_BF16K = 2624    # mixed cache: bf16 keys (8 x 256 B) + packed values (8 x 72 B)
 QO_BYTES_PER_SEQ_LAYER = 32 * 128 * 2 * 2   # bf16 query in + bf16 output
 
 
@@ -46,6 +47,8 @@ def parse():
                     help="ragged (default, the decode-throughput workload); prefill, qwen3_8b, hadamard: "
                          "the chunked-prefill and prefix workloads, for their own kernel numbers")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--k-format", default="nvfp4", choices=["nvfp4", "bf16"],
+                    help="key storage of the ragged workload: packed NVFP4, or bf16 keys with NVFP4 values")
     ap.add_argument("--source-sha", action="store_true",
                     help="print the hash of the decode kernel's sources (the key of the committed ncu counters) and exit")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -209,10 +212,12 @@ def ncu_traffic():
 class Ragged:
     """Device-resident ragged decode workload (one replica)."""
 
-    def __init__(self, kvq, synth, layers=36):
+    def __init__(self, kvq, synth, layers=36, k_format=0):
         self.kvq = kvq
         import dataclasses
         w = dataclasses.replace(synth.WORKLOADS["ragged"], num_layers=layers)
+        self.k_format = k_format
+        self.tlb = TOKEN_LAYER_BYTES_BF16K if k_format else TOKEN_LAYER_BYTES
         self.w = w
         L, B, S = w.num_layers, w.batch, w.decode_steps
         self.L, self.B, self.S = L, B, S
@@ -220,7 +225,7 @@ class Ragged:
         self.lens = synth.ragged_lengths(w)                          # [B] int32
         cap = self.lens + S
         self.page_table, self.num_pages = synth.build_page_table(w, cap)
-        self.shape = kvq.Shape(L, w.num_q_heads, w.num_kv_heads)
+        self.shape = kvq.Shape(L, w.num_q_heads, w.num_kv_heads, k_format=k_format)
         kc = torch.stack([synth.calibration_windows(w, l, dev)[0] for l in range(L)])
         vc = torch.stack([synth.calibration_windows(w, l, dev)[1] for l in range(L)])
         self.calib = kvq.calibrate_smoothing(self.shape, kc, vc, exclude_pos0=True)
@@ -269,11 +274,11 @@ class Ragged:
         self.launches_per_step = 2 + (1 if need else 0)
         torch.cuda.synchronize()
         # bulk append of each layer's prefix (read bf16 K and V, write codes + scales)
-        self.append_bytes = self.prefix_tokens * (2 * w.num_kv_heads * D * 2 + TOKEN_LAYER_BYTES)
+        self.append_bytes = self.prefix_tokens * (2 * w.num_kv_heads * D * 2 + self.tlb)
 
     def decode_bytes(self, s: int) -> int:
         valid = int(self.lens.sum()) + self.B * (s + 1)
-        return valid * self.L * TOKEN_LAYER_BYTES + self.B * self.L * QO_BYTES_PER_SEQ_LAYER
+        return valid * self.L * self.tlb + self.B * self.L * QO_BYTES_PER_SEQ_LAYER
 
     def append(self, s: int):
         self.kvq.quantize_append(self.shape, self.calib, self.cache, self.k_new[s], self.v_new[s], self.slots[s])
@@ -553,10 +558,14 @@ def cores():
 # ------------------------------------------------------------------ main
 def config_block(wl=None):
     layers = wl.L if wl is not None else 36
+    bf16k = wl is not None and wl.k_format == 1
     return {"workload": f"ragged decode: {layers} layers, 32 q / 8 kv heads, head_dim 128, batch 64, "
                         "lengths U[1024,8192], 16-token pages in shuffled order, 64 append+decode steps cycled",
-            "batch": 64, "layers": layers, "kv_cache": "nvfp4 (e2m1 codes, e4m3 per-16 scales, fp32 tensor scale)",
-            "l2": "inputs larger than L2 (about 12.4 GB of cache read per step)",
+            "batch": 64, "layers": layers,
+            "kv_cache": ("mixed: bf16 keys, nvfp4 values" if bf16k else
+                         "nvfp4 (e2m1 codes, e4m3 per-16 scales, fp32 tensor scale)"),
+            "l2": "inputs larger than L2 (about %.1f GB of cache read per step)" % (
+                (28.2 if bf16k else 12.4) * layers / 36),
             "parallelism": "replicas (independent sequences per GPU)"}
 
 
@@ -655,7 +664,7 @@ def main():
     if args.workload != "ragged":
         return other_workload(args, kvq, synth, rank, world)
     t_setup = time.time()
-    wl = Ragged(kvq, synth, args.layers)
+    wl = Ragged(kvq, synth, args.layers, k_format=1 if args.k_format == "bf16" else 0)
     sys.stderr.write(f"[bench] setup {time.time() - t_setup:.1f} s, {wl.num_pages} pages, "
                      f"cache {wl.cache.data.numel() / 1e9:.2f} GB\n")
     clock = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
@@ -666,7 +675,8 @@ def main():
     dec_avg_ms = statistics.mean(dec_ms)
     achieved = dec_bytes / (dec_avg_ms / 1e3) / 1e9
     peak, peak_kind = measured_peak()
-    traffic = ncu_traffic()
+    # the committed ncu counters are those of the packed-key kernel
+    traffic = ncu_traffic() if wl.k_format == 0 else None
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_block(wl),

@@ -31,12 +31,13 @@ TILE_BYTES = 2304
 KVQ_OK, KVQ_EINVAL, KVQ_ECUDA, KVQ_EUNSUPPORTED, KVQ_EWORKSPACE = 0, 1, 2, 3, 4
 DEV_BAD_PAGE, DEV_BAD_SLOT, DEV_BAD_LEN, DEV_TIMEOUT = 1, 2, 4, 8
 KVQ_F32, KVQ_BF16 = 0, 1
+K_NVFP4, K_BF16 = 0, 1          # kvq_shape.k_format: packed keys, or bf16 keys (mixed cache)
 
 
 class _Shape(ctypes.Structure):
     _fields_ = [("num_layers", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("page_size", ctypes.c_int32), ("use_hadamard", ctypes.c_int32)]
+                ("page_size", ctypes.c_int32), ("use_hadamard", ctypes.c_int32), ("k_format", ctypes.c_int32)]
 
 
 class _Calib(ctypes.Structure):
@@ -120,10 +121,11 @@ class Shape:
     use_hadamard: bool = False
     head_dim: int = HEAD_DIM
     page_size: int = PAGE_SIZE
+    k_format: int = K_NVFP4
 
     def c(self) -> _Shape:
         return _Shape(self.num_layers, self.num_q_heads, self.num_kv_heads, self.head_dim,
-                      self.page_size, int(self.use_hadamard))
+                      self.page_size, int(self.use_hadamard), int(self.k_format))
 
 
 @dataclasses.dataclass

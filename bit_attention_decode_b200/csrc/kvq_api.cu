@@ -21,6 +21,9 @@ kvq_status check_shape(const kvq_shape* s) {
     if (s->use_hadamard != 0 && s->use_hadamard != 1) return KVQ_EINVAL;
     // the rotation's cross-lane butterflies need whole warps of key lanes
     if (s->use_hadamard && (s->num_kv_heads & 1)) return KVQ_EUNSUPPORTED;
+    if (s->k_format != KVQ_K_NVFP4 && s->k_format != KVQ_K_BF16) return KVQ_EINVAL;
+    // bf16 keys are stored untransformed
+    if (s->k_format == KVQ_K_BF16 && s->use_hadamard) return KVQ_EINVAL;
     return KVQ_OK;
 }
 
@@ -42,7 +45,8 @@ kvq_status check_calib(const kvq_calib* c) {
 kvq_status check_cache(const kvq_shape* s, const kvq_cache* c) {
     if (!c || !c->data || c->num_pages < 1) return KVQ_EINVAL;
     if (!aligned(c->data, 16) || (c->layer_stride_bytes & 15) != 0) return KVQ_EINVAL;
-    if (c->layer_stride_bytes < (int64_t)c->num_pages * s->num_kv_heads * kvq::kTile) return KVQ_EINVAL;
+    if (c->layer_stride_bytes < (int64_t)c->num_pages * s->num_kv_heads * kvq::tile_bytes(s->k_format))
+        return KVQ_EINVAL;
     return KVQ_OK;
 }
 
@@ -63,7 +67,7 @@ extern "C" {
 
 size_t kvq_page_bytes(const kvq_shape* shape) {
     if (check_shape(shape) != KVQ_OK) return 0;
-    return (size_t)shape->num_kv_heads * kvq::kTile;
+    return (size_t)shape->num_kv_heads * kvq::tile_bytes(shape->k_format);
 }
 
 const char* kvq_status_string(kvq_status st) {
@@ -159,6 +163,8 @@ kvq_status kvq_prefill_attention(const kvq_shape* shape, const kvq_calib* calib,
                                  const int32_t* seq_lens, int32_t batch, void* out, int32_t out_dtype,
                                  void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
     KVQ_TRY(check_shape(shape));
+    // the tensor-core prefill dequantises NVFP4 keys only
+    if (shape->k_format != KVQ_K_NVFP4) return KVQ_EUNSUPPORTED;
     KVQ_TRY(check_calib(calib));
     KVQ_TRY(check_cache(shape, cache));
     KVQ_TRY(check_layers(shape, layer0, nlayers));

@@ -12,6 +12,7 @@ struct AttnArgs {
     const uint8_t* cache;      // layer layer0
     int64_t layer_stride;
     int num_pages, Hkv, Hq, G, hadamard;
+    int kbf16;                 // keys stored as bf16 (mixed cache)
     const float* smooth;       // [nl][Hkv][D] at layer0
     const float* gk;           // [nl] at layer0
     const float* gv;
@@ -29,7 +30,7 @@ struct AttnArgs {
 
 // tensor-core split-K decode (kvq_decode_tc.cu)
 cudaError_t launch_decode_tc(const AttnArgs& a, int nlayers, bool q_bf16, bool out_bf16, cudaStream_t st);
-size_t decode_tc_smem(int Hkv);
+size_t decode_tc_smem(int Hkv, bool kbf16);
 // tensor-core (tcgen05) chunked causal prefill (kvq_prefill_tc.cu)
 cudaError_t launch_prefill_tc(const AttnArgs& a, int nlayers, bool q_bf16, bool out_bf16, cudaStream_t st);
 

@@ -22,6 +22,11 @@ constexpr int kKCodes = 0;       // 16 rows x 64 B
 constexpr int kKScales = 1024;   // 16 rows x 8 B, token-major
 constexpr int kVCodes = 1152;    // 16 rows x 64 B
 constexpr int kVScales = 2176;   // 8 blocks x 16 B, block-major
+// mixed cache (BF16 keys, NVFP4 values): 5248-byte tiles
+constexpr int kTileBf16K = 5248;
+constexpr int kBf16VCodes = 4096;    // after 16 rows x 256 B of bf16 keys
+constexpr int kBf16VScales = 5120;
+__host__ __device__ constexpr int tile_bytes(int k_format) { return k_format == KVQ_K_BF16 ? kTileBf16K : kTile; }
 
 // fp32 nearest to 1/sqrt(128): the normalisation of the Hadamard-128 rotation
 constexpr float kInvSqrt128 = 0.08838834764831845f;

@@ -97,6 +97,7 @@ static AttnArgs make_args(const kvq_shape& s, const kvq_calib& c, const kvq_cach
     a.Hq = s.num_q_heads;
     a.G = s.num_q_heads / s.num_kv_heads;
     a.hadamard = s.use_hadamard;
+    a.kbf16 = s.k_format == KVQ_K_BF16;
     a.smooth = c.k_smooth + (size_t)layer0 * s.num_kv_heads * kD;
     a.gk = c.k_gscale + layer0;
     a.gv = c.v_gscale + layer0;

@@ -42,6 +42,22 @@ __device__ __forceinline__ void mma16816(float* d, uint32_t a0, uint32_t a1, uin
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+// the same with bf16 operands (keys of the mixed cache)
+__device__ __forceinline__ void mma16816_bf16(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+    __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ float2 unpack_bf2(uint32_t a) {
+    return make_float2(__uint_as_float(a << 16), __uint_as_float(a & 0xFFFF0000u));
+}
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
     uint32_t d;
     asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
@@ -117,16 +133,21 @@ __device__ __forceinline__ void store16(__nv_bfloat16* p, const float* x) {
 // ------------------------------------------------------------------ kernel
 // grid (splits, nlayers, batch); block 32 * (Hkv + 1); dynamic smem
 // kStages * Hkv * 2304 + barriers.
-template <typename TQ, typename TO>
+template <typename TQ, typename TO, bool KB>
 __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
+    // KB: keys stored as bf16 (mixed cache, 5248-byte tiles, 2 stages)
+    constexpr int kST = KB ? 2 : kStages;
+    constexpr int kTB = KB ? kTileBf16K : kTile;
+    constexpr int kVC = KB ? kBf16VCodes : kVCodes;
+    constexpr int kVS = KB ? kBf16VScales : kVScales;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ int s_flags;    // 1: a bounded wait gave up
     __shared__ int s_issued;   // pages the producer issued
 
     const int Hkv = a.Hkv;
-    const uint32_t page_bytes = (uint32_t)Hkv * kTile;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * page_bytes);
-    uint64_t* empty = full + kStages;
+    const uint32_t page_bytes = (uint32_t)Hkv * kTB;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kST * page_bytes);
+    uint64_t* empty = full + kST;
 
     __shared__ int s_seq;      // sequence of this CTA (longest-first order)
     const int split = blockIdx.x, li = blockIdx.y;
@@ -162,7 +183,7 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
     if (threadIdx.x == 0) {
         s_flags = 0;
         s_issued = 0;
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kST; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], Hkv);
         }
@@ -193,8 +214,8 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
         if (lane == 0 && !poison) {
             int i = 0;
             for (; i < n; ++i) {
-                const int st = i % kStages;
-                if (i >= kStages && !mbar_wait(&empty[st], ((i / kStages) - 1) & 1)) {
+                const int st = i % kST;
+                if (i >= kST && !mbar_wait(&empty[st], ((i / kST) - 1) & 1)) {
                     atomicOr(&s_flags, 1);
                     break;
                 }
@@ -216,11 +237,19 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
             const TQ* qs = reinterpret_cast<const TQ*>(a.q) +
                            (((size_t)li * a.batch + b) * a.Hq + h * G + (head_ok ? jq : 0)) * kD + 32 * c;
             load32<TQ>(qs, qv);
-            const float* srow = a.smooth + ((size_t)li * Hkv + h) * kD + 32 * c;
+            float scale;
+            if constexpr (KB) {
+                // bf16 keys are stored as given: the query is used unchanged
 #pragma unroll
-            for (int i = 0; i < 32; ++i) qv[i] = head_ok ? qv[i] * __ldg(srow + i) : 0.0f;
-            float scale = __ldg(a.gk + li) * kLog2e * kInvSqrt128;
-            if (a.hadamard) {
+                for (int i = 0; i < 32; ++i) qv[i] = head_ok ? qv[i] : 0.0f;
+                scale = kLog2e * kInvSqrt128;
+            } else {
+                const float* srow = a.smooth + ((size_t)li * Hkv + h) * kD + 32 * c;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) qv[i] = head_ok ? qv[i] * __ldg(srow + i) : 0.0f;
+                scale = __ldg(a.gk + li) * kLog2e * kInvSqrt128;
+            }
+            if (!KB && a.hadamard) {
 #pragma unroll
                 for (int hh = 1; hh < 32; hh <<= 1)
 #pragma unroll
@@ -262,41 +291,72 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 const float x0 = qv[4 * s + 2 * r] * sig, x1 = qv[4 * s + 2 * r + 1] * sig;
-                const uint32_t hv = pack_h2(x0, x1);
-                const float2 f = unpack_h2(hv);
-                qb[2 * s + r] = (g < 4) ? hv : pack_h2(x0 - f.x, x1 - f.y);
+                if constexpr (KB) {
+                    // bf16 hi + lo: 16 significant bits of the query
+                    const uint32_t hv = pack_bf2(x0, x1);
+                    const float2 f = unpack_bf2(hv);
+                    qb[2 * s + r] = (g < 4) ? hv : pack_bf2(x0 - f.x, x1 - f.y);
+                } else {
+                    const uint32_t hv = pack_h2(x0, x1);
+                    const float2 f = unpack_h2(hv);
+                    qb[2 * s + r] = (g < 4) ? hv : pack_h2(x0 - f.x, x1 - f.y);
+                }
             }
         const int ha = 2 * (c & 1), hb = ha + 1;   // heads of this lane's score columns
         const float isg_a = __shfl_sync(kFull, isig, ha * 4);
         const float isg_b = __shfl_sync(kFull, isig, hb * 4);
 
-        const uint8_t* my_tile = smem + h * kTile;
+        const uint8_t* my_tile = smem + h * kTB;
         for (int i = 0; i < n; ++i) {
-            const int st = i % kStages;
-            if (!mbar_wait(&full[st], (i / kStages) & 1)) {
+            const int st = i % kST;
+            if (!mbar_wait(&full[st], (i / kST) & 1)) {
                 atomicOr(&s_flags, 1);
                 break;
             }
             const uint8_t* T = my_tile + st * page_bytes;
             const int nvalid = min(kPage, len - (p0 + i) * kPage);
-            // ---- everything this warp needs from the stage, then release it
-            const uint4 kA = *reinterpret_cast<const uint4*>(T + kKCodes + g * 64 + 16 * c);
-            const uint4 kB = *reinterpret_cast<const uint4*>(T + kKCodes + (g + 8) * 64 + 16 * c);
-            const uint32_t ksA = *reinterpret_cast<const uint16_t*>(T + kKScales + g * 8 + 2 * c);
-            const uint32_t ksB = *reinterpret_cast<const uint16_t*>(T + kKScales + (g + 8) * 8 + 2 * c);
-            const uint2 v0 = *reinterpret_cast<const uint2*>(T + kVCodes + (2 * c) * 64 + 8 * g);
-            const uint2 v1 = *reinterpret_cast<const uint2*>(T + kVCodes + (2 * c + 1) * 64 + 8 * g);
-            const uint2 v2 = *reinterpret_cast<const uint2*>(T + kVCodes + (2 * c + 8) * 64 + 8 * g);
-            const uint2 v3 = *reinterpret_cast<const uint2*>(T + kVCodes + (2 * c + 9) * 64 + 8 * g);
-            uint32_t vs01 = *reinterpret_cast<const uint16_t*>(T + kVScales + 16 * g + 2 * c);
-            uint32_t vs89 = *reinterpret_cast<const uint16_t*>(T + kVScales + 16 * g + 2 * c + 8);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st]);
-
+            uint2 v0, v1, v2, v3;
+            uint32_t vs01, vs89;
             // ---- S = K q~ : tokens (rows) x [4 heads hi | 4 heads lo] (cols);
-            // two accumulators (even / odd code words) halve the dependent MMA chain
+            // two accumulators (even / odd words) halve the dependent MMA chain
             float sacc[4] = {0.0f, 0.0f, 0.0f, 0.0f}, sacc2[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            {
+            if constexpr (KB) {
+                v0 = *reinterpret_cast<const uint2*>(T + kVC + (2 * c) * 64 + 8 * g);
+                v1 = *reinterpret_cast<const uint2*>(T + kVC + (2 * c + 1) * 64 + 8 * g);
+                v2 = *reinterpret_cast<const uint2*>(T + kVC + (2 * c + 8) * 64 + 8 * g);
+                v3 = *reinterpret_cast<const uint2*>(T + kVC + (2 * c + 9) * 64 + 8 * g);
+                vs01 = *reinterpret_cast<const uint16_t*>(T + kVS + 16 * g + 2 * c);
+                vs89 = *reinterpret_cast<const uint16_t*>(T + kVS + 16 * g + 2 * c + 8);
+                // bf16 key rows g and g + 8, dims 32c..32c+31: 16 bytes give
+                // the A operands of two k-steps, in the order of the query's
+                // B operands (the same contraction order as the packed keys)
+                const uint8_t* ra = T + g * 256 + 64 * c;
+                const uint8_t* rb = ra + 8 * 256;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const uint4 x = *reinterpret_cast<const uint4*>(ra + 16 * u);
+                    const uint4 y = *reinterpret_cast<const uint4*>(rb + 16 * u);
+                    float* acc = (u & 1) ? sacc2 : sacc;
+                    mma16816_bf16(acc, x.x, y.x, x.y, y.y, qb[4 * u], qb[4 * u + 1]);
+                    mma16816_bf16(acc, x.z, y.z, x.w, y.w, qb[4 * u + 2], qb[4 * u + 3]);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[st]);
+            } else {
+                // everything this warp needs from the stage, then release it
+                const uint4 kA = *reinterpret_cast<const uint4*>(T + kKCodes + g * 64 + 16 * c);
+                const uint4 kB = *reinterpret_cast<const uint4*>(T + kKCodes + (g + 8) * 64 + 16 * c);
+                const uint32_t ksA = *reinterpret_cast<const uint16_t*>(T + kKScales + g * 8 + 2 * c);
+                const uint32_t ksB = *reinterpret_cast<const uint16_t*>(T + kKScales + (g + 8) * 8 + 2 * c);
+                v0 = *reinterpret_cast<const uint2*>(T + kVC + (2 * c) * 64 + 8 * g);
+                v1 = *reinterpret_cast<const uint2*>(T + kVC + (2 * c + 1) * 64 + 8 * g);
+                v2 = *reinterpret_cast<const uint2*>(T + kVC + (2 * c + 8) * 64 + 8 * g);
+                v3 = *reinterpret_cast<const uint2*>(T + kVC + (2 * c + 9) * 64 + 8 * g);
+                vs01 = *reinterpret_cast<const uint16_t*>(T + kVS + 16 * g + 2 * c);
+                vs89 = *reinterpret_cast<const uint16_t*>(T + kVS + 16 * g + 2 * c + 8);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[st]);
+
                 const uint32_t sfA = e4m3x2_to_f16x2(ksA), sfB = e4m3x2_to_f16x2(ksB);
                 const uint32_t sc[4] = {bcast_lo(sfA), bcast_hi(sfA), bcast_lo(sfB), bcast_hi(sfB)};
                 const uint32_t wa[4] = {kA.x, kA.y, kA.z, kA.w}, wb[4] = {kB.x, kB.y, kB.z, kB.w};
@@ -313,9 +373,9 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
                     mma16816(acc, hmul2(ra[2], sa), hmul2(rb[2], sb), hmul2(ra[3], sa), hmul2(rb[3], sb),
                              qb[4 * w + 2], qb[4 * w + 3]);
                 }
-#pragma unroll
-                for (int k = 0; k < 4; ++k) sacc[k] += sacc2[k];
             }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) sacc[k] += sacc2[k];
             // hi + lo columns -> full scores of heads ha, hb for tokens g, g + 8
             float s0 = sacc[0] + __shfl_xor_sync(kFull, sacc[0], 2);
             float s1 = sacc[1] + __shfl_xor_sync(kFull, sacc[1], 2);
@@ -393,9 +453,9 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
     if (timed_out && threadIdx.x == 32 * Hkv) {
         // drain: wait (bounded) for every copy still in flight before exiting
         const int issued = s_issued;
-        for (int st = 0; st < kStages && st < issued; ++st) {
-            const int last = st + ((issued - 1 - st) / kStages) * kStages;
-            (void)mbar_wait(&full[st], (last / kStages) & 1);
+        for (int st = 0; st < kST && st < issued; ++st) {
+            const int last = st + ((issued - 1 - st) / kST) * kST;
+            (void)mbar_wait(&full[st], (last / kST) & 1);
         }
         set_status(a.status, KVQ_DEV_TIMEOUT);
     }
@@ -442,24 +502,33 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
 }
 
 // ------------------------------------------------------------------ launcher
-size_t decode_tc_smem(int Hkv) { return (size_t)kStages * Hkv * kTile + 2 * kStages * sizeof(uint64_t); }
+size_t decode_tc_smem(int Hkv, bool kbf16) {
+    const int stages = kbf16 ? 2 : kStages;
+    return (size_t)stages * Hkv * (kbf16 ? kTileBf16K : kTile) + 2 * stages * sizeof(uint64_t);
+}
 
-template <typename TQ, typename TO>
+template <typename TQ, typename TO, bool KB>
 static cudaError_t launch_one(const AttnArgs& a, dim3 grid, cudaStream_t st) {
-    const size_t smem = decode_tc_smem(a.Hkv);
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<TQ, TO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const size_t smem = decode_tc_smem(a.Hkv, KB);
+    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<TQ, TO, KB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    decode_tc_kernel<TQ, TO><<<grid, 32 * (a.Hkv + 1), smem, st>>>(a);
+    decode_tc_kernel<TQ, TO, KB><<<grid, 32 * (a.Hkv + 1), smem, st>>>(a);
     return cudaGetLastError();
+}
+
+template <bool KB>
+static cudaError_t launch_kf(const AttnArgs& a, dim3 grid, bool q_bf16, bool out_bf16, cudaStream_t st) {
+    if (q_bf16 && out_bf16) return launch_one<__nv_bfloat16, __nv_bfloat16, KB>(a, grid, st);
+    if (q_bf16) return launch_one<__nv_bfloat16, float, KB>(a, grid, st);
+    if (out_bf16) return launch_one<float, __nv_bfloat16, KB>(a, grid, st);
+    return launch_one<float, float, KB>(a, grid, st);
 }
 
 cudaError_t launch_decode_tc(const AttnArgs& a, int nlayers, bool q_bf16, bool out_bf16, cudaStream_t st) {
     dim3 grid(a.splits, nlayers, a.batch);
-    if (q_bf16 && out_bf16) return launch_one<__nv_bfloat16, __nv_bfloat16>(a, grid, st);
-    if (q_bf16) return launch_one<__nv_bfloat16, float>(a, grid, st);
-    if (out_bf16) return launch_one<float, __nv_bfloat16>(a, grid, st);
-    return launch_one<float, float>(a, grid, st);
+    if (a.kbf16) return launch_kf<true>(a, grid, q_bf16, out_bf16, st);
+    return launch_kf<false>(a, grid, q_bf16, out_bf16, st);
 }
 
 }  // namespace kvq

@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(288, 2)
 append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* __restrict__ slots,
               int num_tokens, int nlayers, int Hkv, int tc, const float* __restrict__ inv_s,
               const float* __restrict__ gk, const float* __restrict__ gv, uint8_t* __restrict__ cache,
-              int64_t layer_stride, int num_pages, int hadamard, int32_t* __restrict__ status) {
+              int64_t layer_stride, int num_pages, int hadamard, int k_bf16, int32_t* __restrict__ status) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t full[kAppendStages], empty[kAppendStages];
     __shared__ int64_t s_slot[kAppendStages][kAppendMaxChunk];
@@ -158,6 +158,9 @@ append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* _
     const int workers = 8;                                     // warps 0..7; warp 8 streams the inputs
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t num_slots = (int64_t)num_pages * kPage;
+    // tile geometry: NVFP4 keys, or bf16 keys (mixed cache)
+    const int tile_b = k_bf16 ? kTileBf16K : kTile;
+    const int v_codes = k_bf16 ? kBf16VCodes : kVCodes, v_scales = k_bf16 ? kBf16VScales : kVScales;
 
     if (threadIdx.x == 0) {
         s_timeout = 0;
@@ -258,25 +261,40 @@ append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* _
                 const size_t e = (size_t)(live ? tt : 0) * row + h * kD + blk * kBlk;
                 float2 y[kBlk / 2];
                 load16(stage + e, y);
-                // key: smoothing multiply, then the optional rotation
-#pragma unroll
-                for (int i = 0; i < kBlk / 2; ++i) y[i] = fmul2(y[i], inv[i]);
-                if (hadamard) hadamard_block(y, blk);
-                uint2 codes;
-                uint32_t sf;
-                quantize_block(y, enc_k, rtab_k, codes, sf);
                 const int64_t page = slot >> 4;
                 const int off = (int)(slot & 15);
-                uint8_t* tile = layer_cache + ((size_t)page * Hkv + h) * kTile;
-                if (ok) {
-                    *reinterpret_cast<uint2*>(tile + kKCodes + off * 64 + blk * 8) = codes;
-                    tile[kKScales + off * 8 + blk] = (uint8_t)sf;
+                uint8_t* tile = layer_cache + ((size_t)page * Hkv + h) * tile_b;
+                uint2 codes;
+                uint32_t sf;
+                if (k_bf16) {
+                    // mixed cache: the key block is kept as bf16, untransformed
+                    if (ok) {
+                        uint32_t wb[8];
+#pragma unroll
+                        for (int i = 0; i < kBlk / 2; ++i) {
+                            const __nv_bfloat162 t2 = __floats2bfloat162_rn(y[i].x, y[i].y);
+                            wb[i] = *reinterpret_cast<const uint32_t*>(&t2);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(tile + off * 256 + blk * 32);
+                        dst[0] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+                        dst[1] = make_uint4(wb[4], wb[5], wb[6], wb[7]);
+                    }
+                } else {
+                    // key: smoothing multiply, then the optional rotation
+#pragma unroll
+                    for (int i = 0; i < kBlk / 2; ++i) y[i] = fmul2(y[i], inv[i]);
+                    if (hadamard) hadamard_block(y, blk);
+                    quantize_block(y, enc_k, rtab_k, codes, sf);
+                    if (ok) {
+                        *reinterpret_cast<uint2*>(tile + kKCodes + off * 64 + blk * 8) = codes;
+                        tile[kKScales + off * 8 + blk] = (uint8_t)sf;
+                    }
                 }
                 load16(stage + half_stage / sizeof(T) + e, y);
                 quantize_block(y, enc_v, rtab_v, codes, sf);
                 if (ok) {
-                    *reinterpret_cast<uint2*>(tile + kVCodes + off * 64 + blk * 8) = codes;
-                    tile[kVScales + blk * 16 + off] = (uint8_t)sf;
+                    *reinterpret_cast<uint2*>(tile + v_codes + off * 64 + blk * 8) = codes;
+                    tile[v_scales + blk * 16 + off] = (uint8_t)sf;
                 }
             }
             __syncwarp();
@@ -372,6 +390,7 @@ kvq_status quantize_append(const kvq_shape& s, const kvq_calib& c, const kvq_cac
                            int nlayers, const void* k, const void* v, int dtype, const int64_t* slots,
                            int num_tokens, int32_t* status, cudaStream_t st) {
     const int H = s.num_kv_heads;
+    const int kbf = s.k_format == KVQ_K_BF16 ? 1 : 0;
     const float* inv_s = c.k_inv_smooth + (size_t)layer0 * H * kD;
     const float* gk = c.k_gscale + layer0;
     const float* gv = c.v_gscale + layer0;
@@ -399,11 +418,11 @@ kvq_status quantize_append(const kvq_shape& s, const kvq_calib& c, const kvq_cac
     if (dtype == KVQ_F32)
         append_kernel<float><<<grid, threads, smem, st>>>((const float*)k, (const float*)v, slots, num_tokens,
                                                         nlayers, H, tc, inv_s, gk, gv, base, cache.layer_stride_bytes,
-                                                        cache.num_pages, s.use_hadamard, status);
+                                                        cache.num_pages, s.use_hadamard, kbf, status);
     else
         append_kernel<__nv_bfloat16><<<grid, threads, smem, st>>>(
             (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, slots, num_tokens, nlayers, H, tc, inv_s, gk, gv, base,
-            cache.layer_stride_bytes, cache.num_pages, s.use_hadamard, status);
+            cache.layer_stride_bytes, cache.num_pages, s.use_hadamard, kbf, status);
     return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ECUDA;
 }
 

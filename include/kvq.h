@@ -47,6 +47,15 @@
  * scale byte b*16+t are the E4M3 scales of elements 16b..16b+15 of token t.
  * Keys are stored in the transformed basis (smoothed, optionally rotated).
  * A cache slot is page * 16 + offset.
+ *
+ * Mixed cache (shape->k_format = KVQ_K_BF16; [P1] results table, row "NVFP4
+ * V only": the keys stay in BF16, the values are NVFP4).  The tile of one kv
+ * head is 5248 bytes:
+ *     bytes [   0, 4096)  keys         16 tokens x 128 bf16, untransformed
+ *     bytes [4096, 5120)  value codes  16 tokens x 64 B
+ *     bytes [5120, 5248)  value scales 8 blocks x 16 B  (block-major)
+ * The keys are neither smoothed nor rotated (use_hadamard must be 0), and
+ * the key entries of kvq_calib are not read.
  */
 #ifndef KVQ_H
 #define KVQ_H
@@ -77,9 +86,13 @@ enum {
 
 enum { KVQ_F32 = 0, KVQ_BF16 = 1 };
 
+/* key storage of the cache (kvq_shape.k_format) */
+enum { KVQ_K_NVFP4 = 0, KVQ_K_BF16 = 1 };
+
 #define KVQ_HEAD_DIM 128
 #define KVQ_PAGE_SIZE 16
-#define KVQ_TILE_BYTES 2304   /* one kv head of one page (see layout above) */
+#define KVQ_TILE_BYTES 2304        /* one kv head of one page (see layout above) */
+#define KVQ_TILE_BYTES_BF16K 5248  /* the same with KVQ_K_BF16 keys             */
 
 typedef struct {
     int32_t num_layers;     /* L                                           */
@@ -88,6 +101,7 @@ typedef struct {
     int32_t head_dim;       /* must be 128                                  */
     int32_t page_size;      /* must be 16                                   */
     int32_t use_hadamard;   /* 1: keys rotated by normalised Hadamard-128   */
+    int32_t k_format;       /* KVQ_K_NVFP4, or KVQ_K_BF16 (mixed cache)     */
 } kvq_shape;
 
 /* Static calibration state, device arrays of fp32 written by
@@ -105,7 +119,8 @@ typedef struct {
     int32_t num_pages;          /* pages per layer                           */
 } kvq_cache;
 
-/* Bytes of one page of one layer: num_kv_heads * 2304; 0 on a bad shape. */
+/* Bytes of one page of one layer: num_kv_heads * 2304 (5248 with BF16
+ * keys); 0 on a bad shape. */
 size_t kvq_page_bytes(const kvq_shape* shape);
 
 /* Text of a status code (static storage). */
@@ -172,6 +187,8 @@ kvq_status kvq_calibrate_native(const kvq_shape* shape, const void* k_calib, con
  *   slot_mapping      [num_tokens] int64 cache slot of each token (the same
  *                     for every layer); a negative slot skips the token.
  *   num_tokens        may be 0 (nothing is launched).
+ * With KVQ_K_BF16 keys only the values are quantised; the keys are stored
+ * as bf16 (bf16 input copied, fp32 input rounded to nearest-even).
  * Errors: KVQ_EINVAL for bad pointers/sizes; slots >= num_pages*16 set
  * KVQ_DEV_BAD_SLOT and are skipped.
  */
@@ -204,6 +221,8 @@ size_t kvq_decode_workspace_bytes(const kvq_shape* shape, int32_t nlayers, int32
  *   out          [nlayers][batch][Hq][128], out_dtype.
  *   workspace    >= kvq_decode_workspace_bytes(...) bytes, 16-byte aligned;
  *                scratch for split partials, contents undefined after.
+ * With KVQ_K_BF16 keys the query is used as given (no smoothing, no
+ * rotation, no key tensor scale): scores are q . k / sqrt(128).
  * Errors: KVQ_EINVAL / KVQ_EWORKSPACE on the host; KVQ_DEV_BAD_PAGE and
  * KVQ_DEV_BAD_LEN on the device (the affected rows are written as zeros).
  */
@@ -228,6 +247,7 @@ size_t kvq_prefill_workspace_bytes(const kvq_shape* shape, int32_t nlayers, int3
  *
  *   q      [nlayers][batch][q_len][Hq][128], q_dtype.
  *   q_start [batch] int32.   out [nlayers][batch][q_len][Hq][128].
+ * A KVQ_K_BF16 cache is not supported here (KVQ_EUNSUPPORTED).
  */
 kvq_status kvq_prefill_attention(const kvq_shape* shape, const kvq_calib* calib, const kvq_cache* cache,
                                  int32_t layer0, int32_t nlayers, const void* q, int32_t q_dtype,

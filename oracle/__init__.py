@@ -189,6 +189,17 @@ def attention(q, q_start: int, s, kx, vx, hadamard: bool = False) -> np.ndarray:
     return out
 
 
+def round_bf16(x) -> np.ndarray:
+    """fp32 -> nearest bf16 value (ties to even), returned as fp32.  A bf16 is
+    the upper half of an fp32 encoding; rounding adds half a unit of the kept
+    part (0x7FFF, plus one when the kept part is odd) before the lower half is
+    dropped.  The keys of the mixed cache ([P1] results table, row "NVFP4 V
+    only": keys in BF16) are stored this way."""
+    b = np.ascontiguousarray(x, np.float32).view(np.uint32).astype(np.uint64)
+    r = (b + 0x7FFF + ((b >> 16) & 1)) & 0xFFFF0000
+    return r.astype(np.uint32).view(np.float32)
+
+
 # ---------------------------------------------------------------- composites
 def quantize_kv(k, v, inv_s, g_k: float, g_v: float, hadamard: bool = False):
     """Quantise one layer's tokens: k, v [n][H][D] -> dict of codes and scales."""

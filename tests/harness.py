@@ -53,13 +53,22 @@ def unpack_nibbles(b: np.ndarray) -> np.ndarray:
     return out
 
 
-def read_tokens(cache_layer: np.ndarray, Hkv: int, page_table_row: np.ndarray, n: int):
+def read_tokens(cache_layer: np.ndarray, Hkv: int, page_table_row: np.ndarray, n: int, k_format: int = 0):
     """Codes and scales of tokens 0..n-1 of one sequence, in logical layout:
-    kc, vc [n][H][128] one code per byte; ksf, vsf [n][H][8]."""
-    tiles = cache_layer.reshape(cache_layer.shape[0], Hkv, 2304)
+    kc, vc [n][H][128] one code per byte; ksf, vsf [n][H][8].  With bf16 keys
+    (k_format 1) kc holds the key values as fp32 [n][H][128] and ksf is None."""
     t = np.arange(n)
     pages = page_table_row[t // 16]
     off = t % 16
+    if k_format == 1:
+        tiles = cache_layer.reshape(cache_layer.shape[0], Hkv, 5248)
+        sel = tiles[pages]                               # [n][H][5248]
+        kb = np.ascontiguousarray(sel[:, :, 0:4096]).view(np.uint16).reshape(n, Hkv, 16, 128)[np.arange(n), :, off]
+        kx = (kb.astype(np.uint32) << 16).view(np.float32)
+        vcb = sel[:, :, 4096:5120].reshape(n, Hkv, 16, 64)[np.arange(n), :, off]
+        vsf = sel[:, :, 5120:5248].reshape(n, Hkv, 8, 16)[np.arange(n), :, :, off]
+        return kx, None, unpack_nibbles(vcb), vsf
+    tiles = cache_layer.reshape(cache_layer.shape[0], Hkv, 2304)
     sel = tiles[pages]                                   # [n][H][2304]
     kcb = sel[:, :, 0:1024].reshape(n, Hkv, 16, 64)[np.arange(n), :, off]
     ksf = sel[:, :, 1024:1152].reshape(n, Hkv, 16, 8)[np.arange(n), :, off]
@@ -87,7 +96,7 @@ class Problem:
 
 def build_problem(kvq, w: synth.Workload, lens, layers=None, extra_tokens: int = 0, shuffle: bool = True,
                   keep_host=True, device="cuda", gen_device="cpu", keep=None, all_layers_one_call=False,
-                  keep_tails=False, native=False):
+                  keep_tails=False, native=False, k_format=0):
     """Calibrate, then append each sequence's first lens[b] tokens.
 
     keep:      optional set of (layer index, sequence) whose host copies are kept
@@ -97,12 +106,13 @@ def build_problem(kvq, w: synth.Workload, lens, layers=None, extra_tokens: int =
     keep_tails: also return the extra_tokens tail of every sequence on the
                device, as tails_k/v [extra][nl][B][Hkv][D].
     native:    calibrate the keys in their native basis (no smoothing).
+    k_format:  1 for the mixed cache (bf16 keys, NVFP4 values).
     """
     layers = list(range(w.num_layers)) if layers is None else list(layers)
     lens = torch.as_tensor(lens, dtype=torch.int32)
     nl, B = len(layers), len(lens)
     shape = kvq.Shape(num_layers=nl, num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads,
-                      use_hadamard=w.hadamard)
+                      use_hadamard=w.hadamard, k_format=k_format)
     wins = [synth.calibration_windows(w, l, gen_device) for l in layers]
     kc = torch.stack([x[0] for x in wins])
     vc = torch.stack([x[1] for x in wins])
@@ -147,6 +157,7 @@ def build_problem(kvq, w: synth.Workload, lens, layers=None, extra_tokens: int =
                 kc.float().cpu().numpy(), vc.float().cpu().numpy(), seqs)
     p.tails = tails
     p.native = native
+    p.k_format = k_format
     return p
 
 
@@ -161,9 +172,13 @@ def calib_host(p: Problem):
 
 
 def oracle_sequence(p: Problem, li: int, b: int, n: int, cal):
-    """Oracle codes of tokens 0..n-1 of sequence b in layer li."""
+    """Oracle codes of tokens 0..n-1 of sequence b in layer li (with bf16
+    keys: kc = the rounded key values, ksf = None)."""
     s, inv, gk, gv = cal
     k, v = p.seqs[(li, b)]
+    if getattr(p, "k_format", 0) == 1:
+        vc, vsf = oracle.quantize_rows(v[:n], gv[li])
+        return {"kc": oracle.round_bf16(k[:n]), "ksf": None, "vc": vc, "vsf": vsf}
     return oracle.quantize_kv(k[:n], v[:n], inv[li], gk[li], gv[li], p.w.hadamard)
 
 
@@ -171,6 +186,9 @@ def oracle_attend(p: Problem, li: int, b: int, q_rows: np.ndarray, q_start: int,
     """Oracle attention of q_rows [Tq][Hq][D] over the first n tokens."""
     s, inv, gk, gv = cal
     qz = oracle_sequence(p, li, b, n, cal)
-    kx = oracle.dequantize_rows(qz["kc"], qz["ksf"], gk[li])
     vx = oracle.dequantize_rows(qz["vc"], qz["vsf"], gv[li])
+    if getattr(p, "k_format", 0) == 1:
+        # bf16 keys: the query is used as given, the keys as stored
+        return oracle.attention(q_rows, q_start, np.ones_like(s[li]), qz["kc"].astype(np.float64), vx, False)
+    kx = oracle.dequantize_rows(qz["kc"], qz["ksf"], gk[li])
     return oracle.attention(q_rows, q_start, s[li], kx, vx, p.w.hadamard)

@@ -22,10 +22,14 @@ def small(name="qwen3_8b", **kw):
 
 def assert_codes_equal(p, li, b, n, cal):
     layer = p.cache.data[li].cpu().numpy()
-    kc, ksf, vc, vsf = harness.read_tokens(layer, p.w.num_kv_heads, p.page_table[b].numpy(), n)
+    kc, ksf, vc, vsf = harness.read_tokens(layer, p.w.num_kv_heads, p.page_table[b].numpy(), n,
+                                           getattr(p, "k_format", 0))
     ref = harness.oracle_sequence(p, li, b, n, cal)
     for name, got in (("kc", kc), ("ksf", ksf), ("vc", vc), ("vsf", vsf)):
         want = ref[name]
+        if want is None:
+            assert got is None
+            continue
         if not np.array_equal(got, want):
             idx = np.argwhere(got != want)[0]
             raise AssertionError(f"{name} mismatch layer {li} seq {b} at {tuple(idx)}: "
@@ -91,6 +95,27 @@ def test_native_basis_keys(kvq, hadamard):
         for b, n in enumerate(lens):
             want = harness.oracle_attend(p, li, b, q[li, b][None], n - 1, n, cal)
             harness.check_attention(out[li, b], want[0], f"native layer {li} seq {b} len {n}")
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen3_8b"])
+def test_mixed_cache_bf16_keys(kvq, name):
+    # "NVFP4 attention cache on W4A4 Qwen3-8B", results table row "NVFP4 V
+    # only": bf16 keys (bit-exact: copied, or rounded from fp32), NVFP4 values
+    if name == "tiny":
+        w, lens, layers = synth.WORKLOADS["tiny"], [256], [0]
+    else:
+        w, lens, layers = small(num_layers=2, batch=3, calib_windows=1, calib_len=64), [7, 160, 333], [0, 1]
+    p = harness.build_problem(kvq, w, lens=lens, layers=layers, k_format=1)
+    cal = harness.oracle_calibration(p)
+    for li in range(len(layers)):
+        for b, n in enumerate(lens):
+            assert_codes_equal(p, li, b, n, cal)
+    for dt, tag in ((torch.float32, "f32"), (torch.bfloat16, "bf16")):
+        q, out = decode_all(kvq, p, out_dtype=dt)
+        for li in range(len(layers)):
+            for b, n in enumerate(lens):
+                want = harness.oracle_attend(p, li, b, q[li, b][None], n - 1, n, cal)
+                harness.check_attention(out[li, b], want[0], f"bf16-key layer {li} seq {b} len {n} {tag}")
 
 
 def test_many_units_single_split(kvq):

@@ -70,3 +70,17 @@ def test_exhaustive_rounding_against_brute_force(tmp_path):
     out = subprocess.run([str(exe), oracle.build()], capture_output=True, text=True, timeout=600)
     assert out.returncode == 0, out.stdout + out.stderr
     assert "e2m1_mismatch 0" in out.stdout and "e4m3_mismatch 0" in out.stdout
+
+
+def test_round_bf16_matches_torch_cast():
+    # the oracle's bf16 rounding (keys of the mixed cache) against torch's
+    # round-to-nearest-even cast, on random values and on exact ties
+    import torch
+    rng = np.random.default_rng(11)
+    x = np.concatenate([rng.standard_normal(100000).astype(np.float32) * 10.0 ** rng.integers(-30, 30, 100000),
+                        np.array([0.0, -0.0, 1.0, 1.00390625, 1.01171875, -1.00390625, 3.0e38, 1e-40], np.float32)])
+    # exact ties: the lower 16 bits are 0x8000, with an even and an odd kept part
+    ties = (np.arange(1000, dtype=np.uint32) << 16 | 0x3F800000 | 0x8000).view(np.float32)
+    x = np.concatenate([x, ties])
+    want = torch.from_numpy(x).to(torch.bfloat16).float().numpy()
+    np.testing.assert_array_equal(oracle.round_bf16(x).view(np.uint32), want.view(np.uint32))
