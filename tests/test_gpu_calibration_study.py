@@ -3,8 +3,8 @@
 "NVFP4 attention cache on W4A4 Qwen3-8B" (rstation.ai), results table rows
 "NVFP4 K only, native basis", "K: static per-channel smoothing, sqrt(absmax)
 from 4 C4 windows, position 0 excluded", "K: same smoothing, but sink token
-included in the absmax", "K: Hadamard-128 on head_dim" and "K: Hadamard-128 +
-smoothing", with observation 2 (calibrate without the sink).  The pages score
+included in the absmax", "K: Hadamard-128 on head_dim", "K: Hadamard-128 +
+smoothing" and "NVFP4 V only" (bf16 keys), with observation 2 (calibrate without the sink).  The pages score
 these rows by perplexity of a trained model; with synthetic inputs the score
 here is the attention output error of one decode step: relative L2 norm of
 (NVFP4-cache attention - exact fp64 attention on the unquantised bf16 cache)
@@ -58,12 +58,14 @@ def _reference(w, kv, q):
 
 def _run(kvq, w, kv, q, mode):
     """Calibrate (mode: 'excl' sink left out, 'incl' sink in, 'native' no
-    smoothing), append every sequence, decode one step; [nl][B][Hq][D] fp32."""
-    shape = kvq.Shape(len(LAYERS), w.num_q_heads, w.num_kv_heads, use_hadamard=w.hadamard)
+    smoothing, 'bf16k' bf16 keys with packed values), append every sequence,
+    decode one step; [nl][B][Hq][D] fp32."""
+    shape = kvq.Shape(len(LAYERS), w.num_q_heads, w.num_kv_heads, use_hadamard=w.hadamard,
+                      k_format=kvq.K_BF16 if mode == "bf16k" else kvq.K_NVFP4)
     win = [synth.calibration_windows(w, l, "cuda") for l in LAYERS]
     kc = torch.stack([x[0] for x in win]).contiguous()
     vc = torch.stack([x[1] for x in win]).contiguous()
-    if mode == "native":
+    if mode in ("native", "bf16k"):
         calib = kvq.calibrate_native(shape, kc, vc)
     else:
         calib = kvq.calibrate_smoothing(shape, kc, vc, exclude_pos0=(mode == "excl"))
@@ -100,7 +102,8 @@ def test_calibration_ablations(kvq, capsys):
             ("smoothing, sink included, 4 windows", base, "incl"),
             ("native basis (no smoothing)", base, "native"),
             ("Hadamard-128 + smoothing", _workload(hadamard=True), "excl"),
-            ("Hadamard-128 alone", _workload(hadamard=True), "native")):
+            ("Hadamard-128 alone", _workload(hadamard=True), "native"),
+            ("bf16 keys, NVFP4 values", base, "bf16k")):
         rows.append((name,) + _errors(_run(kvq, w, kv, q, mode), ref))
     with capsys.disabled():
         print("\nkey calibration ablation (qwen3_8b shapes, 4 layers x 4 sequences x 2304 tokens)")
@@ -117,3 +120,5 @@ def test_calibration_ablations(kvq, capsys):
     # rows "NVFP4 K only, native basis" and "K: Hadamard-128 on head_dim": the
     # rotation alone is worse than the native basis
     assert err["Hadamard-128 alone"] > 1.1 * native
+    # row "NVFP4 V only": the keys carry the gap; packed values alone cost far less
+    assert err["bf16 keys, NVFP4 values"] < 0.5 * smooth
