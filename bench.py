@@ -293,9 +293,10 @@ class Prefill:
     512-token chunk.  One step = append the chunk's K/V into every layer, then
     prefill attention of every layer (tcgen05)."""
 
-    def __init__(self, kvq, synth, layers=36):
+    def __init__(self, kvq, synth, layers=36, k_format=0):
         import dataclasses
         w = dataclasses.replace(synth.WORKLOADS["prefill"], num_layers=layers)
+        self.k_format = k_format
         self.kvq, self.w = kvq, w
         L, B, P0, Tq = w.num_layers, w.batch, w.context, w.prefill_chunk
         self.L, self.B, self.P0, self.Tq = L, B, P0, Tq
@@ -303,7 +304,7 @@ class Prefill:
         total = P0 + Tq
         lens = torch.full((B,), total, dtype=torch.int32)
         self.page_table, self.num_pages = synth.build_page_table(w, lens)
-        self.shape = kvq.Shape(L, w.num_q_heads, w.num_kv_heads)
+        self.shape = kvq.Shape(L, w.num_q_heads, w.num_kv_heads, k_format=k_format)
         kc = torch.stack([synth.calibration_windows(w, l, dev)[0] for l in range(L)])
         vc = torch.stack([synth.calibration_windows(w, l, dev)[1] for l in range(L)])
         self.calib = kvq.calibrate_smoothing(self.shape, kc, vc, exclude_pos0=True)
@@ -582,7 +583,7 @@ def other_workload(args, kvq, synth, rank, world):
     warm = max(3, args.warmup)
     clock = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if args.workload == "prefill":
-        wl = Prefill(kvq, synth, args.layers)
+        wl = Prefill(kvq, synth, args.layers, k_format=1 if args.k_format == "bf16" else 0)
         total, app_ms, pre_ms = time_two_kernels(wl.append, wl.attend, warm, args.steps, world)
         clocks = clock.stop() if clock else None
         total = max_over_ranks(total, world)
@@ -594,7 +595,8 @@ def other_workload(args, kvq, synth, rank, world):
                 "warmup": warm, "ms_per_step": total / args.steps, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f16 mma (q split hi+lo), f32 accumulate", "data": "synthetic",
                 "config": {"workload": f"chunked prefill: {wl.L} layers, batch 8, 8192 cached + 512-token causal "
-                                       "chunk, 32 q / 8 kv heads, head_dim 128", "layers": wl.L},
+                                       "chunk, 32 q / 8 kv heads, head_dim 128", "layers": wl.L,
+                           "kv_cache": "mixed: bf16 keys, nvfp4 values" if wl.k_format else "nvfp4"},
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
                              "frac": achieved / peak_tf, "frac_of_sustained": achieved / peak_tf_sus,
                              "traffic": None, "peak_source": tf_kind,

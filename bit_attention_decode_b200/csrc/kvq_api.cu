@@ -163,8 +163,6 @@ kvq_status kvq_prefill_attention(const kvq_shape* shape, const kvq_calib* calib,
                                  const int32_t* seq_lens, int32_t batch, void* out, int32_t out_dtype,
                                  void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
     KVQ_TRY(check_shape(shape));
-    // the tensor-core prefill dequantises NVFP4 keys only
-    if (shape->k_format != KVQ_K_NVFP4) return KVQ_EUNSUPPORTED;
     KVQ_TRY(check_calib(calib));
     KVQ_TRY(check_cache(shape, cache));
     KVQ_TRY(check_layers(shape, layer0, nlayers));

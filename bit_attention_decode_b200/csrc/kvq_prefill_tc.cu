@@ -52,6 +52,7 @@ constexpr int kQBytes = kRows * kD * 2;           // 32 KB per fp16 query tile p
 constexpr int kKBytes = kBlkTok * kD * 2;         // 16 KB per fp16 key tile
 constexpr int kVBytes = kBlkTok * kD * 2;         // 16 KB per fp16 value tile
 constexpr int kStageBytes = 4 * kTile;            // 4 packed page tiles of one head
+constexpr int kVPart = kTileBf16K - kBf16VCodes;  // 1152: values of a bf16-key tile (staged alone)
 constexpr int kOffQ = 0;                          // [tile][hi, lo]
 constexpr int kOffK = kOffQ + kTiles * 2 * kQBytes;   // 2 buffers
 constexpr int kOffV = kOffK + 2 * kKBytes;        // 2 buffers
@@ -177,6 +178,17 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ uint32_t sw128(int row, int ch) {
     return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((ch ^ (row & 7)) << 4));
 }
+// 16-byte asynchronous copy global -> shared (bf16 key rows of the mixed
+// cache go straight into the swizzled key tile)
+__device__ __forceinline__ void cp_async16(uint8_t* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ uint32_t bf2(float lo, float hi) {
+    __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&r);
+}
 __device__ __forceinline__ void sts128(uint8_t* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     *reinterpret_cast<uint4*>(p) = make_uint4(a, b, c, d);
 }
@@ -222,7 +234,10 @@ struct PrefillBars {
 
 // ------------------------------------------------------------------ kernel
 // grid (query-tile pairs, batch * Hkv, nlayers), block 384.
-template <typename TQ, typename TO>
+// KB: mixed cache (bf16 keys, untransformed; only the value parts of the
+// tiles are staged, the key rows are copied into the key tile directly, and
+// Q.K runs on bf16 operands).
+template <typename TQ, typename TO, bool KB>
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -309,11 +324,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                     const TQ* src = reinterpret_cast<const TQ*>(a.q) +
                                     ((((size_t)li * a.batch + b) * a.q_len + qi) * a.Hq + h * a.G + head) * kD;
                     load_row128<TQ>(src, x);
-                    const float* srow = a.smooth + ((size_t)li * a.Hkv + h) * kD;
+                    float scale;
+                    if constexpr (KB) {
+                        scale = kLog2e * kInvSqrt128;     // bf16 keys: the query as given
+                    } else {
+                        const float* srow = a.smooth + ((size_t)li * a.Hkv + h) * kD;
 #pragma unroll
-                    for (int i = 0; i < kD; ++i) x[i] *= __ldg(srow + i);
-                    float scale = __ldg(a.gk + li) * kLog2e * kInvSqrt128;
-                    if (a.hadamard) {
+                        for (int i = 0; i < kD; ++i) x[i] *= __ldg(srow + i);
+                        scale = __ldg(a.gk + li) * kLog2e * kInvSqrt128;
+                    }
+                    if (!KB && a.hadamard) {
 #pragma unroll
                         for (int hh = 1; hh < kD; hh <<= 1)
 #pragma unroll
@@ -350,9 +370,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float u = x[8 * ch + 2 * e] * sig, v = x[8 * ch + 2 * e + 1] * sig;
-                        hi[e] = h2(u, v);
-                        const float2 f = __half22float2(*reinterpret_cast<__half2*>(&hi[e]));
-                        lo[e] = h2(u - f.x, v - f.y);
+                        if constexpr (KB) {
+                            hi[e] = bf2(u, v);
+                            const float2 f = make_float2(__uint_as_float(hi[e] << 16),
+                                                         __uint_as_float(hi[e] & 0xFFFF0000u));
+                            lo[e] = bf2(u - f.x, v - f.y);
+                        } else {
+                            hi[e] = h2(u, v);
+                            const float2 f = __half22float2(*reinterpret_cast<__half2*>(&hi[e]));
+                            lo[e] = h2(u - f.x, v - f.y);
+                        }
                     }
                     const uint32_t off = (ch >> 3) * (kRows * 128) + sw128(r, ch & 7);
                     sts128(qhi + off, hi[0], hi[1], hi[2], hi[3]);
@@ -470,12 +497,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
 #pragma unroll
                 for (int k = 0; k < 4; ++k) pg[k] = pgn[k];
                 fetch_ids(j + 1);
-                mbar_arrive_expect_tx(&bars.stage_full[st], (uint32_t)n_p * kTile);
+                constexpr int part = KB ? kVPart : kTile;          // bytes staged per page
+                constexpr int part0 = KB ? kBf16VCodes : 0;       // offset of that part in the tile
+                constexpr int tile = KB ? kTileBf16K : kTile;
+                mbar_arrive_expect_tx(&bars.stage_full[st], (uint32_t)n_p * part);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     if (k < n_p)
-                        bulk_g2s(smem + kOffStage + st * kStageBytes + k * kTile,
-                                 layer_base + ((size_t)pg[k] * a.Hkv + h) * kTile, kTile, &bars.stage_full[st]);
+                        bulk_g2s(smem + kOffStage + st * kStageBytes + k * part,
+                                 layer_base + ((size_t)pg[k] * a.Hkv + h) * tile + part0, part, &bars.stage_full[st]);
             };
             if (issuer) fetch_ids(0);
             // every stage is filled up front; a stage is refilled (block j +
@@ -502,15 +532,24 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                     S.ks[e] = 0;
                     S.vs[e][0] = S.vs[e][1] = S.vs[e][2] = S.vs[e][3] = 0;
                     if (it < kItems && j * kBlkTok + tkn < kv_end) {
-                        const uint8_t* T = smem + kOffStage + st * kStageBytes + (tkn >> 4) * kTile;
                         const int trow = tkn & 15;
-                        S.kc[e][0] = *reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32);
-                        S.kc[e][1] = *reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32 + 16);
-                        S.ks[e] = *reinterpret_cast<const uint32_t*>(T + kKScales + trow * 8 + half * 4);
-                        S.vc[e][0] = *reinterpret_cast<const uint4*>(T + kVCodes + trow * 64 + half * 32);
-                        S.vc[e][1] = *reinterpret_cast<const uint4*>(T + kVCodes + trow * 64 + half * 32 + 16);
+                        if constexpr (KB) {
+                            // the stage holds the value parts only
+                            const uint8_t* T = smem + kOffStage + st * kStageBytes + (tkn >> 4) * kVPart;
+                            S.vc[e][0] = *reinterpret_cast<const uint4*>(T + trow * 64 + half * 32);
+                            S.vc[e][1] = *reinterpret_cast<const uint4*>(T + trow * 64 + half * 32 + 16);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) S.vs[e][q] = T[kVScales + (half * 4 + q) * 16 + trow];
+                            for (int q = 0; q < 4; ++q) S.vs[e][q] = T[1024 + (half * 4 + q) * 16 + trow];
+                        } else {
+                            const uint8_t* T = smem + kOffStage + st * kStageBytes + (tkn >> 4) * kTile;
+                            S.kc[e][0] = *reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32);
+                            S.kc[e][1] = *reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32 + 16);
+                            S.ks[e] = *reinterpret_cast<const uint32_t*>(T + kKScales + trow * 8 + half * 4);
+                            S.vc[e][0] = *reinterpret_cast<const uint4*>(T + kVCodes + trow * 64 + half * 32);
+                            S.vc[e][1] = *reinterpret_cast<const uint4*>(T + kVCodes + trow * 64 + half * 32 + 16);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) S.vs[e][q] = T[kVScales + (half * 4 + q) * 16 + trow];
+                        }
                     }
                 }
                 __syncwarp();
@@ -563,6 +602,39 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                 if ((dt & 31) == 0) mbar_arrive(&bars.k_full[buf]);
                 return true;
             };
+            // bf16 keys of block j: once K buffer j & 1 is free, 16-byte async
+            // copies of each row straight into its swizzled place (zeros past
+            // the sequence); finish_k waits for them and hands the tile over
+            auto issue_k = [&](int j) -> bool {
+                const int buf = j & 1;
+                if (j >= 2 && !mbar_wait_warp(&bars.s_full[kTiles - 1][buf], ((j - 2) >> 1) & 1)) return false;
+                uint8_t* Kt = smem + kOffK + buf * kKBytes;
+#pragma unroll
+                for (int e = 0; e < kPer; ++e) {
+                    const int it = dt + e * kDqThreads;
+                    if (it >= kItems) break;
+                    const int tkn = it >> 1, half = it & 1;
+                    uint8_t* dst = Kt + half * (kBlkTok * 128);
+                    if (j * kBlkTok + tkn < kv_end) {
+                        const int pg = __ldg(pt + j * 4 + (tkn >> 4));
+                        const uint8_t* src = layer_base + ((size_t)pg * a.Hkv + h) * kTileBf16K + (tkn & 15) * 256 +
+                                             half * 128;
+#pragma unroll
+                        for (int ch = 0; ch < 8; ++ch) cp_async16(dst + sw128(tkn, ch), src + ch * 16);
+                    } else {
+#pragma unroll
+                        for (int ch = 0; ch < 8; ++ch) sts128(dst + sw128(tkn, ch), 0u, 0u, 0u, 0u);
+                    }
+                }
+                cp_async_commit();
+                return true;
+            };
+            auto finish_k = [&](int j) {
+                cp_async_wait_all();
+                fence_async_smem();
+                __syncwarp();
+                if ((dt & 31) == 0) mbar_arrive(&bars.k_full[j & 1]);
+            };
             // values of block j into V buffer j & 1, free once both tiles'
             // P.V(j - 2) are done
             auto store_v = [&](int j, const Staged& S) -> bool {
@@ -602,11 +674,28 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
             // the values of block j, because the MMA warp needs them first
             // (Q.K(j + 1) is issued before P.V(j)).
             Staged cur, nxt;
-            bool dq_ok = nb == 0 || (load_block(0, cur) && store_k(0, cur));
-            for (int j = 0; dq_ok && j < nb; ++j) {
-                if (j + 1 < nb) dq_ok = load_block(j + 1, nxt) && store_k(j + 1, nxt);
-                dq_ok = dq_ok && store_v(j, cur);
-                cur = nxt;
+            bool dq_ok = true;
+            if constexpr (KB) {
+                // the copies of block j + 1's keys overlap the values of block j
+                if (nb > 0) {
+                    dq_ok = load_block(0, cur) && issue_k(0);
+                    if (dq_ok) finish_k(0);
+                }
+                for (int j = 0; dq_ok && j < nb; ++j) {
+                    const bool more = j + 1 < nb;
+                    if (more) dq_ok = load_block(j + 1, nxt) && issue_k(j + 1);
+                    dq_ok = dq_ok && store_v(j, cur);
+                    if (more && dq_ok) finish_k(j + 1);
+                    cur = nxt;
+                }
+                cp_async_wait_all();   // nothing in flight past this point
+            } else {
+                dq_ok = nb == 0 || (load_block(0, cur) && store_k(0, cur));
+                for (int j = 0; dq_ok && j < nb; ++j) {
+                    if (j + 1 < nb) dq_ok = load_block(j + 1, nxt) && store_k(j + 1, nxt);
+                    dq_ok = dq_ok && store_v(j, cur);
+                    cur = nxt;
+                }
             }
             if (!dq_ok) atomicOr(&bars.flags, 1);
             if (issuer) bars.issued = issued;
@@ -615,7 +704,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
             // Descriptors are built once; a k-step only advances the 14-bit
             // start-address field (16-byte units) by a constant, which never
             // carries out of the field for shared-memory addresses.
-            const uint32_t qk = f16_idesc(kRows, kBlkTok, false);
+            // bf16 keys: both Q.K operands bf16 (A and B formats 1)
+            const uint32_t qk = f16_idesc(kRows, kBlkTok, false) | (KB ? ((1u << 7) | (1u << 10)) : 0u);
             const uint32_t pv = f16_idesc(kRows, kD, true);
             uint64_t qd[kTiles][2], kd[2], vd[2];
 #pragma unroll
@@ -753,12 +843,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
 }  // namespace
 
 // ------------------------------------------------------------------ launcher
+template <bool KB>
 static cudaError_t launch_prefill(const AttnArgs& a, dim3 grid, bool qb, bool ob, cudaStream_t st) {
     cudaError_t e;
 #define KVQ_LAUNCH(TQ, TO)                                                                                     \
-    e = cudaFuncSetAttribute(prefill_tc_kernel<TQ, TO>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc); \
+    e = cudaFuncSetAttribute(prefill_tc_kernel<TQ, TO, KB>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc); \
     if (e != cudaSuccess) return e;                                                                            \
-    prefill_tc_kernel<TQ, TO><<<grid, kThreads, kSmemAlloc, st>>>(a);
+    prefill_tc_kernel<TQ, TO, KB><<<grid, kThreads, kSmemAlloc, st>>>(a);
     if (qb && ob) { KVQ_LAUNCH(__nv_bfloat16, __nv_bfloat16) }
     else if (qb) { KVQ_LAUNCH(__nv_bfloat16, float) }
     else if (ob) { KVQ_LAUNCH(float, __nv_bfloat16) }
@@ -769,7 +860,8 @@ static cudaError_t launch_prefill(const AttnArgs& a, dim3 grid, bool qb, bool ob
 
 cudaError_t launch_prefill_tc(const AttnArgs& a, int nlayers, bool q_bf16, bool out_bf16, cudaStream_t st) {
     dim3 grid((a.q_len + kTiles * kQTok - 1) / (kTiles * kQTok), a.batch * a.Hkv, nlayers);
-    return launch_prefill(a, grid, q_bf16, out_bf16, st);
+    if (a.kbf16) return launch_prefill<true>(a, grid, q_bf16, out_bf16, st);
+    return launch_prefill<false>(a, grid, q_bf16, out_bf16, st);
 }
 
 }  // namespace kvq

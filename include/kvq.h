@@ -247,7 +247,8 @@ size_t kvq_prefill_workspace_bytes(const kvq_shape* shape, int32_t nlayers, int3
  *
  *   q      [nlayers][batch][q_len][Hq][128], q_dtype.
  *   q_start [batch] int32.   out [nlayers][batch][q_len][Hq][128].
- * A KVQ_K_BF16 cache is not supported here (KVQ_EUNSUPPORTED).
+ * With a KVQ_K_BF16 cache the query is used as given (as in decode) and Q.K
+ * runs on bf16 operands.
  */
 kvq_status kvq_prefill_attention(const kvq_shape* shape, const kvq_calib* calib, const kvq_cache* cache,
                                  int32_t layer0, int32_t nlayers, const void* q, int32_t q_dtype,

@@ -126,8 +126,8 @@ def test_mixed_cache_key_format_validation(kvq_lib):
     assert _call_decode(kvq, kvq.Shape(2, 32, 8, use_hadamard=True, k_format=kvq.K_BF16)) == kvq.KVQ_EINVAL
     # a layer stride sized for packed keys is too small for bf16 keys
     assert _call_decode(kvq, bf, cache=kvq._Cache(4096, 8 * 2304 * 4, 4)) == kvq.KVQ_EINVAL
-    # the tensor-core prefill dequantises packed keys only
+    # the prefill checks the cache against the bf16-key tile size too
     st = kvq._lib.kvq_prefill_attention(
-        ctypes.byref(bf.c()), ctypes.byref(kvq._Calib(16, 16, 16, 16)), ctypes.byref(kvq._Cache(4096, 8 * 5248 * 4, 4)),
+        ctypes.byref(bf.c()), ctypes.byref(kvq._Calib(16, 16, 16, 16)), ctypes.byref(kvq._Cache(4096, 8 * 2304 * 4, 4)),
         0, 1, 256, 1, 8, 512, 768, 64, 1024, 2, 2048, 1, None, 0, None, None)
-    assert st == kvq.KVQ_EUNSUPPORTED
+    assert st == kvq.KVQ_EINVAL

@@ -153,12 +153,14 @@ def test_page_order_does_not_change_results(kvq):
     np.testing.assert_array_equal(oa, ob)
 
 
-def test_prefill_chunk(kvq):
+@pytest.mark.parametrize("k_format", [0, 1])
+def test_prefill_chunk(kvq, k_format):
+    # k_format 1: the mixed cache (bf16 keys copied into the key tile, bf16 Q.K)
     w = small(num_layers=2, batch=2, calib_windows=1, calib_len=64, prefill_chunk=48)
     P0 = [100, 33]
     Tq = 48
     lens = [n + Tq for n in P0]
-    p = harness.build_problem(kvq, w, lens=lens)
+    p = harness.build_problem(kvq, w, lens=lens, k_format=k_format)
     cal = harness.oracle_calibration(p)
     q = torch.stack([synth.prefill_queries(w, l) for l in p.layers])        # [nl][B][Tq][Hq][D]
     q_start = torch.tensor(P0, dtype=torch.int32)
@@ -168,7 +170,7 @@ def test_prefill_chunk(kvq):
         for li in range(2):
             for b in range(2):
                 want = harness.oracle_attend(p, li, b, q[li, b].float().numpy(), P0[b], lens[b], cal)
-                harness.check_attention(out[li, b], want, f"prefill layer {li} seq {b} {tag}")
+                harness.check_attention(out[li, b], want, f"prefill k_format {k_format} layer {li} seq {b} {tag}")
 
 
 def test_zero_length_gives_zero_rows(kvq):
