@@ -70,11 +70,12 @@ def _load():
         lib.oracle_e4m3_encode_n.argtypes = [P, P, i64]
         lib.oracle_transform_keys.argtypes = [P, P, i64, i32, i32, P]
         lib.oracle_calibrate.argtypes = [P, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, P]
+        lib.oracle_klt_apply.argtypes = [P, P, ctypes.c_int64, P]
         lib.oracle_quantize_rows.argtypes = [P, i64, f32, P, P]
         lib.oracle_dequantize_rows.argtypes = [P, P, i64, f32, P]
         lib.oracle_attention.argtypes = [P, i32, i32, i32, i32, P, i32, P, P, i32, P]
         for name in ("oracle_e2m1_encode_n", "oracle_e4m3_encode_n", "oracle_transform_keys",
-                     "oracle_calibrate", "oracle_quantize_rows", "oracle_dequantize_rows",
+                     "oracle_calibrate", "oracle_klt_apply", "oracle_quantize_rows", "oracle_dequantize_rows",
                      "oracle_attention"):
             getattr(lib, name).restype = None
         _lib = lib
@@ -198,6 +199,74 @@ def round_bf16(x) -> np.ndarray:
     b = np.ascontiguousarray(x, np.float32).view(np.uint32).astype(np.uint64)
     r = (b + 0x7FFF + ((b >> 16) & 1)) & 0xFFFF0000
     return r.astype(np.uint32).view(np.float32)
+
+
+def klt_apply(y, U) -> np.ndarray:
+    """y [..., 128] fp32, U [128][128] fp32 -> U^T y per row, each output one
+    fp32 fused multiply-add chain over c = 0..127 (the library's order)."""
+    y, py = _c(_f32(y), np.float32)
+    U, pu = _c(_f32(U), np.float32)
+    n = y.size // HEAD_DIM
+    out = np.empty_like(y)
+    _load().oracle_klt_apply(py, pu, n, out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def klt_basis(y) -> np.ndarray:
+    """Static per-head KLT basis ("NVFP4 attention cache on W4A4 Qwen3-8B",
+    results table rows "K: static per-head KLT" and "K: static KLT +
+    smoothing"): the eigenvectors of the second-moment matrix
+    C = sum_t y_t y_t^T / N of the (smoothed) calibration keys y [N][128], in
+    fp64, ordered by decreasing eigenvalue, each signed so that its component
+    of largest magnitude is positive.  Returns (U [128][128] fp64 with
+    U[c][i] = component c of vector i, eigenvalues [128] fp64)."""
+    y = np.asarray(y, np.float64)
+    C = y.T @ y / y.shape[0]
+    w, U = np.linalg.eigh(C)
+    order = np.argsort(-w, kind="stable")
+    w, U = w[order], U[:, order]
+    big = np.argmax(np.abs(U), axis=0)
+    U = U * np.where(U[big, np.arange(U.shape[1])] < 0, -1.0, 1.0)
+    return U, w
+
+
+def calibrate_klt(k_calib, v_calib, exclude_pos0: bool = True):
+    """Smoothing (as calibrate) followed by a KLT basis per (layer, kv head)
+    from the smoothed calibration keys, position 0 of each window left out
+    when exclude_pos0 (as for the smoothing absmax).
+    Returns (s, inv_s, U [L][H][128][128] fp32, eigenvalues [L][H][128])."""
+    k = _f32(k_calib)
+    s, inv, _, _ = calibrate(k_calib, v_calib, exclude_pos0=exclude_pos0, hadamard=False)
+    L, W, T, H, D = k.shape
+    t0 = 1 if exclude_pos0 else 0
+    U = np.empty((L, H, D, D), np.float32)
+    ev = np.empty((L, H, D))
+    for l in range(L):
+        y = transform_keys(k[l, :, t0:].reshape(-1, H, D), inv[l], False)
+        for h in range(H):
+            u, w = klt_basis(y[:, h])
+            U[l, h], ev[l, h] = u.astype(np.float32), w
+    return s, inv, U, ev
+
+
+def klt_tensor_scales(k_calib, v_calib, inv_s, U):
+    """g_K, g_V [L] for keys transformed by smoothing then U (any U, e.g. the
+    library's): max |U^T (k * inv_s)| over every calibration token, position 0
+    included, / 2688 (1 if zero); g_V as calibrate."""
+    k = _f32(k_calib)
+    v = _f32(v_calib)
+    L, W, T, H, D = k.shape
+    gk = np.empty(L, np.float32)
+    gv = np.empty(L, np.float32)
+    for l in range(L):
+        y = transform_keys(k[l].reshape(-1, H, D), inv_s[l], False)
+        a = np.float32(0.0)
+        for h in range(H):
+            a = max(a, np.abs(klt_apply(y[:, h], U[l, h])).max())
+        b = np.abs(v[l]).max()
+        gk[l] = np.float32(a) / np.float32(2688.0) if a > 0 else np.float32(1.0)
+        gv[l] = np.float32(b) / np.float32(2688.0) if b > 0 else np.float32(1.0)
+    return gk, gv
 
 
 # ---------------------------------------------------------------- composites

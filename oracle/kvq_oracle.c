@@ -152,6 +152,28 @@ void oracle_transform_keys(const float* k, const float* inv_s, int64_t n, int H,
                           y + ((size_t)t * H + h) * HD);
 }
 
+/* Static per-head KLT ([P1] results table, rows "K: static per-head KLT" and
+ * "K: static KLT + smoothing"): y' = U^T y for a 128 x 128 orthogonal U per
+ * (layer, kv head), U[c][i] = component c of basis vector i.  Each output is
+ * one fp32 fused multiply-add chain over c = 0, 1, ..., 127 starting from 0:
+ * the library applies the transform in exactly this order, so the codes
+ * that follow are reproducible bit for bit.
+ *
+ * y, out: [n][128] fp32; U: [128][128] fp32. */
+void oracle_klt_apply(const float* y, const float* U, int64_t n, float* out)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n; ++r) {
+        const float* yr = y + (size_t)r * HD;
+        float* o = out + (size_t)r * HD;
+        for (int i = 0; i < HD; ++i) {
+            float acc = 0.0f;
+            for (int c = 0; c < HD; ++c) acc = fmaf(U[(size_t)c * HD + i], yr[c], acc);
+            o[i] = acc;
+        }
+    }
+}
+
 /* ------------------------------------------------------------------------- */
 /* Calibration ([P1] results table row 4 and observation 2): the smoothing
  * factor of each (layer, kv head, channel) is sqrt of the absolute maximum of
