@@ -37,12 +37,13 @@ K_NVFP4, K_BF16 = 0, 1          # kvq_shape.k_format: packed keys, or bf16 keys 
 class _Shape(ctypes.Structure):
     _fields_ = [("num_layers", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("page_size", ctypes.c_int32), ("use_hadamard", ctypes.c_int32), ("k_format", ctypes.c_int32)]
+                ("page_size", ctypes.c_int32), ("use_hadamard", ctypes.c_int32), ("k_format", ctypes.c_int32),
+                ("use_klt", ctypes.c_int32)]
 
 
 class _Calib(ctypes.Structure):
     _fields_ = [("k_smooth", ctypes.c_void_p), ("k_inv_smooth", ctypes.c_void_p),
-                ("k_gscale", ctypes.c_void_p), ("v_gscale", ctypes.c_void_p)]
+                ("k_gscale", ctypes.c_void_p), ("v_gscale", ctypes.c_void_p), ("k_klt", ctypes.c_void_p)]
 
 
 class _Cache(ctypes.Structure):
@@ -62,6 +63,8 @@ _lib.kvq_version.restype = ctypes.c_char_p
 _lib.kvq_version.argtypes = []
 _lib.kvq_calibrate_smoothing.restype = _I32
 _lib.kvq_calibrate_smoothing.argtypes = [_SHP, _P, _P, _I32, _I32, _I32, _I32, _CAL, _P]
+_lib.kvq_calibrate_klt.restype = _I32
+_lib.kvq_calibrate_klt.argtypes = [_SHP, _P, _P, _I32, _I32, _I32, _I32, _CAL, _P]
 _lib.kvq_calibrate_native.restype = _I32
 _lib.kvq_calibrate_native.argtypes = [_SHP, _P, _P, _I32, _I32, _I32, _CAL, _P]
 _lib.kvq_quantize_append.restype = _I32
@@ -87,6 +90,7 @@ _lib.kvq_round_e4m3.restype = _I32
 _lib.kvq_round_e4m3.argtypes = [_P, _P, ctypes.c_int64, _P]
 
 EXPORTED = ("kvq_page_bytes", "kvq_status_string", "kvq_version", "kvq_calibrate_smoothing", "kvq_calibrate_native",
+            "kvq_calibrate_klt",
             "kvq_quantize_append", "kvq_decode_workspace_bytes", "kvq_decode_attention",
             "kvq_prefill_workspace_bytes", "kvq_prefill_attention", "kvq_decode_attention_noalloc",
             "kvq_round_e2m1", "kvq_round_e4m3", "kvq_selftest_wait_timeout")
@@ -122,10 +126,11 @@ class Shape:
     head_dim: int = HEAD_DIM
     page_size: int = PAGE_SIZE
     k_format: int = K_NVFP4
+    use_klt: bool = False
 
     def c(self) -> _Shape:
         return _Shape(self.num_layers, self.num_q_heads, self.num_kv_heads, self.head_dim,
-                      self.page_size, int(self.use_hadamard), int(self.k_format))
+                      self.page_size, int(self.use_hadamard), int(self.k_format), int(self.use_klt))
 
 
 @dataclasses.dataclass
@@ -135,10 +140,11 @@ class Calibration:
     k_inv_smooth: torch.Tensor   # [L][Hkv][128]
     k_gscale: torch.Tensor       # [L]
     v_gscale: torch.Tensor       # [L]
+    k_klt: Optional[torch.Tensor] = None   # [L][Hkv][128][128] KLT bases (use_klt shapes)
 
     def c(self) -> _Calib:
         return _Calib(self.k_smooth.data_ptr(), self.k_inv_smooth.data_ptr(),
-                      self.k_gscale.data_ptr(), self.v_gscale.data_ptr())
+                      self.k_gscale.data_ptr(), self.v_gscale.data_ptr(), _ptr(self.k_klt))
 
 
 @dataclasses.dataclass
@@ -183,8 +189,9 @@ def page_bytes(shape: Shape) -> int:
 def new_calibration(shape: Shape, device="cuda") -> Calibration:
     L, H = shape.num_layers, shape.num_kv_heads
     f = dict(dtype=torch.float32, device=device)
+    klt = torch.empty(L, H, HEAD_DIM, HEAD_DIM, **f) if shape.use_klt else None
     return Calibration(torch.empty(L, H, HEAD_DIM, **f), torch.empty(L, H, HEAD_DIM, **f),
-                       torch.empty(L, **f), torch.empty(L, **f))
+                       torch.empty(L, **f), torch.empty(L, **f), klt)
 
 
 def new_cache(shape: Shape, num_pages: int, device="cuda") -> PagedCache:
@@ -217,6 +224,21 @@ def calibrate_native(shape: Shape, k_calib: torch.Tensor, v_calib: torch.Tensor,
     _check(_lib.kvq_calibrate_native(ctypes.byref(shape.c()), k_calib.data_ptr(), v_calib.data_ptr(),
                                      _dtype_code(k_calib), W, T, ctypes.byref(c), _stream()),
            "kvq_calibrate_native")
+    return out
+
+
+def calibrate_klt(shape: Shape, k_calib: torch.Tensor, v_calib: torch.Tensor, exclude_pos0: bool = True,
+                  out: Optional[Calibration] = None) -> Calibration:
+    """Smoothing then a static per-head KLT (shape.use_klt);
+    k/v_calib [L][W][T][Hkv][128]."""
+    _need_cuda(k_calib, v_calib)
+    L, W, T, H, D = k_calib.shape
+    if out is None:
+        out = new_calibration(shape, k_calib.device)
+    c = out.c()
+    _check(_lib.kvq_calibrate_klt(ctypes.byref(shape.c()), k_calib.data_ptr(), v_calib.data_ptr(),
+                                  _dtype_code(k_calib), W, T, int(bool(exclude_pos0)), ctypes.byref(c), _stream()),
+           "kvq_calibrate_klt")
     return out
 
 

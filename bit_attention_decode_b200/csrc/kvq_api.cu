@@ -11,6 +11,12 @@ namespace {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+#define KVQ_TRY_LOCAL(x)                 \
+    do {                                 \
+        kvq_status _st = (x);            \
+        if (_st != KVQ_OK) return _st;   \
+    } while (0)
+
 kvq_status check_shape(const kvq_shape* s) {
     if (!s) return KVQ_EINVAL;
     if (s->head_dim != kvq::kD || s->page_size != kvq::kPage) return KVQ_EUNSUPPORTED;
@@ -24,6 +30,9 @@ kvq_status check_shape(const kvq_shape* s) {
     if (s->k_format != KVQ_K_NVFP4 && s->k_format != KVQ_K_BF16) return KVQ_EINVAL;
     // bf16 keys are stored untransformed
     if (s->k_format == KVQ_K_BF16 && s->use_hadamard) return KVQ_EINVAL;
+    // the KLT replaces the rotation and rotates packed keys only
+    if (s->use_klt != 0 && s->use_klt != 1) return KVQ_EINVAL;
+    if (s->use_klt && (s->use_hadamard || s->k_format != KVQ_K_NVFP4)) return KVQ_EINVAL;
     return KVQ_OK;
 }
 
@@ -39,6 +48,13 @@ bool good_dtype(int32_t d) { return d == KVQ_F32 || d == KVQ_BF16; }
 
 kvq_status check_calib(const kvq_calib* c) {
     if (!c || !c->k_smooth || !c->k_inv_smooth || !c->k_gscale || !c->v_gscale) return KVQ_EINVAL;
+    return KVQ_OK;
+}
+
+// a KLT shape also needs the bases
+kvq_status check_calib(const kvq_shape* s, const kvq_calib* c) {
+    KVQ_TRY_LOCAL(check_calib(c));
+    if (s->use_klt && (!c->k_klt || !aligned(c->k_klt, 16))) return KVQ_EINVAL;
     return KVQ_OK;
 }
 
@@ -109,12 +125,29 @@ kvq_status kvq_calibrate_native(const kvq_shape* shape, const void* k_calib, con
                                  (cudaStream_t)stream);
 }
 
+kvq_status kvq_calibrate_klt(const kvq_shape* shape, const void* k_calib, const void* v_calib, int32_t dtype,
+                             int32_t num_windows, int32_t window_len, int32_t exclude_pos0, const kvq_calib* out,
+                             void* stream) {
+    KVQ_TRY(check_shape(shape));
+    if (!shape->use_klt) return KVQ_EINVAL;
+    KVQ_TRY(check_calib(shape, out));
+    if (!k_calib || !v_calib || !good_dtype(dtype) || num_windows < 1 || window_len < 1) return KVQ_EINVAL;
+    if (exclude_pos0 != 0 && exclude_pos0 != 1) return KVQ_EINVAL;
+    if (window_len <= exclude_pos0) return KVQ_EINVAL;
+    if (!aligned(k_calib, 16) || !aligned(v_calib, 16)) return KVQ_EINVAL;
+    if (num_windows > 65535 || (long)num_windows * window_len * shape->num_kv_heads > (1L << 28)) return KVQ_EINVAL;
+    KVQ_TRY(check_device());
+    return kvq::calibrate_klt(*shape, k_calib, v_calib, dtype, num_windows, window_len, exclude_pos0, *out,
+                              (cudaStream_t)stream);
+}
+
 kvq_status kvq_quantize_append(const kvq_shape* shape, const kvq_calib* calib, const kvq_cache* cache,
                                int32_t layer0, int32_t nlayers, const void* k, const void* v, int32_t dtype,
                                const int64_t* slot_mapping, int32_t num_tokens, int32_t* dev_status,
                                void* stream) {
     KVQ_TRY(check_shape(shape));
-    KVQ_TRY(check_calib(calib));
+    KVQ_TRY(check_calib(shape, calib));
+    if (shape->use_klt) return KVQ_EUNSUPPORTED;
     KVQ_TRY(check_cache(shape, cache));
     KVQ_TRY(check_layers(shape, layer0, nlayers));
     if (num_tokens < 0 || !good_dtype(dtype)) return KVQ_EINVAL;
@@ -138,7 +171,8 @@ kvq_status kvq_decode_attention(const kvq_shape* shape, const kvq_calib* calib, 
                                 int32_t batch, void* out, int32_t out_dtype, void* workspace,
                                 size_t workspace_bytes, int32_t* dev_status, void* stream) {
     KVQ_TRY(check_shape(shape));
-    KVQ_TRY(check_calib(calib));
+    KVQ_TRY(check_calib(shape, calib));
+    if (shape->use_klt) return KVQ_EUNSUPPORTED;
     KVQ_TRY(check_cache(shape, cache));
     KVQ_TRY(check_layers(shape, layer0, nlayers));
     if (batch < 1 || max_pages_per_seq < 1 || (long)batch * shape->num_kv_heads > 65535) return KVQ_EINVAL;
@@ -163,7 +197,8 @@ kvq_status kvq_prefill_attention(const kvq_shape* shape, const kvq_calib* calib,
                                  const int32_t* seq_lens, int32_t batch, void* out, int32_t out_dtype,
                                  void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
     KVQ_TRY(check_shape(shape));
-    KVQ_TRY(check_calib(calib));
+    KVQ_TRY(check_calib(shape, calib));
+    if (shape->use_klt) return KVQ_EUNSUPPORTED;
     KVQ_TRY(check_cache(shape, cache));
     KVQ_TRY(check_layers(shape, layer0, nlayers));
     if (batch < 1 || q_len < 1 || max_pages_per_seq < 1 || (long)batch * shape->num_kv_heads > 65535)

@@ -1,0 +1,315 @@
+// kvq_klt.cu -- static per-head KLT of the keys: calibration (second moment,
+// eigenbasis, tensor scale), the key transform of the append, and the query
+// transform of the attention calls.
+//
+// Method: "NVFP4 attention cache on W4A4 Qwen3-8B" (rstation.ai), results
+// table rows "K: static per-head KLT" and "K: static KLT + smoothing": after
+// the static smoothing, each (layer, kv head) rotates its keys by a fixed
+// orthogonal 128 x 128 basis fitted on the calibration windows, and the query
+// is rotated to match (q~ = U^T (q * s), so q~ . U^T y = q . k).
+//
+// The basis is the eigenbasis of the second-moment matrix C = sum y y^T of
+// the smoothed calibration keys (position 0 of each window left out, as for
+// the smoothing absmax), ordered by decreasing eigenvalue, each vector signed
+// so that its largest-magnitude component is positive.  The key transform is
+// y'_i = sum_c U[c][i] y_c, each output one fp32 fused multiply-add chain
+// over c = 0..127 starting from 0 -- a fixed order, so the codes that follow
+// are reproducible bit for bit.
+#include <cuda_bf16.h>
+
+#include <type_traits>
+
+#include "kvq_common.cuh"
+#include "kvq_internal.h"
+#include "kvq_sync.cuh"
+#include "kvq_transform.cuh"
+
+namespace kvq {
+
+constexpr int kKltRows = 32;          // calibration tokens staged per step
+
+// ------------------------------------------------------------------ covariance
+// C[l][h] = sum over calibration tokens t >= t0 of y y^T, y = k * inv_s
+// (fp32).  One CTA per (layer, head), tokens in order: deterministic.
+// Thread (i, j) of a 16 x 16 grid owns the 8 x 8 block C[8i.., 8j..].
+template <typename T>
+__global__ void __launch_bounds__(256)
+klt_covariance_kernel(const T* __restrict__ k, int W, int Tlen, int Hkv, int t0,
+                      const float* __restrict__ inv_s, float* __restrict__ C) {
+    __shared__ __align__(16) float ys[kKltRows][kD];
+    const int h = blockIdx.x, l = blockIdx.y;
+    const int bi = threadIdx.x >> 4, bj = threadIdx.x & 15;
+    float acc[8][8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
+    const float* inv = inv_s + ((size_t)l * Hkv + h) * kD;
+    const int per_win = Tlen - t0;
+    const int total = W * per_win;
+    for (int base = 0; base < total; base += kKltRows) {
+        const int nrow = min(kKltRows, total - base);
+        __syncthreads();
+        for (int e = threadIdx.x; e < nrow * kD; e += blockDim.x) {
+            const int r = e / kD, c = e % kD;
+            const int idx = base + r, w = idx / per_win, t = t0 + idx % per_win;
+            const size_t off = ((((size_t)l * W + w) * Tlen + t) * Hkv + h) * kD + c;
+            ys[r][c] = __fmul_rn(load_elem(k + off), __ldg(inv + c));
+        }
+        __syncthreads();
+        for (int r = 0; r < nrow; ++r) {
+            float yi[8], yj[8];
+#pragma unroll
+            for (int a = 0; a < 8; ++a) {
+                yi[a] = ys[r][8 * bi + a];
+                yj[a] = ys[r][8 * bj + a];
+            }
+#pragma unroll
+            for (int a = 0; a < 8; ++a)
+#pragma unroll
+                for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(yi[a], yj[b], acc[a][b]);
+        }
+    }
+    float* out = C + ((size_t)l * Hkv + h) * kD * kD;
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) out[(8 * bi + a) * kD + 8 * bj + b] = acc[a][b];
+}
+
+// ------------------------------------------------------------------ eigenbasis
+// Cyclic parallel Jacobi on one symmetric 128 x 128 matrix (one CTA): each
+// round rotates 64 disjoint (p, q) planes chosen by the circle method (127
+// rounds cover every pair once per sweep); a rotation zeroes A[p][q]:
+//   theta = (A_qq - A_pp) / (2 A_pq),  t = sgn(theta) / (|theta| + sqrt(theta^2 + 1)),
+//   c = 1 / sqrt(t^2 + 1),  s = t c,
+// applied as A <- J^T A J and V <- V J.  The matrix is read from and the
+// basis written to the same array (U[c][i] = component c of vector i).
+constexpr int kJacobiSweeps = 12;
+constexpr size_t kJacobiSmem = 2 * kD * kD * sizeof(float) + 2 * 64 * sizeof(float) + 2 * 64 * sizeof(int) +
+                               kD * sizeof(float) + kD * sizeof(int);
+
+__global__ void __launch_bounds__(256) klt_jacobi_kernel(float* __restrict__ CU, int Hkv) {
+    extern __shared__ __align__(16) float sm[];
+    float* A = sm;                       // [128][128]
+    float* V = A + kD * kD;              // [128][128]
+    float* cs = V + kD * kD;             // c[64], s[64]
+    int* pq = reinterpret_cast<int*>(cs + 128);   // p[64], q[64]
+    float* ev = reinterpret_cast<float*>(pq + 128);
+    int* rank = reinterpret_cast<int*>(ev + kD);
+    const int h = blockIdx.x, l = blockIdx.y;
+    float* M = CU + ((size_t)l * Hkv + h) * kD * kD;
+    for (int e = threadIdx.x; e < kD * kD; e += blockDim.x) {
+        A[e] = M[e];
+        V[e] = (e / kD == e % kD) ? 1.0f : 0.0f;
+    }
+    __syncthreads();
+    for (int sweep = 0; sweep < kJacobiSweeps; ++sweep) {
+        for (int round = 0; round < kD - 1; ++round) {
+            if (threadIdx.x < 64) {
+                // circle method: 127 rotates around the fixed player 127
+                const int k = threadIdx.x;
+                int p, q;
+                if (k == 0) {
+                    p = round;
+                    q = kD - 1;
+                } else {
+                    p = (round + k) % (kD - 1);
+                    q = (round - k + (kD - 1)) % (kD - 1);
+                }
+                if (p > q) { const int x = p; p = q; q = x; }
+                const float apq = A[p * kD + q], app = A[p * kD + p], aqq = A[q * kD + q];
+                float c = 1.0f, s = 0.0f;
+                if (apq != 0.0f && fabsf(apq) > 1e-30f * (fabsf(app) + fabsf(aqq))) {
+                    const float theta = (aqq - app) / (2.0f * apq);
+                    const float t = copysignf(1.0f, theta) / (fabsf(theta) + sqrtf(theta * theta + 1.0f));
+                    c = 1.0f / sqrtf(t * t + 1.0f);
+                    s = t * c;
+                }
+                pq[k] = p;
+                pq[64 + k] = q;
+                cs[k] = c;
+                cs[64 + k] = s;
+            }
+            __syncthreads();
+            // rows: A <- J^T A   (pair k owns rows p_k and q_k)
+            for (int e = threadIdx.x; e < 64 * kD; e += blockDim.x) {
+                const int k = e / kD, col = e % kD;
+                const int p = pq[k], q = pq[64 + k];
+                const float c = cs[k], s = cs[64 + k];
+                const float ap = A[p * kD + col], aq = A[q * kD + col];
+                A[p * kD + col] = c * ap - s * aq;
+                A[q * kD + col] = s * ap + c * aq;
+            }
+            __syncthreads();
+            // columns: A <- A J, V <- V J
+            for (int e = threadIdx.x; e < 64 * kD; e += blockDim.x) {
+                const int k = e % 64, row = e / 64;
+                const int p = pq[k], q = pq[64 + k];
+                const float c = cs[k], s = cs[64 + k];
+                const float ap = A[row * kD + p], aq = A[row * kD + q];
+                A[row * kD + p] = c * ap - s * aq;
+                A[row * kD + q] = s * ap + c * aq;
+                const float vp = V[row * kD + p], vq = V[row * kD + q];
+                V[row * kD + p] = c * vp - s * vq;
+                V[row * kD + q] = s * vp + c * vq;
+            }
+            __syncthreads();
+        }
+    }
+    // unit length (the rotations' roundings drift the norms by ~1e-5), then
+    // order by decreasing eigenvalue (ties by index) and sign each vector
+    if (threadIdx.x < kD) {
+        const int i = threadIdx.x;
+        float n2 = 0.0f;
+        for (int c = 0; c < kD; ++c) n2 = fmaf(V[c * kD + i], V[c * kD + i], n2);
+        const float inv = 1.0f / sqrtf(n2);
+        for (int c = 0; c < kD; ++c) V[c * kD + i] *= inv;
+        ev[i] = A[i * kD + i];
+    }
+    __syncthreads();
+    if (threadIdx.x < kD) {
+        const int i = threadIdx.x;
+        int r = 0;
+        for (int j = 0; j < kD; ++j) r += (ev[j] > ev[i]) || (ev[j] == ev[i] && j < i);
+        rank[i] = r;
+    }
+    __syncthreads();
+    if (threadIdx.x < kD) {
+        const int i = threadIdx.x;          // source column
+        int big = 0;
+        float bv = -1.0f;
+        for (int c = 0; c < kD; ++c) {
+            const float a = fabsf(V[c * kD + i]);
+            if (a > bv) { bv = a; big = c; }
+        }
+        const float sg = V[big * kD + i] < 0.0f ? -1.0f : 1.0f;
+        const int dst = rank[i];
+        for (int c = 0; c < kD; ++c) M[c * kD + dst] = sg * V[c * kD + i];
+    }
+}
+
+// ------------------------------------------------------------------ transform
+// out_i = sum_c U[c][i] y_c for the rows of a tile, one fp32 FMA chain per
+// output over c in order.  The tile is 64 rows (tokens) x 128; thread
+// (tg, dg) of a 16 x 16 grid owns rows 4tg..4tg+3 and outputs 8dg..8dg+7.
+// Yt: [128][64] (transposed), U: [128][128], both in shared memory.
+__device__ __forceinline__ void klt_tile(const float* __restrict__ Yt, const float* __restrict__ U, int tg, int dg,
+                                         float (&acc)[4][8]) {
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
+#pragma unroll 4
+    for (int c = 0; c < kD; ++c) {
+        const float4 y4 = *reinterpret_cast<const float4*>(Yt + c * 64 + 4 * tg);
+        const float4 u0 = *reinterpret_cast<const float4*>(U + c * kD + 8 * dg);
+        const float4 u1 = *reinterpret_cast<const float4*>(U + c * kD + 8 * dg + 4);
+        const float y[4] = {y4.x, y4.y, y4.z, y4.w};
+        const float u[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(u[b], y[a], acc[a][b]);
+    }
+}
+
+constexpr size_t kKltTileSmem = (size_t)kD * kD * sizeof(float) + (size_t)kD * 64 * sizeof(float);
+
+// Load U of (l, h) into shared memory.
+__device__ __forceinline__ void klt_load_basis(float* Us, const float* __restrict__ U) {
+    for (int e = threadIdx.x; e < kD * kD / 4; e += blockDim.x)
+        reinterpret_cast<float4*>(Us)[e] = __ldg(reinterpret_cast<const float4*>(U) + e);
+}
+
+// Tensor absmax of the transformed calibration keys (every token, position 0
+// included): grid (token tiles, Hkv, L).
+template <typename T>
+__global__ void __launch_bounds__(256)
+klt_tensor_amax_kernel(const T* __restrict__ k, int rows, int Hkv, const float* __restrict__ inv_s,
+                       const float* __restrict__ U, uint32_t* __restrict__ gk_bits) {
+    extern __shared__ __align__(16) float sm[];
+    float* Us = sm;
+    float* Yt = sm + kD * kD;
+    const int h = blockIdx.y, l = blockIdx.z, r0 = blockIdx.x * 64;
+    klt_load_basis(Us, U + ((size_t)l * Hkv + h) * kD * kD);
+    const float* inv = inv_s + ((size_t)l * Hkv + h) * kD;
+    for (int e = threadIdx.x; e < 64 * kD; e += blockDim.x) {
+        const int r = e / kD, c = e % kD;
+        float y = 0.0f;
+        if (r0 + r < rows)
+            y = __fmul_rn(load_elem(k + (((size_t)l * rows + r0 + r) * Hkv + h) * kD + c), __ldg(inv + c));
+        Yt[c * 64 + r] = y;
+    }
+    __syncthreads();
+    const int tg = threadIdx.x >> 4, dg = threadIdx.x & 15;
+    float acc[4][8];
+    klt_tile(Yt, Us, tg, dg, acc);
+    float m = 0.0f;
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) m = fmaxf(m, fabsf(acc[a][b]));   // padded rows are 0
+#pragma unroll
+    for (int x = 16; x >= 1; x >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, x));
+    if ((threadIdx.x & 31) == 0) atomicMax(gk_bits + l, __float_as_uint(m));
+}
+
+// Value absmax (every token) for g_V.
+template <typename T>
+__global__ void klt_value_amax_kernel(const T* __restrict__ v, size_t per_layer, uint32_t* __restrict__ gv_bits) {
+    const int l = blockIdx.y;
+    float m = 0.0f;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < per_layer; i += (size_t)gridDim.x * blockDim.x)
+        m = fmaxf(m, fabsf(load_elem(v + (size_t)l * per_layer + i)));
+#pragma unroll
+    for (int x = 16; x >= 1; x >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, x));
+    if ((threadIdx.x & 31) == 0) atomicMax(gv_bits + l, __float_as_uint(m));
+}
+
+__global__ void klt_finalize_kernel(float* __restrict__ gk, float* __restrict__ gv, int L) {
+    const int l = blockIdx.x * blockDim.x + threadIdx.x;
+    if (l >= L) return;
+    const float a = gk[l], b = gv[l];
+    gk[l] = (a > 0.0f) ? __fdiv_rn(a, kTensorRange) : 1.0f;
+    gv[l] = (b > 0.0f) ? __fdiv_rn(b, kTensorRange) : 1.0f;
+}
+
+template <typename T>
+static kvq_status launch_calibrate_klt(const kvq_shape& s, const T* k, const T* v, int W, int Tlen, int exclude_pos0,
+                                       const kvq_calib& out, cudaStream_t st) {
+    // smoothing factors as kvq_calibrate_smoothing (its tensor scales are
+    // recomputed below for the rotated keys)
+    kvq_status r = calibrate(s, k, v, std::is_same<T, float>::value ? KVQ_F32 : KVQ_BF16, W, Tlen, exclude_pos0, out,
+                             st);
+    if (r != KVQ_OK) return r;
+    const int L = s.num_layers, H = s.num_kv_heads;
+    klt_covariance_kernel<T><<<dim3(H, L), 256, 0, st>>>(k, W, Tlen, H, exclude_pos0 ? 1 : 0, out.k_inv_smooth,
+                                                         out.k_klt);
+    if (cudaFuncSetAttribute(klt_jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kJacobiSmem) !=
+        cudaSuccess)
+        return KVQ_ECUDA;
+    klt_jacobi_kernel<<<dim3(H, L), 256, kJacobiSmem, st>>>(out.k_klt, H);
+    if (cudaMemsetAsync(out.k_gscale, 0, L * sizeof(float), st) != cudaSuccess ||
+        cudaMemsetAsync(out.v_gscale, 0, L * sizeof(float), st) != cudaSuccess)
+        return KVQ_ECUDA;
+    const int rows = W * Tlen;
+    if (cudaFuncSetAttribute(klt_tensor_amax_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kKltTileSmem) != cudaSuccess)
+        return KVQ_ECUDA;
+    klt_tensor_amax_kernel<T><<<dim3((rows + 63) / 64, H, L), 256, kKltTileSmem, st>>>(
+        k, rows, H, out.k_inv_smooth, out.k_klt, reinterpret_cast<uint32_t*>(out.k_gscale));
+    const size_t per_layer = (size_t)rows * H * kD;
+    klt_value_amax_kernel<T><<<dim3(64, L), 256, 0, st>>>(v, per_layer, reinterpret_cast<uint32_t*>(out.v_gscale));
+    klt_finalize_kernel<<<(L + 63) / 64, 64, 0, st>>>(out.k_gscale, out.v_gscale, L);
+    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ECUDA;
+}
+
+kvq_status calibrate_klt(const kvq_shape& s, const void* k, const void* v, int dtype, int W, int Tlen,
+                         int exclude_pos0, const kvq_calib& out, cudaStream_t st) {
+    if (dtype == KVQ_F32)
+        return launch_calibrate_klt(s, (const float*)k, (const float*)v, W, Tlen, exclude_pos0, out, st);
+    return launch_calibrate_klt(s, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, W, Tlen, exclude_pos0, out, st);
+}
+
+}  // namespace kvq

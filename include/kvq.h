@@ -102,6 +102,7 @@ typedef struct {
     int32_t page_size;      /* must be 16                                   */
     int32_t use_hadamard;   /* 1: keys rotated by normalised Hadamard-128   */
     int32_t k_format;       /* KVQ_K_NVFP4, or KVQ_K_BF16 (mixed cache)     */
+    int32_t use_klt;        /* 1: keys rotated by a static per-head KLT     */
 } kvq_shape;
 
 /* Static calibration state, device arrays of fp32 written by
@@ -111,6 +112,9 @@ typedef struct {
     float* k_inv_smooth;    /* [L][Hkv][128] 1 / s                          */
     float* k_gscale;        /* [L] FP32 tensor scale g_K of the keys        */
     float* v_gscale;        /* [L] FP32 tensor scale g_V of the values      */
+    float* k_klt;           /* [L][Hkv][128][128] KLT bases U (U[c][i] =    */
+                            /* component c of vector i); read only with     */
+                            /* use_klt, may be NULL otherwise               */
 } kvq_calib;
 
 typedef struct {
@@ -170,6 +174,26 @@ kvq_status kvq_calibrate_smoothing(const kvq_shape* shape, const void* k_calib, 
 kvq_status kvq_calibrate_native(const kvq_shape* shape, const void* k_calib, const void* v_calib,
                                 int32_t dtype, int32_t num_windows, int32_t window_len,
                                 const kvq_calib* out, void* stream);
+
+/*
+ * kvq_calibrate_klt -- smoothing followed by a static per-head KLT.
+ *
+ * [P1] results table, rows "K: static per-head KLT" and "K: static KLT +
+ * smoothing" (the best WT-val row).  The smoothing factors are those of
+ * kvq_calibrate_smoothing.  For each (layer, kv head) the basis U is the
+ * eigenbasis of C = sum y y^T over the smoothed calibration keys y = k * inv
+ * (positions t >= exclude_pos0 of every window), ordered by decreasing
+ * eigenvalue, each vector signed so that its largest-magnitude component is
+ * positive (fp32 cyclic Jacobi, 12 sweeps).  The keys are then transformed
+ * as y'_i = sum_c U[c][i] y_c, one fp32 fused multiply-add chain per output
+ * over c = 0..127; g_K = max |y'| / 2688 over every calibration token
+ * (position 0 included), g_V as kvq_calibrate_smoothing.  out->k_klt must be
+ * a [L][Hkv][128][128] fp32 device array; shape->use_klt must be 1 and
+ * use_hadamard 0.  Errors as kvq_calibrate_smoothing.
+ */
+kvq_status kvq_calibrate_klt(const kvq_shape* shape, const void* k_calib, const void* v_calib,
+                             int32_t dtype, int32_t num_windows, int32_t window_len,
+                             int32_t exclude_pos0, const kvq_calib* out, void* stream);
 
 /*
  * kvq_quantize_append -- transform, quantise and scatter tokens into the cache.

@@ -1,0 +1,60 @@
+"""Static per-head KLT on the GPU against the oracle ("NVFP4 attention cache
+on W4A4 Qwen3-8B", results table rows "K: static per-head KLT" and "K:
+static KLT + smoothing").
+
+The basis comes out of an fp32 Jacobi eigensolver on the device and of fp64
+eigh in the oracle; it is compared as a basis (orthogonal, diagonalising the
+second moment, same order and signs, each vector close to the oracle's where
+the eigenvalue gap makes it well defined).  Everything after the basis --
+tensor scales, codes, attention -- is compared given the device's basis.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _windows(layers=2, windows=4, length=128):
+    w = dataclasses.replace(synth.WORKLOADS["qwen3_8b"], num_layers=layers, calib_windows=windows,
+                            calib_len=length)
+    win = [synth.calibration_windows(w, l) for l in range(layers)]
+    return w, torch.stack([x[0] for x in win]), torch.stack([x[1] for x in win])
+
+
+def test_klt_calibration_matches_oracle(kvq):
+    w, kc, vc = _windows()
+    shape = kvq.Shape(2, w.num_q_heads, w.num_kv_heads, use_klt=True)
+    cal = kvq.calibrate_klt(shape, kc.cuda().contiguous(), vc.cuda().contiguous())
+    torch.cuda.synchronize()
+    k, v = kc.float().numpy(), vc.float().numpy()
+    s_o, inv_o, U_o, ev_o = oracle.calibrate_klt(k, v, exclude_pos0=True)
+    np.testing.assert_array_equal(cal.k_smooth.cpu().numpy(), s_o)
+    np.testing.assert_array_equal(cal.k_inv_smooth.cpu().numpy(), inv_o)
+    U = cal.k_klt.cpu().numpy()
+    for l in range(2):
+        y = oracle.transform_keys(k[l, :, 1:].reshape(-1, 8, 128), inv_o[l])
+        for h in range(8):
+            u = U[l, h].astype(np.float64)
+            np.testing.assert_allclose(u.T @ u, np.eye(128), atol=2e-5)
+            C = y[:, h].astype(np.float64).T @ y[:, h].astype(np.float64)
+            D = u.T @ C @ u
+            lam = np.diag(D)
+            assert np.abs(D - np.diag(lam)).max() <= 2e-5 * lam.max(), (l, h)
+            assert np.all(np.diff(lam) <= 1e-5 * lam.max()), (l, h)        # decreasing
+            assert np.all(u[np.argmax(np.abs(u), axis=0), np.arange(128)] > 0)
+            # vector by vector against fp64 eigh where the relative gap is wide
+            lo = ev_o[l, h] * y.shape[0]                                 # oracle's C is / N
+            gap = np.minimum(np.abs(np.diff(lo, prepend=np.inf)), np.abs(np.diff(lo, append=-np.inf)))
+            wide = gap > 1e-3 * lo.max()
+            dots = np.abs(np.sum(u * U_o[l, h].astype(np.float64), axis=0))
+            assert np.all(dots[wide] > 1 - 1e-4), (l, h, dots[wide].min())
+    # tensor scales given the device's basis: bit for bit
+    gk, gv = oracle.klt_tensor_scales(k, v, inv_o, U)
+    np.testing.assert_array_equal(cal.k_gscale.cpu().numpy(), gk)
+    np.testing.assert_array_equal(cal.v_gscale.cpu().numpy(), gv)
