@@ -147,7 +147,6 @@ kvq_status kvq_quantize_append(const kvq_shape* shape, const kvq_calib* calib, c
                                void* stream) {
     KVQ_TRY(check_shape(shape));
     KVQ_TRY(check_calib(shape, calib));
-    if (shape->use_klt) return KVQ_EUNSUPPORTED;
     KVQ_TRY(check_cache(shape, cache));
     KVQ_TRY(check_layers(shape, layer0, nlayers));
     if (num_tokens < 0 || !good_dtype(dtype)) return KVQ_EINVAL;

@@ -23,6 +23,9 @@ kvq_status calibrate_native(const kvq_shape& s, const void* k, const void* v, in
                             const kvq_calib& out, cudaStream_t st);
 kvq_status calibrate_klt(const kvq_shape& s, const void* k, const void* v, int dtype, int W, int Tlen,
                          int exclude_pos0, const kvq_calib& out, cudaStream_t st);
+kvq_status append_klt_keys(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cache, int layer0, int nlayers,
+                           const void* k, int dtype, const int64_t* slots, int num_tokens, int32_t* status,
+                           cudaStream_t st);
 kvq_status quantize_append(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cache, int layer0,
                            int nlayers, const void* k, const void* v, int dtype, const int64_t* slots,
                            int num_tokens, int32_t* status, cudaStream_t st);

@@ -275,6 +275,110 @@ __global__ void klt_finalize_kernel(float* __restrict__ gk, float* __restrict__ 
     gv[l] = (b > 0.0f) ? __fdiv_rn(b, kTensorRange) : 1.0f;
 }
 
+// ------------------------------------------------------------------ append
+// Keys of the KLT cache: grid (tiles of 64 tokens, Hkv, nlayers).  Smoothing
+// y = k * inv_s, the transform y' = U^T y (klt_tile), then the NVFP4
+// quantiser of the append (absmax -> E4M3 scale -> reciprocal -> E2M1, each
+// step one fp32 rounding) and the scatter to the token's slot.  Thread
+// (tg, dg) holds dims 8dg..8dg+7 of 4 tokens; the two threads of a 16-block
+// (dg, dg ^ 1) are neighbouring lanes and share its absmax by a shuffle.
+__device__ __forceinline__ uint32_t klt_e2m1x2(float hi, float lo) {
+    uint16_t r;
+    asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u16.u8 %0, t; }" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+constexpr size_t kKltAppendSmem = kKltTileSmem + 128 * sizeof(float) + 64 * sizeof(int64_t) + 16;
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+klt_append_keys_kernel(const T* __restrict__ k, const int64_t* __restrict__ slots, int num_tokens, int Hkv,
+                       const float* __restrict__ inv_s, const float* __restrict__ U, const float* __restrict__ gk,
+                       uint8_t* __restrict__ cache, int64_t layer_stride, int num_pages, int32_t* __restrict__ status) {
+    extern __shared__ __align__(16) float sm[];
+    float* Us = sm;
+    float* Yt = Us + kD * kD;
+    float* rtab = Yt + kD * 64;
+    int64_t* sslot = reinterpret_cast<int64_t*>(rtab + 128);
+    const int h = blockIdx.y, li = blockIdx.z, t0 = blockIdx.x * 64;
+    klt_load_basis(Us, U + ((size_t)li * Hkv + h) * kD * kD);
+    const float g = __ldg(gk + li);
+    const float enc = __frcp_rn(__fmul_rn(6.0f, g));
+    if (threadIdx.x < 128) {
+        // the append's reciprocal of every E4M3 scale code: 1/(val(c) g)
+        const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), g);
+        rtab[threadIdx.x] = (d == 0.0f) ? 0.0f : __frcp_rn(d);
+    } else if (threadIdx.x < 192) {
+        const int tt = threadIdx.x - 128;
+        sslot[tt] = (t0 + tt < num_tokens) ? __ldg(slots + t0 + tt) : -1;
+    }
+    const float* inv = inv_s + ((size_t)li * Hkv + h) * kD;
+    for (int e = threadIdx.x; e < 64 * kD; e += blockDim.x) {
+        const int r = e / kD, c = e % kD;
+        float y = 0.0f;
+        if (t0 + r < num_tokens)
+            y = __fmul_rn(load_elem(k + (((size_t)li * num_tokens + t0 + r) * Hkv + h) * kD + c), __ldg(inv + c));
+        Yt[c * 64 + r] = y;
+    }
+    __syncthreads();
+    const int tg = threadIdx.x >> 4, dg = threadIdx.x & 15;
+    float acc[4][8];
+    klt_tile(Yt, Us, tg, dg, acc);
+    const int64_t num_slots = (int64_t)num_pages * kPage;
+    uint8_t* layer_cache = cache + (size_t)li * layer_stride;
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        float m = 0.0f;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) m = fmaxf(m, fabsf(acc[a][b]));
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));       // the other half of the 16-block
+        const uint32_t sf = e4m3_rn(__fmul_rn(m, enc));
+        const float r = rtab[sf & 0x7Fu];
+        uint32_t w = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            w |= klt_e2m1x2(__fmul_rn(acc[a][2 * j + 1], r), __fmul_rn(acc[a][2 * j], r)) << (8 * j);
+        const int tt = 4 * tg + a;
+        const int64_t slot = sslot[tt];
+        if (slot >= num_slots) {
+            if (dg == 0) set_status(status, KVQ_DEV_BAD_SLOT);
+        } else if (slot >= 0) {
+            uint8_t* tile = layer_cache + ((size_t)(slot >> 4) * Hkv + h) * kTile;
+            const int off = (int)(slot & 15);
+            *reinterpret_cast<uint32_t*>(tile + kKCodes + off * 64 + 4 * dg) = w;
+            if ((dg & 1) == 0) tile[kKScales + off * 8 + (dg >> 1)] = (uint8_t)sf;
+        }
+    }
+}
+
+kvq_status append_klt_keys(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cache, int layer0, int nlayers,
+                           const void* k, int dtype, const int64_t* slots, int num_tokens, int32_t* status,
+                           cudaStream_t st) {
+    const int H = s.num_kv_heads;
+    const float* inv = c.k_inv_smooth + (size_t)layer0 * H * kD;
+    const float* U = c.k_klt + (size_t)layer0 * H * kD * kD;
+    const float* gk = c.k_gscale + layer0;
+    uint8_t* base = cache.data + (size_t)layer0 * cache.layer_stride_bytes;
+    const dim3 grid((num_tokens + 63) / 64, H, nlayers);
+    cudaError_t e;
+    if (dtype == KVQ_F32) {
+        e = cudaFuncSetAttribute(klt_append_keys_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kKltAppendSmem);
+        if (e != cudaSuccess) return KVQ_ECUDA;
+        klt_append_keys_kernel<float><<<grid, 256, kKltAppendSmem, st>>>((const float*)k, slots, num_tokens, H, inv,
+                                                                       U, gk, base, cache.layer_stride_bytes,
+                                                                       cache.num_pages, status);
+    } else {
+        e = cudaFuncSetAttribute(klt_append_keys_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kKltAppendSmem);
+        if (e != cudaSuccess) return KVQ_ECUDA;
+        klt_append_keys_kernel<__nv_bfloat16><<<grid, 256, kKltAppendSmem, st>>>(
+            (const __nv_bfloat16*)k, slots, num_tokens, H, inv, U, gk, base, cache.layer_stride_bytes,
+            cache.num_pages, status);
+    }
+    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ECUDA;
+}
+
 template <typename T>
 static kvq_status launch_calibrate_klt(const kvq_shape& s, const T* k, const T* v, int W, int Tlen, int exclude_pos0,
                                        const kvq_calib& out, cudaStream_t st) {

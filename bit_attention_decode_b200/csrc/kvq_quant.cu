@@ -159,8 +159,10 @@ append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* _
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t num_slots = (int64_t)num_pages * kPage;
     // tile geometry: NVFP4 keys, or bf16 keys (mixed cache)
-    const int tile_b = k_bf16 ? kTileBf16K : kTile;
-    const int v_codes = k_bf16 ? kBf16VCodes : kVCodes, v_scales = k_bf16 ? kBf16VScales : kVScales;
+    // k_bf16: 0 packed keys, 1 bf16 keys (mixed cache), 2 keys written by the
+    // KLT kernel (packed layout, this kernel does the values only)
+    const int tile_b = k_bf16 == 1 ? kTileBf16K : kTile;
+    const int v_codes = k_bf16 == 1 ? kBf16VCodes : kVCodes, v_scales = k_bf16 == 1 ? kBf16VScales : kVScales;
 
     if (threadIdx.x == 0) {
         s_timeout = 0;
@@ -266,7 +268,9 @@ append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* _
                 uint8_t* tile = layer_cache + ((size_t)page * Hkv + h) * tile_b;
                 uint2 codes;
                 uint32_t sf;
-                if (k_bf16) {
+                if (k_bf16 == 2) {
+                    // KLT cache: the keys are transformed and written by their own kernel
+                } else if (k_bf16) {
                     // mixed cache: the key block is kept as bf16, untransformed
                     if (ok) {
                         uint32_t wb[8];
@@ -390,7 +394,7 @@ kvq_status quantize_append(const kvq_shape& s, const kvq_calib& c, const kvq_cac
                            int nlayers, const void* k, const void* v, int dtype, const int64_t* slots,
                            int num_tokens, int32_t* status, cudaStream_t st) {
     const int H = s.num_kv_heads;
-    const int kbf = s.k_format == KVQ_K_BF16 ? 1 : 0;
+    const int kbf = s.use_klt ? 2 : (s.k_format == KVQ_K_BF16 ? 1 : 0);
     const float* inv_s = c.k_inv_smooth + (size_t)layer0 * H * kD;
     const float* gk = c.k_gscale + layer0;
     const float* gv = c.v_gscale + layer0;
@@ -423,7 +427,9 @@ kvq_status quantize_append(const kvq_shape& s, const kvq_calib& c, const kvq_cac
         append_kernel<__nv_bfloat16><<<grid, threads, smem, st>>>(
             (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, slots, num_tokens, nlayers, H, tc, inv_s, gk, gv, base,
             cache.layer_stride_bytes, cache.num_pages, s.use_hadamard, kbf, status);
-    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ECUDA;
+    if (cudaGetLastError() != cudaSuccess) return KVQ_ECUDA;
+    if (s.use_klt) return append_klt_keys(s, c, cache, layer0, nlayers, k, dtype, slots, num_tokens, status, st);
+    return KVQ_OK;
 }
 
 kvq_status round_e2m1(const float* x, uint8_t* out, int64_t n, cudaStream_t st) {

@@ -96,7 +96,7 @@ class Problem:
 
 def build_problem(kvq, w: synth.Workload, lens, layers=None, extra_tokens: int = 0, shuffle: bool = True,
                   keep_host=True, device="cuda", gen_device="cpu", keep=None, all_layers_one_call=False,
-                  keep_tails=False, native=False, k_format=0):
+                  keep_tails=False, native=False, k_format=0, klt=False):
     """Calibrate, then append each sequence's first lens[b] tokens.
 
     keep:      optional set of (layer index, sequence) whose host copies are kept
@@ -107,17 +107,20 @@ def build_problem(kvq, w: synth.Workload, lens, layers=None, extra_tokens: int =
                device, as tails_k/v [extra][nl][B][Hkv][D].
     native:    calibrate the keys in their native basis (no smoothing).
     k_format:  1 for the mixed cache (bf16 keys, NVFP4 values).
+    klt:       smoothing plus the static per-head KLT (kvq.calibrate_klt).
     """
     layers = list(range(w.num_layers)) if layers is None else list(layers)
     lens = torch.as_tensor(lens, dtype=torch.int32)
     nl, B = len(layers), len(lens)
     shape = kvq.Shape(num_layers=nl, num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads,
-                      use_hadamard=w.hadamard, k_format=k_format)
+                      use_hadamard=w.hadamard, k_format=k_format, use_klt=klt)
     wins = [synth.calibration_windows(w, l, gen_device) for l in layers]
     kc = torch.stack([x[0] for x in wins])
     vc = torch.stack([x[1] for x in wins])
     del wins
-    if native:
+    if klt:
+        calib = kvq.calibrate_klt(shape, kc.to(device).contiguous(), vc.to(device).contiguous())
+    elif native:
         calib = kvq.calibrate_native(shape, kc.to(device).contiguous(), vc.to(device).contiguous())
     else:
         calib = kvq.calibrate_smoothing(shape, kc.to(device).contiguous(), vc.to(device).contiguous())
@@ -158,6 +161,7 @@ def build_problem(kvq, w: synth.Workload, lens, layers=None, extra_tokens: int =
     p.tails = tails
     p.native = native
     p.k_format = k_format
+    p.klt = klt
     return p
 
 
@@ -179,6 +183,14 @@ def oracle_sequence(p: Problem, li: int, b: int, n: int, cal):
     if getattr(p, "k_format", 0) == 1:
         vc, vsf = oracle.quantize_rows(v[:n], gv[li])
         return {"kc": oracle.round_bf16(k[:n]), "ksf": None, "vc": vc, "vsf": vsf}
+    if getattr(p, "klt", False):
+        # smoothing, then the device's KLT basis in the fixed FMA order
+        U = p.calib.k_klt[li].cpu().numpy()
+        y = oracle.transform_keys(k[:n], inv[li])
+        yk = np.stack([oracle.klt_apply(y[:, h], U[h]) for h in range(y.shape[1])], axis=1)
+        kc, ksf = oracle.quantize_rows(yk, gk[li])
+        vc, vsf = oracle.quantize_rows(v[:n], gv[li])
+        return {"kc": kc, "ksf": ksf, "vc": vc, "vsf": vsf}
     return oracle.quantize_kv(k[:n], v[:n], inv[li], gk[li], gv[li], p.w.hadamard)
 
 
@@ -191,4 +203,11 @@ def oracle_attend(p: Problem, li: int, b: int, q_rows: np.ndarray, q_start: int,
         # bf16 keys: the query is used as given, the keys as stored
         return oracle.attention(q_rows, q_start, np.ones_like(s[li]), qz["kc"].astype(np.float64), vx, False)
     kx = oracle.dequantize_rows(qz["kc"], qz["ksf"], gk[li])
+    if getattr(p, "klt", False):
+        # the query rotated to match: q~ = U^T (q * s) per kv head, in fp64
+        U = p.calib.k_klt[li].cpu().numpy().astype(np.float64)
+        G = q_rows.shape[1] // U.shape[0]
+        qs = np.asarray(q_rows, np.float64) * np.repeat(np.asarray(s[li], np.float64), G, axis=0)[None]
+        qt = np.einsum("thc,hci->thi", qs, np.repeat(U, G, axis=0))
+        return oracle.attention(qt.astype(np.float32), q_start, np.ones_like(s[li]), kx, vx, False)
     return oracle.attention(q_rows, q_start, s[li], kx, vx, p.w.hadamard)

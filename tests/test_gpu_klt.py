@@ -58,3 +58,24 @@ def test_klt_calibration_matches_oracle(kvq):
     gk, gv = oracle.klt_tensor_scales(k, v, inv_o, U)
     np.testing.assert_array_equal(cal.k_gscale.cpu().numpy(), gk)
     np.testing.assert_array_equal(cal.v_gscale.cpu().numpy(), gv)
+
+
+def _klt_problem(kvq, lens, layers=2):
+    import harness
+    w = dataclasses.replace(synth.WORKLOADS["qwen3_8b"], num_layers=layers, batch=len(lens), calib_windows=4,
+                            calib_len=128)
+    return harness.build_problem(kvq, w, lens=lens, klt=True)
+
+
+def test_klt_append_codes_bit_exact(kvq):
+    import harness
+    lens = [5, 150, 301]
+    p = _klt_problem(kvq, lens)
+    cal = harness.calib_host(p)
+    for li in range(2):
+        layer = p.cache.data[li].cpu().numpy()
+        for b, n in enumerate(lens):
+            got = harness.read_tokens(layer, 8, p.page_table[b].numpy(), n)
+            want = harness.oracle_sequence(p, li, b, n, cal)
+            for name, g in zip(("kc", "ksf", "vc", "vsf"), got):
+                np.testing.assert_array_equal(g, want[name], err_msg=f"{name} layer {li} seq {b}")
