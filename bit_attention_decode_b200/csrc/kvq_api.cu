@@ -171,7 +171,6 @@ kvq_status kvq_decode_attention(const kvq_shape* shape, const kvq_calib* calib, 
                                 size_t workspace_bytes, int32_t* dev_status, void* stream) {
     KVQ_TRY(check_shape(shape));
     KVQ_TRY(check_calib(shape, calib));
-    if (shape->use_klt) return KVQ_EUNSUPPORTED;
     KVQ_TRY(check_cache(shape, cache));
     KVQ_TRY(check_layers(shape, layer0, nlayers));
     if (batch < 1 || max_pages_per_seq < 1 || (long)batch * shape->num_kv_heads > 65535) return KVQ_EINVAL;
@@ -197,7 +196,6 @@ kvq_status kvq_prefill_attention(const kvq_shape* shape, const kvq_calib* calib,
                                  void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
     KVQ_TRY(check_shape(shape));
     KVQ_TRY(check_calib(shape, calib));
-    if (shape->use_klt) return KVQ_EUNSUPPORTED;
     KVQ_TRY(check_cache(shape, cache));
     KVQ_TRY(check_layers(shape, layer0, nlayers));
     if (batch < 1 || q_len < 1 || max_pages_per_seq < 1 || (long)batch * shape->num_kv_heads > 65535)

@@ -13,6 +13,7 @@ struct AttnArgs {
     int64_t layer_stride;
     int num_pages, Hkv, Hq, G, hadamard;
     int kbf16;                 // keys stored as bf16 (mixed cache)
+    int qpre;                  // q already carries the smoothing and the KLT (fp32)
     const float* smooth;       // [nl][Hkv][D] at layer0
     const float* gk;           // [nl] at layer0
     const float* gv;

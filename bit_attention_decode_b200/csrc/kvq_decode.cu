@@ -80,10 +80,18 @@ DecodePlan decode_plan(const kvq_shape& s, int nlayers, int batch, int max_pages
     return {pps, splits};
 }
 
-size_t decode_workspace(const kvq_shape& s, int nlayers, int batch, int max_pages) {
+// workspace: split partials, then (KLT cache) the transformed queries
+static size_t partial_bytes(const kvq_shape& s, int nlayers, int batch, int max_pages) {
     DecodePlan p = decode_plan(s, nlayers, batch, max_pages);
     if (p.splits == 1) return 0;
     return (size_t)nlayers * batch * s.num_q_heads * p.splits * kPartialStride * sizeof(float);
+}
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t decode_workspace(const kvq_shape& s, int nlayers, int batch, int max_pages) {
+    const size_t part = partial_bytes(s, nlayers, batch, max_pages);
+    if (!s.use_klt) return part;
+    return align256(part) + (size_t)nlayers * batch * s.num_q_heads * kD * sizeof(float);
 }
 
 static AttnArgs make_args(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cache, int layer0,
@@ -121,7 +129,18 @@ kvq_status decode(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cache
     a.pps = p.pages_per_split;
     a.q_len = 1;
     a.partials = reinterpret_cast<float*>(ws);
-    const bool qb = q_dtype == KVQ_BF16, ob = out_dtype == KVQ_BF16;
+    bool qb = q_dtype == KVQ_BF16;
+    const bool ob = out_dtype == KVQ_BF16;
+    if (s.use_klt) {
+        // the queries, rotated by the KLT (and smoothed), go through the workspace
+        float* qt = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                             align256(partial_bytes(s, nlayers, batch, max_pages)));
+        const kvq_status r = klt_queries(s, c, layer0, nlayers, q, q_dtype, batch, qt, st);
+        if (r != KVQ_OK) return r;
+        a.q = qt;
+        a.qpre = 1;
+        qb = false;
+    }
     if (launch_decode_tc(a, nlayers, qb, ob, st) != cudaSuccess) return KVQ_ECUDA;
     if (p.splits > 1) {
         dim3 g2(batch * s.num_q_heads, nlayers);
@@ -131,16 +150,29 @@ kvq_status decode(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cache
     return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ECUDA;
 }
 
-size_t prefill_workspace(const kvq_shape&, int, int, int) { return 0; }
+size_t prefill_workspace(const kvq_shape& s, int nlayers, int batch, int q_len) {
+    // KLT cache: the rotated queries
+    if (!s.use_klt) return 0;
+    return (size_t)nlayers * batch * q_len * s.num_q_heads * kD * sizeof(float);
+}
 
 kvq_status prefill(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cache, int layer0, int nlayers,
                    const void* q, int q_dtype, int q_len, const int32_t* q_start, const int32_t* page_table,
-                   int max_pages, const int32_t* seq_lens, int batch, void* out, int out_dtype, void*, size_t,
+                   int max_pages, const int32_t* seq_lens, int batch, void* out, int out_dtype, void* ws, size_t,
                    int32_t* status, cudaStream_t st) {
     AttnArgs a = make_args(s, c, cache, layer0, q, page_table, max_pages, seq_lens, batch, out, status);
     a.q_len = q_len;
     a.q_start = q_start;
-    const bool qb = q_dtype == KVQ_BF16, ob = out_dtype == KVQ_BF16;
+    bool qb = q_dtype == KVQ_BF16;
+    const bool ob = out_dtype == KVQ_BF16;
+    if (s.use_klt) {
+        float* qt = reinterpret_cast<float*>(ws);
+        const kvq_status r = klt_queries(s, c, layer0, nlayers, q, q_dtype, batch * q_len, qt, st);
+        if (r != KVQ_OK) return r;
+        a.q = qt;
+        a.qpre = 1;
+        qb = false;
+    }
     if (launch_prefill_tc(a, nlayers, qb, ob, st) != cudaSuccess) return KVQ_ECUDA;
     return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ECUDA;
 }

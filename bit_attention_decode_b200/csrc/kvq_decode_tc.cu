@@ -244,9 +244,15 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
                 for (int i = 0; i < 32; ++i) qv[i] = head_ok ? qv[i] : 0.0f;
                 scale = kLog2e * kInvSqrt128;
             } else {
-                const float* srow = a.smooth + ((size_t)li * Hkv + h) * kD + 32 * c;
+                if (a.qpre) {
+                    // the KLT cache: q already carries the smoothing and the rotation
 #pragma unroll
-                for (int i = 0; i < 32; ++i) qv[i] = head_ok ? qv[i] * __ldg(srow + i) : 0.0f;
+                    for (int i = 0; i < 32; ++i) qv[i] = head_ok ? qv[i] : 0.0f;
+                } else {
+                    const float* srow = a.smooth + ((size_t)li * Hkv + h) * kD + 32 * c;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) qv[i] = head_ok ? qv[i] * __ldg(srow + i) : 0.0f;
+                }
                 scale = __ldg(a.gk + li) * kLog2e * kInvSqrt128;
             }
             if (!KB && a.hadamard) {

@@ -26,6 +26,8 @@ kvq_status calibrate_klt(const kvq_shape& s, const void* k, const void* v, int d
 kvq_status append_klt_keys(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cache, int layer0, int nlayers,
                            const void* k, int dtype, const int64_t* slots, int num_tokens, int32_t* status,
                            cudaStream_t st);
+kvq_status klt_queries(const kvq_shape& s, const kvq_calib& c, int layer0, int nlayers, const void* q, int q_dtype,
+                       int rows, float* out, cudaStream_t st);
 kvq_status quantize_append(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cache, int layer0,
                            int nlayers, const void* k, const void* v, int dtype, const int64_t* slots,
                            int num_tokens, int32_t* status, cudaStream_t st);

@@ -379,6 +379,67 @@ kvq_status append_klt_keys(const kvq_shape& s, const kvq_calib& c, const kvq_cac
     return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ECUDA;
 }
 
+// ------------------------------------------------------------------ queries
+// q~ = U^T (q * s) for every query vector of a KLT cache (decode and
+// prefill), written as fp32: grid (tiles of 64 vectors, Hkv, nlayers); the
+// vectors of kv head h are (row r, group member j) -> q[(l, r)][h G + j].
+template <typename TQ>
+__global__ void __launch_bounds__(256)
+klt_query_kernel(const TQ* __restrict__ q, int rows, int Hq, int Hkv, const float* __restrict__ smooth,
+                 const float* __restrict__ U, float* __restrict__ out) {
+    extern __shared__ __align__(16) float sm[];
+    float* Us = sm;
+    float* Yt = Us + kD * kD;
+    const int h = blockIdx.y, l = blockIdx.z, v0 = blockIdx.x * 64;
+    const int G = Hq / Hkv, nvec = rows * G;
+    klt_load_basis(Us, U + ((size_t)l * Hkv + h) * kD * kD);
+    const float* sr = smooth + ((size_t)l * Hkv + h) * kD;
+    for (int e = threadIdx.x; e < 64 * kD; e += blockDim.x) {
+        const int vv = e / kD, c = e % kD, vec = v0 + vv;
+        float y = 0.0f;
+        if (vec < nvec) {
+            const int r = vec / G, j = vec % G;
+            y = load_elem(q + (((size_t)l * rows + r) * Hq + h * G + j) * kD + c) * __ldg(sr + c);
+        }
+        Yt[c * 64 + vv] = y;
+    }
+    __syncthreads();
+    const int tg = threadIdx.x >> 4, dg = threadIdx.x & 15;
+    float acc[4][8];
+    klt_tile(Yt, Us, tg, dg, acc);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const int vec = v0 + 4 * tg + a;
+        if (vec >= nvec) continue;
+        const int r = vec / G, j = vec % G;
+        float4* o = reinterpret_cast<float4*>(out + (((size_t)l * rows + r) * Hq + h * G + j) * kD + 8 * dg);
+        o[0] = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+        o[1] = make_float4(acc[a][4], acc[a][5], acc[a][6], acc[a][7]);
+    }
+}
+
+kvq_status klt_queries(const kvq_shape& s, const kvq_calib& c, int layer0, int nlayers, const void* q, int q_dtype,
+                       int rows, float* out, cudaStream_t st) {
+    const int H = s.num_kv_heads, G = s.num_q_heads / H;
+    const float* sm = c.k_smooth + (size_t)layer0 * H * kD;
+    const float* U = c.k_klt + (size_t)layer0 * H * kD * kD;
+    const dim3 grid((unsigned)(((long)rows * G + 63) / 64), H, nlayers);
+    cudaError_t e;
+    if (q_dtype == KVQ_F32) {
+        e = cudaFuncSetAttribute(klt_query_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kKltTileSmem);
+        if (e != cudaSuccess) return KVQ_ECUDA;
+        klt_query_kernel<float><<<grid, 256, kKltTileSmem, st>>>((const float*)q, rows, s.num_q_heads, H, sm, U, out);
+    } else {
+        e = cudaFuncSetAttribute(klt_query_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kKltTileSmem);
+        if (e != cudaSuccess) return KVQ_ECUDA;
+        klt_query_kernel<__nv_bfloat16><<<grid, 256, kKltTileSmem, st>>>((const __nv_bfloat16*)q, rows,
+                                                                         s.num_q_heads, H, sm, U, out);
+    }
+    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ECUDA;
+}
+
 template <typename T>
 static kvq_status launch_calibrate_klt(const kvq_shape& s, const T* k, const T* v, int W, int Tlen, int exclude_pos0,
                                        const kvq_calib& out, cudaStream_t st) {

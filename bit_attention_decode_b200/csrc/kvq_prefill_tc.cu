@@ -328,9 +328,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                     if constexpr (KB) {
                         scale = kLog2e * kInvSqrt128;     // bf16 keys: the query as given
                     } else {
-                        const float* srow = a.smooth + ((size_t)li * a.Hkv + h) * kD;
+                        if (!a.qpre) {   // (the KLT cache's queries arrive smoothed and rotated)
+                            const float* srow = a.smooth + ((size_t)li * a.Hkv + h) * kD;
 #pragma unroll
-                        for (int i = 0; i < kD; ++i) x[i] *= __ldg(srow + i);
+                            for (int i = 0; i < kD; ++i) x[i] *= __ldg(srow + i);
+                        }
                         scale = __ldg(a.gk + li) * kLog2e * kInvSqrt128;
                     }
                     if (!KB && a.hadamard) {

@@ -79,3 +79,36 @@ def test_klt_append_codes_bit_exact(kvq):
             want = harness.oracle_sequence(p, li, b, n, cal)
             for name, g in zip(("kc", "ksf", "vc", "vsf"), got):
                 np.testing.assert_array_equal(g, want[name], err_msg=f"{name} layer {li} seq {b}")
+
+
+def test_klt_decode_within_tolerance(kvq):
+    import harness
+    lens = [5, 150, 301]
+    p = _klt_problem(kvq, lens)
+    cal = harness.calib_host(p)
+    q = torch.stack([synth.decode_queries(p.w, l, 0) for l in p.layers])
+    for dt, tag in ((torch.float32, "f32"), (torch.bfloat16, "bf16")):
+        out = kvq.decode_attention(p.shape, p.calib, p.cache, q.cuda(), p.page_table.cuda(), p.lens.cuda(),
+                                   out_dtype=dt).float().cpu().numpy()
+        for li in range(2):
+            for b, n in enumerate(lens):
+                want = harness.oracle_attend(p, li, b, q[li, b].float().numpy()[None], n - 1, n, cal)
+                harness.check_attention(out[li, b], want[0], f"klt decode layer {li} seq {b} {tag}")
+
+
+def test_klt_prefill_within_tolerance(kvq):
+    import harness
+    w = dataclasses.replace(synth.WORKLOADS["qwen3_8b"], num_layers=2, batch=2, calib_windows=4, calib_len=128,
+                            prefill_chunk=48)
+    P0, Tq = [100, 33], 48
+    lens = [n + Tq for n in P0]
+    p = harness.build_problem(kvq, w, lens=lens, klt=True)
+    cal = harness.calib_host(p)
+    q = torch.stack([synth.prefill_queries(w, l) for l in p.layers])
+    q_start = torch.tensor(P0, dtype=torch.int32)
+    out = kvq.prefill_attention(p.shape, p.calib, p.cache, q.cuda(), q_start.cuda(), p.page_table.cuda(),
+                                p.lens.cuda(), out_dtype=torch.float32).float().cpu().numpy()
+    for li in range(2):
+        for b in range(2):
+            want = harness.oracle_attend(p, li, b, q[li, b].float().numpy(), P0[b], lens[b], cal)
+            harness.check_attention(out[li, b], want, f"klt prefill layer {li} seq {b}")
