@@ -47,6 +47,8 @@ def parse():
                     help="ragged (default, the decode-throughput workload); prefill, qwen3_8b, hadamard: "
                          "the chunked-prefill and prefix workloads, for their own kernel numbers")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--klt", action="store_true",
+                    help="ragged workload with smoothing plus the static per-head KLT of the keys")
     ap.add_argument("--k-format", default="nvfp4", choices=["nvfp4", "bf16"],
                     help="key storage of the ragged workload: packed NVFP4, or bf16 keys with NVFP4 values")
     ap.add_argument("--source-sha", action="store_true",
@@ -212,11 +214,12 @@ def ncu_traffic():
 class Ragged:
     """Device-resident ragged decode workload (one replica)."""
 
-    def __init__(self, kvq, synth, layers=36, k_format=0):
+    def __init__(self, kvq, synth, layers=36, k_format=0, klt=False):
         self.kvq = kvq
         import dataclasses
         w = dataclasses.replace(synth.WORKLOADS["ragged"], num_layers=layers)
         self.k_format = k_format
+        self.klt = klt
         self.tlb = TOKEN_LAYER_BYTES_BF16K if k_format else TOKEN_LAYER_BYTES
         self.w = w
         L, B, S = w.num_layers, w.batch, w.decode_steps
@@ -225,10 +228,13 @@ class Ragged:
         self.lens = synth.ragged_lengths(w)                          # [B] int32
         cap = self.lens + S
         self.page_table, self.num_pages = synth.build_page_table(w, cap)
-        self.shape = kvq.Shape(L, w.num_q_heads, w.num_kv_heads, k_format=k_format)
+        self.shape = kvq.Shape(L, w.num_q_heads, w.num_kv_heads, k_format=k_format, use_klt=klt)
         kc = torch.stack([synth.calibration_windows(w, l, dev)[0] for l in range(L)])
         vc = torch.stack([synth.calibration_windows(w, l, dev)[1] for l in range(L)])
-        self.calib = kvq.calibrate_smoothing(self.shape, kc, vc, exclude_pos0=True)
+        if klt:
+            self.calib = kvq.calibrate_klt(self.shape, kc, vc, exclude_pos0=True)
+        else:
+            self.calib = kvq.calibrate_smoothing(self.shape, kc, vc, exclude_pos0=True)
         del kc, vc
         self.cache = kvq.new_cache(self.shape, self.num_pages, dev)
         H, D = w.num_kv_heads, w.head_dim
@@ -271,7 +277,9 @@ class Ragged:
         self.out = torch.empty(L, B, w.num_q_heads, D, dtype=torch.bfloat16, device=dev)
         need = kvq.decode_workspace_bytes(self.shape, L, B, self.page_table.shape[1])
         self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-        self.launches_per_step = 2 + (1 if need else 0)
+        # append (+ KLT keys) and decode (+ KLT queries), plus a combine when split
+        part = kvq.decode_workspace_bytes(kvq.Shape(L, w.num_q_heads, w.num_kv_heads), L, B, self.page_table.shape[1])
+        self.launches_per_step = (4 if klt else 2) + (1 if part else 0)
         torch.cuda.synchronize()
         # bulk append of each layer's prefix (read bf16 K and V, write codes + scales)
         self.append_bytes = self.prefix_tokens * (2 * w.num_kv_heads * D * 2 + self.tlb)
@@ -564,7 +572,8 @@ def config_block(wl=None):
                         "lengths U[1024,8192], 16-token pages in shuffled order, 64 append+decode steps cycled",
             "batch": 64, "layers": layers,
             "kv_cache": ("mixed: bf16 keys, nvfp4 values" if bf16k else
-                         "nvfp4 (e2m1 codes, e4m3 per-16 scales, fp32 tensor scale)"),
+                         "nvfp4 (e2m1 codes, e4m3 per-16 scales, fp32 tensor scale)" +
+                         (", keys smoothed then rotated by a static per-head KLT" if wl is not None and wl.klt else "")),
             "l2": "inputs larger than L2 (about %.1f GB of cache read per step)" % (
                 (28.2 if bf16k else 12.4) * layers / 36),
             "parallelism": "replicas (independent sequences per GPU)"}
@@ -666,7 +675,7 @@ def main():
     if args.workload != "ragged":
         return other_workload(args, kvq, synth, rank, world)
     t_setup = time.time()
-    wl = Ragged(kvq, synth, args.layers, k_format=1 if args.k_format == "bf16" else 0)
+    wl = Ragged(kvq, synth, args.layers, k_format=1 if args.k_format == "bf16" else 0, klt=args.klt)
     sys.stderr.write(f"[bench] setup {time.time() - t_setup:.1f} s, {wl.num_pages} pages, "
                      f"cache {wl.cache.data.numel() / 1e9:.2f} GB\n")
     clock = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
@@ -678,7 +687,7 @@ def main():
     achieved = dec_bytes / (dec_avg_ms / 1e3) / 1e9
     peak, peak_kind = measured_peak()
     # the committed ncu counters are those of the packed-key kernel
-    traffic = ncu_traffic() if wl.k_format == 0 else None
+    traffic = ncu_traffic() if wl.k_format == 0 and not wl.klt else None
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_block(wl),

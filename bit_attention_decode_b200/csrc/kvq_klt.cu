@@ -216,6 +216,21 @@ __device__ __forceinline__ void klt_tile(const float* __restrict__ Yt, const flo
 
 constexpr size_t kKltTileSmem = (size_t)kD * kD * sizeof(float) + (size_t)kD * 64 * sizeof(float);
 
+// 8 consecutive elements (16-byte aligned for bf16, 32 for fp32) as fp32
+__device__ __forceinline__ void load8(const float* p, float* x) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float* x) {
+    const uint4 t = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        x[2 * j] = __uint_as_float(w[j] << 16);
+        x[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+}
+
 // Load U of (l, h) into shared memory.
 __device__ __forceinline__ void klt_load_basis(float* Us, const float* __restrict__ U) {
     for (int e = threadIdx.x; e < kD * kD / 4; e += blockDim.x)
@@ -300,7 +315,7 @@ klt_append_keys_kernel(const T* __restrict__ k, const int64_t* __restrict__ slot
     float* Yt = Us + kD * kD;
     float* rtab = Yt + kD * 64;
     int64_t* sslot = reinterpret_cast<int64_t*>(rtab + 128);
-    const int h = blockIdx.y, li = blockIdx.z, t0 = blockIdx.x * 64;
+    const int h = blockIdx.y, li = blockIdx.z;
     klt_load_basis(Us, U + ((size_t)li * Hkv + h) * kD * kD);
     const float g = __ldg(gk + li);
     const float enc = __frcp_rn(__fmul_rn(6.0f, g));
@@ -308,45 +323,58 @@ klt_append_keys_kernel(const T* __restrict__ k, const int64_t* __restrict__ slot
         // the append's reciprocal of every E4M3 scale code: 1/(val(c) g)
         const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), g);
         rtab[threadIdx.x] = (d == 0.0f) ? 0.0f : __frcp_rn(d);
-    } else if (threadIdx.x < 192) {
-        const int tt = threadIdx.x - 128;
-        sslot[tt] = (t0 + tt < num_tokens) ? __ldg(slots + t0 + tt) : -1;
     }
     const float* inv = inv_s + ((size_t)li * Hkv + h) * kD;
-    for (int e = threadIdx.x; e < 64 * kD; e += blockDim.x) {
-        const int r = e / kD, c = e % kD;
-        float y = 0.0f;
-        if (t0 + r < num_tokens)
-            y = __fmul_rn(load_elem(k + (((size_t)li * num_tokens + t0 + r) * Hkv + h) * kD + c), __ldg(inv + c));
-        Yt[c * 64 + r] = y;
-    }
-    __syncthreads();
-    const int tg = threadIdx.x >> 4, dg = threadIdx.x & 15;
-    float acc[4][8];
-    klt_tile(Yt, Us, tg, dg, acc);
     const int64_t num_slots = (int64_t)num_pages * kPage;
     uint8_t* layer_cache = cache + (size_t)li * layer_stride;
+    const int tg = threadIdx.x >> 4, dg = threadIdx.x & 15;
+    const int ntiles = (num_tokens + 63) / 64;
+    // the basis is loaded once; the CTA walks tiles of its (layer, head)
+    for (int tile_i = blockIdx.x; tile_i < ntiles; tile_i += gridDim.x) {
+        const int t0 = tile_i * 64;
+        __syncthreads();     // the previous tile's Yt and slots are consumed
+        if (threadIdx.x < 64) sslot[threadIdx.x] = (t0 + threadIdx.x < num_tokens) ? __ldg(slots + t0 + threadIdx.x) : -1;
+        // rows of 8 elements: 64 tokens x 16 groups; neighbouring lanes take
+        // neighbouring tokens, so the transposed stores hit distinct banks
+        for (int e = threadIdx.x; e < 64 * 16; e += blockDim.x) {
+            const int r = e & 63, c8 = (e >> 6) * 8;
+            float x[8];
+            if (t0 + r < num_tokens) {
+                load8(k + (((size_t)li * num_tokens + t0 + r) * Hkv + h) * kD + c8, x);
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-        float m = 0.0f;
+                for (int j = 0; j < 8; ++j) x[j] = __fmul_rn(x[j], __ldg(inv + c8 + j));
+            } else {
 #pragma unroll
-        for (int b = 0; b < 8; ++b) m = fmaxf(m, fabsf(acc[a][b]));
-        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));       // the other half of the 16-block
-        const uint32_t sf = e4m3_rn(__fmul_rn(m, enc));
-        const float r = rtab[sf & 0x7Fu];
-        uint32_t w = 0;
+                for (int j = 0; j < 8; ++j) x[j] = 0.0f;
+            }
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-            w |= klt_e2m1x2(__fmul_rn(acc[a][2 * j + 1], r), __fmul_rn(acc[a][2 * j], r)) << (8 * j);
-        const int tt = 4 * tg + a;
-        const int64_t slot = sslot[tt];
-        if (slot >= num_slots) {
-            if (dg == 0) set_status(status, KVQ_DEV_BAD_SLOT);
-        } else if (slot >= 0) {
-            uint8_t* tile = layer_cache + ((size_t)(slot >> 4) * Hkv + h) * kTile;
-            const int off = (int)(slot & 15);
-            *reinterpret_cast<uint32_t*>(tile + kKCodes + off * 64 + 4 * dg) = w;
-            if ((dg & 1) == 0) tile[kKScales + off * 8 + (dg >> 1)] = (uint8_t)sf;
+            for (int j = 0; j < 8; ++j) Yt[(c8 + j) * 64 + r] = x[j];
+        }
+        __syncthreads();
+        float acc[4][8];
+        klt_tile(Yt, Us, tg, dg, acc);
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            float m = 0.0f;
+#pragma unroll
+            for (int b = 0; b < 8; ++b) m = fmaxf(m, fabsf(acc[a][b]));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));       // the other half of the 16-block
+            const uint32_t sf = e4m3_rn(__fmul_rn(m, enc));
+            const float r = rtab[sf & 0x7Fu];
+            uint32_t w = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                w |= klt_e2m1x2(__fmul_rn(acc[a][2 * j + 1], r), __fmul_rn(acc[a][2 * j], r)) << (8 * j);
+            const int tt = 4 * tg + a;
+            const int64_t slot = sslot[tt];
+            if (slot >= num_slots) {
+                if (dg == 0) set_status(status, KVQ_DEV_BAD_SLOT);
+            } else if (slot >= 0) {
+                uint8_t* tile = layer_cache + ((size_t)(slot >> 4) * Hkv + h) * kTile;
+                const int off = (int)(slot & 15);
+                *reinterpret_cast<uint32_t*>(tile + kKCodes + off * 64 + 4 * dg) = w;
+                if ((dg & 1) == 0) tile[kKScales + off * 8 + (dg >> 1)] = (uint8_t)sf;
+            }
         }
     }
 }
@@ -359,7 +387,12 @@ kvq_status append_klt_keys(const kvq_shape& s, const kvq_calib& c, const kvq_cac
     const float* U = c.k_klt + (size_t)layer0 * H * kD * kD;
     const float* gk = c.k_gscale + layer0;
     uint8_t* base = cache.data + (size_t)layer0 * cache.layer_stride_bytes;
-    const dim3 grid((num_tokens + 63) / 64, H, nlayers);
+    // about two CTAs per SM in all; each walks tiles of its (layer, head)
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long ntiles = (num_tokens + 63) / 64;
+    const long per = (2L * sms + (long)H * nlayers - 1) / ((long)H * nlayers);
+    const dim3 grid((unsigned)(ntiles < per ? ntiles : (per < 1 ? 1 : per)), H, nlayers);
     cudaError_t e;
     if (dtype == KVQ_F32) {
         e = cudaFuncSetAttribute(klt_append_keys_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,

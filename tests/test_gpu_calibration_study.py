@@ -4,7 +4,7 @@
 "NVFP4 K only, native basis", "K: static per-channel smoothing, sqrt(absmax)
 from 4 C4 windows, position 0 excluded", "K: same smoothing, but sink token
 included in the absmax", "K: Hadamard-128 on head_dim", "K: Hadamard-128 +
-smoothing" and "NVFP4 V only" (bf16 keys), with observation 2 (calibrate without the sink).  The pages score
+smoothing", "K: static KLT + smoothing" and "NVFP4 V only" (bf16 keys), with observation 2 (calibrate without the sink).  The pages score
 these rows by perplexity of a trained model; with synthetic inputs the score
 here is the attention output error of one decode step: relative L2 norm of
 (NVFP4-cache attention - exact fp64 attention on the unquantised bf16 cache)
@@ -58,14 +58,17 @@ def _reference(w, kv, q):
 
 def _run(kvq, w, kv, q, mode):
     """Calibrate (mode: 'excl' sink left out, 'incl' sink in, 'native' no
-    smoothing, 'bf16k' bf16 keys with packed values), append every sequence,
-    decode one step; [nl][B][Hq][D] fp32."""
+    smoothing, 'bf16k' bf16 keys with packed values, 'klt' smoothing then the
+    static per-head KLT), append every sequence, decode one step;
+    [nl][B][Hq][D] fp32."""
     shape = kvq.Shape(len(LAYERS), w.num_q_heads, w.num_kv_heads, use_hadamard=w.hadamard,
-                      k_format=kvq.K_BF16 if mode == "bf16k" else kvq.K_NVFP4)
+                      k_format=kvq.K_BF16 if mode == "bf16k" else kvq.K_NVFP4, use_klt=(mode == "klt"))
     win = [synth.calibration_windows(w, l, "cuda") for l in LAYERS]
     kc = torch.stack([x[0] for x in win]).contiguous()
     vc = torch.stack([x[1] for x in win]).contiguous()
-    if mode in ("native", "bf16k"):
+    if mode == "klt":
+        calib = kvq.calibrate_klt(shape, kc, vc)
+    elif mode in ("native", "bf16k"):
         calib = kvq.calibrate_native(shape, kc, vc)
     else:
         calib = kvq.calibrate_smoothing(shape, kc, vc, exclude_pos0=(mode == "excl"))
@@ -103,6 +106,7 @@ def test_calibration_ablations(kvq, capsys):
             ("native basis (no smoothing)", base, "native"),
             ("Hadamard-128 + smoothing", _workload(hadamard=True), "excl"),
             ("Hadamard-128 alone", _workload(hadamard=True), "native"),
+            ("static KLT + smoothing", base, "klt"),
             ("bf16 keys, NVFP4 values", base, "bf16k")):
         rows.append((name,) + _errors(_run(kvq, w, kv, q, mode), ref))
     with capsys.disabled():
