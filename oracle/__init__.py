@@ -18,6 +18,13 @@ Parity status of each function (the pins live in ``tests/test_oracle_*.py``):
   dequantize_rows            pinned (products of the pinned format values)
   attention                  pinned (numpy/scipy softmax formula, one token,
                              equal keys, smoothing invariance)
+  klt_apply / klt_basis /    pinned (permutation, fp64 product bound, known
+  calibrate_klt              basis, diagonalised second moment)
+  quantize_query /           pinned (reduction to quantize_rows row by row,
+  query_rows_fp4             row absmax -> scale 448 and code 6, power-of-two
+                             invariance, error bound, zero row)
+  attention_x                pinned (equals attention on the fp64 transformed
+                             query; one visible key; equal scores)
 """
 
 from __future__ import annotations
@@ -74,9 +81,11 @@ def _load():
         lib.oracle_quantize_rows.argtypes = [P, i64, f32, P, P]
         lib.oracle_dequantize_rows.argtypes = [P, P, i64, f32, P]
         lib.oracle_attention.argtypes = [P, i32, i32, i32, i32, P, i32, P, P, i32, P]
+        lib.oracle_quantize_query_rows.argtypes = [P, i64, P, P, P]
+        lib.oracle_attention_x.argtypes = [P, i32, i32, i32, i32, P, P, i32, P]
         for name in ("oracle_e2m1_encode_n", "oracle_e4m3_encode_n", "oracle_transform_keys",
                      "oracle_calibrate", "oracle_klt_apply", "oracle_quantize_rows", "oracle_dequantize_rows",
-                     "oracle_attention"):
+                     "oracle_attention", "oracle_quantize_query_rows", "oracle_attention_x"):
             getattr(lib, name).restype = None
         _lib = lib
         return lib
@@ -267,6 +276,64 @@ def klt_tensor_scales(k_calib, v_calib, inv_s, U):
         gk[l] = np.float32(a) / np.float32(2688.0) if a > 0 else np.float32(1.0)
         gv[l] = np.float32(b) / np.float32(2688.0) if b > 0 else np.float32(1.0)
     return gk, gv
+
+
+# ---------------------------------------------------------------- FP4 queries
+def query_rows_fp4(q, s, hadamard: bool = False, U=None) -> np.ndarray:
+    """The query in the keys' basis, in fp32, as the FP4 Q.K product
+    quantises it: q [Tq][Hq][D], s [Hkv][D] -> [Tq][Hq][D] fp32.
+    Query head hq uses kv head hq // G.  Either the key transform with the
+    smoothing factor in place of its reciprocal (q * s, then the normalised
+    Hadamard-128 when hadamard; [P1] observation 2, [P5]), or, with a KLT
+    basis U [Hkv][D][D], q * s followed by U^T as one fp32 fused
+    multiply-add chain per output (klt_apply)."""
+    q = _f32(q)
+    Tq, Hq, D = q.shape
+    s = _f32(s)
+    G = Hq // s.shape[0]
+    rep = np.repeat(s, G, axis=0)
+    if U is None:
+        return transform_keys(q, rep, hadamard)
+    y = transform_keys(q, rep, False)
+    out = np.empty_like(y)
+    for hq in range(Hq):
+        out[:, hq] = klt_apply(y[:, hq], _f32(U)[hq // G])
+    return out
+
+
+def quantize_query(y):
+    """Transformed query rows y [..., D] fp32 -> (codes [..., D] one code per
+    byte, sf [..., D/16], g [...] fp32): NVFP4 with an FP32 scale per row,
+    g = amax(row) / 2688 (1 for a zero row), then the cache's block
+    quantiser (oracle_quantize_query_rows)."""
+    y, py = _c(_f32(y), np.float32)
+    n = y.size // HEAD_DIM
+    codes = np.empty(y.shape, np.uint8)
+    sf = np.empty(y.shape[:-1] + (HEAD_DIM // BLOCK,), np.uint8)
+    g = np.empty(y.shape[:-1], np.float32)
+    P = ctypes.c_void_p
+    _load().oracle_quantize_query_rows(py, n, codes.ctypes.data_as(P), sf.ctypes.data_as(P), g.ctypes.data_as(P))
+    return codes, sf, g
+
+
+def dequantize_query(codes, sf, g) -> np.ndarray:
+    """Exact fp64 value of quantised query rows: val(code) * val(sf) * g."""
+    codes = np.asarray(codes)
+    step = e4m3_value(np.repeat(np.asarray(sf), BLOCK, axis=-1)) * np.asarray(g, np.float64)[..., None]
+    return e2m1_value(codes) * step
+
+
+def attention_x(qx, q_start: int, kx, vx) -> np.ndarray:
+    """Causal GQA attention (as attention) of queries already in the keys'
+    basis: qx [Tq][Hq][D] fp64, kx, vx [T][Hkv][D] fp64 -> [Tq][Hq][D] fp64."""
+    qx, pq = _c(qx, np.float64)
+    kx, pk = _c(kx, np.float64)
+    vx, pv = _c(vx, np.float64)
+    Tq, Hq, D = qx.shape
+    T, Hkv, _ = kx.shape
+    out = np.empty((Tq, Hq, D), np.float64)
+    _load().oracle_attention_x(pq, Tq, int(q_start), Hq, Hkv, pk, pv, T, out.ctypes.data_as(ctypes.c_void_p))
+    return out
 
 
 # ---------------------------------------------------------------- composites

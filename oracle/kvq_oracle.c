@@ -2,7 +2,8 @@
  * kvq_oracle.c -- plain, slow CPU reference of the NVFP4 attention cache.
  *
  * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
- * bench's CPU-baseline leg load this file (through oracle/oracle.py).  The
+ * bench's CPU-baseline leg load this file (through the oracle package's
+ * ctypes loader).  The
  * CUDA library never links, calls or includes it, and it includes nothing of
  * the library: the two share no code.
  *
@@ -23,7 +24,7 @@
  * so no fused multiply-add and no reassociation).  Everything after
  * dequantisation -- the query transform, scores, softmax and P.V -- is fp64.
  *
- * Readings of points the pages leave open (each also listed in the design doc):
+ * Readings of points the pages leave open:
  *   - FP32 per-tensor scale: static, one per (layer, K|V), g = amax / (6*448)
  *     over the transformed calibration tensor including position 0.
  *   - E4M3 block scale: round-to-nearest-even with saturation at 448.
@@ -260,6 +261,32 @@ void oracle_quantize_rows(const float* y, int64_t n, float g, uint8_t* codes, ui
                            codes + (size_t)r * HD + b * BLK, sf + (size_t)r * (HD / BLK) + b);
 }
 
+/* Query rows quantised to NVFP4 for a Q.K product taken on FP4 tensor cores
+ * with block scales ([P1] setup: W4A4, activations in NVFP4; [P4] Problem
+ * bullet, sec. 1 and sec. D.1: absmax of each 16-entry block mapped to 6,
+ * an E4M3 scale per block, an FP32 scale above it).  The pages fix no
+ * static scale for queries, so the FP32 scale is taken online per row, the
+ * same way the static tensor scale is fitted: g = amax(row) / (6 * 448)
+ * (1 for an all-zero row); the blocks are then quantised exactly as the
+ * cache's (quantize_block above).
+ *   y:     [n][D] fp32, already transformed (smoothing, rotation)
+ *   codes: [n][D] one code per byte;  sf: [n][D/16];  g: [n] */
+void oracle_quantize_query_rows(const float* y, int64_t n, uint8_t* codes, uint8_t* sf, float* g)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n; ++r) {
+        const float* yr = y + (size_t)r * HD;
+        float a = 0.0f;
+        for (int c = 0; c < HD; ++c) if (fabsf(yr[c]) > a) a = fabsf(yr[c]);
+        const float gr = (a > 0.0f) ? a / 2688.0f : 1.0f;
+        const float six_g = 6.0f * gr;
+        const float enc = 1.0f / six_g;
+        for (int b = 0; b < HD / BLK; ++b)
+            quantize_block(yr + b * BLK, enc, gr, codes + (size_t)r * HD + b * BLK, sf + (size_t)r * (HD / BLK) + b);
+        g[r] = gr;
+    }
+}
+
 /* Dequantisation, exact in fp64: x = val(code) * val(sf) * g. */
 void oracle_dequantize_rows(const uint8_t* codes, const uint8_t* sf, int64_t n, float g, double* x)
 {
@@ -288,6 +315,33 @@ static void query_transform(const float* q, const float* s, int hadamard, double
     memcpy(out, tmp, sizeof tmp);
 }
 
+/* Exact softmax attention of one transformed query row qt (fp64) against the
+ * first n cached positions of kv head h: scores qt . k_j / sqrt(D), softmax
+ * over j < n, output sum_j p_j v_j.  kx, vx: [T][Hkv][D] fp64. */
+static void attend_row(const double* qt, int h, int n, int Hkv, const double* kx, const double* vx, double* o)
+{
+    const double scale = 1.0 / sqrt((double)HD);
+    for (int c = 0; c < HD; ++c) o[c] = 0.0;
+    if (n <= 0) return;
+    double* sc = (double*)malloc(sizeof(double) * (size_t)n);
+    double m = -INFINITY;
+    for (int j = 0; j < n; ++j) {
+        const double* kj = kx + ((size_t)j * Hkv + h) * HD;
+        double acc = 0.0;
+        for (int c = 0; c < HD; ++c) acc += qt[c] * kj[c];
+        sc[j] = acc * scale;
+        if (sc[j] > m) m = sc[j];
+    }
+    double l = 0.0;
+    for (int j = 0; j < n; ++j) { sc[j] = exp(sc[j] - m); l += sc[j]; }
+    for (int j = 0; j < n; ++j) {
+        const double* vj = vx + ((size_t)j * Hkv + h) * HD;
+        double p = sc[j] / l;
+        for (int c = 0; c < HD; ++c) o[c] += p * vj[c];
+    }
+    free(sc);
+}
+
 /* Causal GQA attention of Tq queries of one sequence and one layer against its
  * dequantised cache, exact softmax in fp64.
  *   q:    [Tq][Hq][D] fp32 (post-RoPE, untransformed)
@@ -302,7 +356,6 @@ void oracle_attention(const float* q, int Tq, int q_start, int Hq, int Hkv,
                       const double* kx, const double* vx, int T, double* out)
 {
     const int G = Hq / Hkv;
-    const double scale = 1.0 / sqrt((double)HD);
     #pragma omp parallel for collapse(2) schedule(dynamic)
     for (int i = 0; i < Tq; ++i)
         for (int hq = 0; hq < Hq; ++hq) {
@@ -311,25 +364,22 @@ void oracle_attention(const float* q, int Tq, int q_start, int Hq, int Hkv,
             if (n > T) n = T;
             double qt[HD];
             query_transform(q + ((size_t)i * Hq + hq) * HD, s + (size_t)h * HD, hadamard, qt);
-            double* o = out + ((size_t)i * Hq + hq) * HD;
-            for (int c = 0; c < HD; ++c) o[c] = 0.0;
-            if (n <= 0) continue;
-            double* sc = (double*)malloc(sizeof(double) * (size_t)n);
-            double m = -INFINITY;
-            for (int j = 0; j < n; ++j) {
-                const double* kj = kx + ((size_t)j * Hkv + h) * HD;
-                double acc = 0.0;
-                for (int c = 0; c < HD; ++c) acc += qt[c] * kj[c];
-                sc[j] = acc * scale;
-                if (sc[j] > m) m = sc[j];
-            }
-            double l = 0.0;
-            for (int j = 0; j < n; ++j) { sc[j] = exp(sc[j] - m); l += sc[j]; }
-            for (int j = 0; j < n; ++j) {
-                const double* vj = vx + ((size_t)j * Hkv + h) * HD;
-                double p = sc[j] / l;
-                for (int c = 0; c < HD; ++c) o[c] += p * vj[c];
-            }
-            free(sc);
+            attend_row(qt, h, n, Hkv, kx, vx, out + ((size_t)i * Hq + hq) * HD);
+        }
+}
+
+/* The same attention for queries given already in the keys' basis, in fp64
+ * (the dequantised NVFP4 queries of an FP4 Q.K product).
+ *   qx: [Tq][Hq][D] fp64; the rest as oracle_attention. */
+void oracle_attention_x(const double* qx, int Tq, int q_start, int Hq, int Hkv,
+                        const double* kx, const double* vx, int T, double* out)
+{
+    const int G = Hq / Hkv;
+    #pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int i = 0; i < Tq; ++i)
+        for (int hq = 0; hq < Hq; ++hq) {
+            int n = q_start + i + 1;
+            if (n > T) n = T;
+            attend_row(qx + ((size_t)i * Hq + hq) * HD, hq / G, n, Hkv, kx, vx, out + ((size_t)i * Hq + hq) * HD);
         }
 }
