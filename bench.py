@@ -51,6 +51,8 @@ def parse():
                     help="ragged workload with smoothing plus the static per-head KLT of the keys")
     ap.add_argument("--k-format", default="nvfp4", choices=["nvfp4", "bf16"],
                     help="key storage of the ragged workload: packed NVFP4, or bf16 keys with NVFP4 values")
+    ap.add_argument("--qk", default="fp16", choices=["fp16", "fp4"],
+                    help="Q.K of the prefill workload: fp16 (query hi + lo) or block-scaled FP4 (query quantised)")
     ap.add_argument("--source-sha", action="store_true",
                     help="print the hash of the decode kernel's sources (the key of the committed ncu counters) and exit")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -301,10 +303,11 @@ class Prefill:
     512-token chunk.  One step = append the chunk's K/V into every layer, then
     prefill attention of every layer (tcgen05)."""
 
-    def __init__(self, kvq, synth, layers=36, k_format=0):
+    def __init__(self, kvq, synth, layers=36, k_format=0, qk_fp4=False):
         import dataclasses
         w = dataclasses.replace(synth.WORKLOADS["prefill"], num_layers=layers)
         self.k_format = k_format
+        self.qk_fp4 = qk_fp4
         self.kvq, self.w = kvq, w
         L, B, P0, Tq = w.num_layers, w.batch, w.context, w.prefill_chunk
         self.L, self.B, self.P0, self.Tq = L, B, P0, Tq
@@ -350,7 +353,7 @@ class Prefill:
 
     def attend(self):
         self.kvq.prefill_attention(self.shape, self.calib, self.cache, self.q, self.q_start, self.pt, self.seq_lens,
-                                   out=self.out)
+                                   out=self.out, qk_fp4=self.qk_fp4)
 
 
 class Prefix:
@@ -592,26 +595,37 @@ def other_workload(args, kvq, synth, rank, world):
     warm = max(3, args.warmup)
     clock = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if args.workload == "prefill":
-        wl = Prefill(kvq, synth, args.layers, k_format=1 if args.k_format == "bf16" else 0)
+        wl = Prefill(kvq, synth, args.layers, k_format=1 if args.k_format == "bf16" else 0, qk_fp4=args.qk == "fp4")
         total, app_ms, pre_ms = time_two_kernels(wl.append, wl.attend, warm, args.steps, world)
         clocks = clock.stop() if clock else None
         total = max_over_ranks(total, world)
         tokens = world * wl.B * wl.Tq * args.steps
         pre = statistics.mean(pre_ms)
         achieved = wl.flops / (pre / 1e3) / 1e12
+        if wl.qk_fp4:
+            # half the algorithmic flops (Q.K) run on FP4 operands at 4x the bf16 rate
+            # (nominal 9 vs 2.25 PFLOP/s dense), half (P.V) on fp16 at the bf16 rate:
+            # the mix's peak is 2 / (1/4 + 1) = 1.6x the bf16 one
+            peak_tf, peak_tf_sus = 1.6 * peak_tf, 1.6 * peak_tf_sus
+            tf_kind += "; x1.6 for the FP4 Q.K / fp16 P.V mix (FP4 = 4x bf16, nominal ratio)"
         line = {"metric": "NVFP4-KV chunked causal prefill tokens/s; achieved tensor TFLOP/s vs B200 peak",
                 "value": tokens / (total / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": warm, "ms_per_step": total / args.steps, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "f16 mma (q split hi+lo), f32 accumulate", "data": "synthetic",
+                "vs_baseline": None, "data": "synthetic",
+                "dtype": ("nvfp4 Q.K (query quantised per row) + f16 P.V, f32 accumulate" if wl.qk_fp4
+                          else "f16 mma (q split hi+lo), f32 accumulate"),
                 "config": {"workload": f"chunked prefill: {wl.L} layers, batch 8, 8192 cached + 512-token causal "
                                        "chunk, 32 q / 8 kv heads, head_dim 128", "layers": wl.L,
-                           "kv_cache": "mixed: bf16 keys, nvfp4 values" if wl.k_format else "nvfp4"},
+                           "kv_cache": "mixed: bf16 keys, nvfp4 values" if wl.k_format else "nvfp4",
+                           "qk": "fp4" if wl.qk_fp4 else "fp16"},
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
                              "frac": achieved / peak_tf, "frac_of_sustained": achieved / peak_tf_sus,
                              "traffic": None, "peak_source": tf_kind,
-                             "kernel": "kvq prefill (tcgen05)", "alg_flops_per_launch": wl.flops,
-                             "note": "algorithmic flops count 4 per attended (query head, key, dim); the kernel "
-                                     "issues 1.5x that on the tensor pipe (query hi + lo)"},
+                             "kernel": "kvq prefill fp4 Q.K (tcgen05 mxf4nvf4 + f16)" if wl.qk_fp4
+                             else "kvq prefill (tcgen05)", "alg_flops_per_launch": wl.flops,
+                             "note": "algorithmic flops count 4 per attended (query head, key, dim)" +
+                                     ("" if wl.qk_fp4 else "; the kernel issues 1.5x that on the tensor pipe "
+                                                           "(query hi + lo)")},
                 "append_ms": statistics.mean(app_ms), "prefill_ms": pre, "gpu_launches": 2 * args.steps,
                 "clocks": clocks}
     else:

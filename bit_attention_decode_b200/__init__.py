@@ -79,6 +79,8 @@ _lib.kvq_prefill_workspace_bytes.argtypes = [_SHP, _I32, _I32, _I32]
 _lib.kvq_prefill_attention.restype = _I32
 _lib.kvq_prefill_attention.argtypes = [_SHP, _CAL, _CCH, _I32, _I32, _P, _I32, _I32, _P, _P, _I32, _P, _I32,
                                        _P, _I32, _P, ctypes.c_size_t, _P, _P]
+_lib.kvq_prefill_attention_fp4.restype = _I32
+_lib.kvq_prefill_attention_fp4.argtypes = _lib.kvq_prefill_attention.argtypes
 _lib.kvq_decode_attention_noalloc.restype = _I32
 _lib.kvq_decode_attention_noalloc.argtypes = [_SHP, _CAL, _CCH, _I32, _I32, _P, _I32, _P, _I32, _P, _I32, _P,
                                               _I32, _P, _P]
@@ -92,7 +94,8 @@ _lib.kvq_round_e4m3.argtypes = [_P, _P, ctypes.c_int64, _P]
 EXPORTED = ("kvq_page_bytes", "kvq_status_string", "kvq_version", "kvq_calibrate_smoothing", "kvq_calibrate_native",
             "kvq_calibrate_klt",
             "kvq_quantize_append", "kvq_decode_workspace_bytes", "kvq_decode_attention",
-            "kvq_prefill_workspace_bytes", "kvq_prefill_attention", "kvq_decode_attention_noalloc",
+            "kvq_prefill_workspace_bytes", "kvq_prefill_attention", "kvq_prefill_attention_fp4",
+            "kvq_decode_attention_noalloc",
             "kvq_round_e2m1", "kvq_round_e4m3", "kvq_selftest_wait_timeout")
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -307,8 +310,11 @@ def prefill_workspace_bytes(shape: Shape, nlayers: int, batch: int, q_len: int) 
 def prefill_attention(shape: Shape, calib: Calibration, cache: PagedCache, q: torch.Tensor,
                       q_start: torch.Tensor, page_table: torch.Tensor, seq_lens: torch.Tensor, layer0: int = 0,
                       out: Optional[torch.Tensor] = None, out_dtype=torch.bfloat16,
-                      workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None):
-    """q [nlayers][B][q_len][Hq][128] -> out of the same shape."""
+                      workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                      qk_fp4: bool = False):
+    """q [nlayers][B][q_len][Hq][128] -> out of the same shape.  qk_fp4:
+    Q.K on the block-scaled FP4 tensor cores, the query quantised to NVFP4
+    per row (kvq_prefill_attention_fp4)."""
     if q.dim() == 4:
         q = q[None]
     nl, B, Tq = q.shape[0], q.shape[1], q.shape[2]
@@ -320,11 +326,11 @@ def prefill_attention(shape: Shape, calib: Calibration, cache: PagedCache, q: to
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     _need_cuda(q, q_start, page_table, seq_lens, out, workspace, status)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(_lib.kvq_prefill_attention(ctypes.byref(shape.c()), ctypes.byref(calib.c()), ctypes.byref(cache.c()),
-                                      layer0, nl, q.data_ptr(), _dtype_code(q), Tq, q_start.data_ptr(),
-                                      page_table.data_ptr(), maxp, seq_lens.data_ptr(), B, out.data_ptr(),
-                                      _dtype_code(out), _ptr(workspace), ws_bytes, _ptr(status), _stream()),
-           "kvq_prefill_attention")
+    name = "kvq_prefill_attention_fp4" if qk_fp4 else "kvq_prefill_attention"
+    _check(getattr(_lib, name)(ctypes.byref(shape.c()), ctypes.byref(calib.c()), ctypes.byref(cache.c()),
+                               layer0, nl, q.data_ptr(), _dtype_code(q), Tq, q_start.data_ptr(),
+                               page_table.data_ptr(), maxp, seq_lens.data_ptr(), B, out.data_ptr(),
+                               _dtype_code(out), _ptr(workspace), ws_bytes, _ptr(status), _stream()), name)
     return out
 
 

@@ -189,15 +189,17 @@ size_t kvq_prefill_workspace_bytes(const kvq_shape* shape, int32_t nlayers, int3
     return kvq::prefill_workspace(*shape, nlayers, batch, q_len);
 }
 
-kvq_status kvq_prefill_attention(const kvq_shape* shape, const kvq_calib* calib, const kvq_cache* cache,
+static kvq_status prefill_common(const kvq_shape* shape, const kvq_calib* calib, const kvq_cache* cache,
                                  int32_t layer0, int32_t nlayers, const void* q, int32_t q_dtype, int32_t q_len,
                                  const int32_t* q_start, const int32_t* page_table, int32_t max_pages_per_seq,
                                  const int32_t* seq_lens, int32_t batch, void* out, int32_t out_dtype,
-                                 void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+                                 void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream, bool qk_fp4) {
     KVQ_TRY(check_shape(shape));
     KVQ_TRY(check_calib(shape, calib));
     KVQ_TRY(check_cache(shape, cache));
     KVQ_TRY(check_layers(shape, layer0, nlayers));
+    // FP4 Q.K needs packed keys
+    if (qk_fp4 && shape->k_format != KVQ_K_NVFP4) return KVQ_EINVAL;
     if (batch < 1 || q_len < 1 || max_pages_per_seq < 1 || (long)batch * shape->num_kv_heads > 65535)
         return KVQ_EINVAL;
     if (!good_dtype(q_dtype) || !good_dtype(out_dtype)) return KVQ_EINVAL;
@@ -208,7 +210,28 @@ kvq_status kvq_prefill_attention(const kvq_shape* shape, const kvq_calib* calib,
     KVQ_TRY(check_device());
     return kvq::prefill(*shape, *calib, *cache, layer0, nlayers, q, q_dtype, q_len, q_start, page_table,
                         max_pages_per_seq, seq_lens, batch, out, out_dtype, workspace, workspace_bytes,
-                        dev_status, (cudaStream_t)stream);
+                        dev_status, (cudaStream_t)stream, qk_fp4);
+}
+
+
+kvq_status kvq_prefill_attention(const kvq_shape* shape, const kvq_calib* calib, const kvq_cache* cache,
+                                 int32_t layer0, int32_t nlayers, const void* q, int32_t q_dtype, int32_t q_len,
+                                 const int32_t* q_start, const int32_t* page_table, int32_t max_pages_per_seq,
+                                 const int32_t* seq_lens, int32_t batch, void* out, int32_t out_dtype,
+                                 void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+    return prefill_common(shape, calib, cache, layer0, nlayers, q, q_dtype, q_len, q_start, page_table,
+                          max_pages_per_seq, seq_lens, batch, out, out_dtype, workspace, workspace_bytes, dev_status,
+                          stream, false);
+}
+
+kvq_status kvq_prefill_attention_fp4(const kvq_shape* shape, const kvq_calib* calib, const kvq_cache* cache,
+                                     int32_t layer0, int32_t nlayers, const void* q, int32_t q_dtype, int32_t q_len,
+                                     const int32_t* q_start, const int32_t* page_table, int32_t max_pages_per_seq,
+                                     const int32_t* seq_lens, int32_t batch, void* out, int32_t out_dtype,
+                                     void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+    return prefill_common(shape, calib, cache, layer0, nlayers, q, q_dtype, q_len, q_start, page_table,
+                          max_pages_per_seq, seq_lens, batch, out, out_dtype, workspace, workspace_bytes, dev_status,
+                          stream, true);
 }
 
 kvq_status kvq_selftest_wait_timeout(int32_t* dev_status, int64_t limit_ns, void* stream) {

@@ -34,5 +34,7 @@ cudaError_t launch_decode_tc(const AttnArgs& a, int nlayers, bool q_bf16, bool o
 size_t decode_tc_smem(int Hkv, bool kbf16);
 // tensor-core (tcgen05) chunked causal prefill (kvq_prefill_tc.cu)
 cudaError_t launch_prefill_tc(const AttnArgs& a, int nlayers, bool q_bf16, bool out_bf16, cudaStream_t st);
+// the same with Q.K on block-scaled FP4 operands (kvq_prefill_fp4.cu)
+cudaError_t launch_prefill_fp4(const AttnArgs& a, int nlayers, bool q_bf16, bool out_bf16, cudaStream_t st);
 
 }  // namespace kvq

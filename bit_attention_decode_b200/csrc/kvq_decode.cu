@@ -159,7 +159,7 @@ size_t prefill_workspace(const kvq_shape& s, int nlayers, int batch, int q_len) 
 kvq_status prefill(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cache, int layer0, int nlayers,
                    const void* q, int q_dtype, int q_len, const int32_t* q_start, const int32_t* page_table,
                    int max_pages, const int32_t* seq_lens, int batch, void* out, int out_dtype, void* ws, size_t,
-                   int32_t* status, cudaStream_t st) {
+                   int32_t* status, cudaStream_t st, bool qk_fp4) {
     AttnArgs a = make_args(s, c, cache, layer0, q, page_table, max_pages, seq_lens, batch, out, status);
     a.q_len = q_len;
     a.q_start = q_start;
@@ -173,7 +173,8 @@ kvq_status prefill(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cach
         a.qpre = 1;
         qb = false;
     }
-    if (launch_prefill_tc(a, nlayers, qb, ob, st) != cudaSuccess) return KVQ_ECUDA;
+    const cudaError_t e = qk_fp4 ? launch_prefill_fp4(a, nlayers, qb, ob, st) : launch_prefill_tc(a, nlayers, qb, ob, st);
+    if (e != cudaSuccess) return KVQ_ECUDA;
     return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ECUDA;
 }
 

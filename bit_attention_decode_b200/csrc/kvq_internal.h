@@ -39,7 +39,7 @@ size_t prefill_workspace(const kvq_shape& s, int nlayers, int batch, int q_len);
 kvq_status prefill(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cache, int layer0, int nlayers,
                    const void* q, int q_dtype, int q_len, const int32_t* q_start, const int32_t* page_table,
                    int max_pages, const int32_t* seq_lens, int batch, void* out, int out_dtype, void* ws,
-                   size_t ws_bytes, int32_t* status, cudaStream_t st);
+                   size_t ws_bytes, int32_t* status, cudaStream_t st, bool qk_fp4 = false);
 kvq_status round_e2m1(const float* x, uint8_t* out, int64_t n, cudaStream_t st);
 kvq_status selftest_wait_timeout(int32_t* status, long long limit_ns, cudaStream_t st);
 kvq_status round_e4m3(const float* x, uint8_t* out, int64_t n, cudaStream_t st);

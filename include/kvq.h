@@ -282,6 +282,33 @@ kvq_status kvq_prefill_attention(const kvq_shape* shape, const kvq_calib* calib,
                                  int32_t* dev_status, void* stream);
 
 /*
+ * kvq_prefill_attention_fp4 -- kvq_prefill_attention with Q.K taken on the
+ * block-scaled FP4 tensor cores ("NVFP4 attention cache on W4A4 Qwen3-8B"
+ * (rstation.ai), setup: W4A4, activations in NVFP4; "OSFP4" (paperlayer.ai
+ * summary), Problem bullet, sec. 1 and sec. D.1).  The packed keys are the
+ * MMA's operand as stored (E2M1 codes with their E4M3 block scales); the
+ * query, after the same smoothing / rotation / KLT as kvq_prefill_attention,
+ * is quantised to NVFP4 per row: g_q = amax(row) / 2688 (1 for a zero row),
+ * then per 16-block sf = E4M3(absmax * (1 / (6 g_q))), d = val(sf) * g_q,
+ * codes E2M1(x / d) -- the cache's quantiser with the row's own FP32 scale,
+ * each step one IEEE fp32 rounding.  Scores are then
+ * (sum over blocks of sf_q sf_k (codes . codes)) * g_q * g_K / sqrt(128);
+ * softmax and P.V are those of kvq_prefill_attention.
+ *
+ * The result differs from kvq_prefill_attention's by the query's
+ * quantisation error (4-bit codes), which is far above the fp32 rounding of
+ * the unquantised query: compare it with attention on the dequantised query.
+ * Same arguments, workspace, results and errors as kvq_prefill_attention;
+ * a KVQ_K_BF16 (mixed) cache has no FP4 keys and returns KVQ_EINVAL.
+ */
+kvq_status kvq_prefill_attention_fp4(const kvq_shape* shape, const kvq_calib* calib, const kvq_cache* cache,
+                                     int32_t layer0, int32_t nlayers, const void* q, int32_t q_dtype,
+                                     int32_t q_len, const int32_t* q_start, const int32_t* page_table,
+                                     int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                                     void* out, int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                                     int32_t* dev_status, void* stream);
+
+/*
  * kvq_decode_attention_noalloc -- kvq_decode_attention without a workspace
  * argument, for callers that cannot allocate device memory (code running
  * inside a host runtime that owns the device-memory budget and forbids

@@ -211,3 +211,18 @@ def oracle_attend(p: Problem, li: int, b: int, q_rows: np.ndarray, q_start: int,
         qt = np.einsum("thc,hci->thi", qs, np.repeat(U, G, axis=0))
         return oracle.attention(qt.astype(np.float32), q_start, np.ones_like(s[li]), kx, vx, False)
     return oracle.attention(q_rows, q_start, s[li], kx, vx, p.w.hadamard)
+
+
+def oracle_attend_fp4q(p: Problem, li: int, b: int, q_rows: np.ndarray, q_start: int, n: int, cal):
+    """Oracle of the FP4 Q.K prefill: the query in the keys' basis (smoothing,
+    rotation or the device's KLT basis), quantised to NVFP4 per row by the
+    oracle, dequantised exactly, then attended in fp64 against the
+    dequantised cache."""
+    s, inv, gk, gv = cal
+    qz = oracle_sequence(p, li, b, n, cal)
+    kx = oracle.dequantize_rows(qz["kc"], qz["ksf"], gk[li])
+    vx = oracle.dequantize_rows(qz["vc"], qz["vsf"], gv[li])
+    U = p.calib.k_klt[li].cpu().numpy() if getattr(p, "klt", False) else None
+    y = oracle.query_rows_fp4(q_rows, s[li], hadamard=bool(p.w.hadamard) and U is None, U=U)
+    qx = oracle.dequantize_query(*oracle.quantize_query(y))
+    return oracle.attention_x(qx, q_start, kx, vx)

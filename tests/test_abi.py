@@ -131,3 +131,19 @@ def test_mixed_cache_key_format_validation(kvq_lib):
         ctypes.byref(bf.c()), ctypes.byref(kvq._Calib(16, 16, 16, 16)), ctypes.byref(kvq._Cache(4096, 8 * 2304 * 4, 4)),
         0, 1, 256, 1, 8, 512, 768, 64, 1024, 2, 2048, 1, None, 0, None, None)
     assert st == kvq.KVQ_EINVAL
+
+
+def test_fp4_prefill_needs_packed_keys(kvq_lib):
+    # FP4 Q.K reads the keys' E2M1 codes: a bf16-key (mixed) cache is refused
+    kvq = kvq_lib
+    bf = kvq.Shape(2, 32, 8, k_format=kvq.K_BF16)
+    args = (ctypes.byref(kvq._Calib(16, 16, 16, 16)), ctypes.byref(kvq._Cache(4096, 8 * 5248 * 4, 4)),
+            0, 1, 256, 1, 8, 512, 768, 64, 1024, 2, 2048, 1, None, 0, None, None)
+    assert kvq._lib.kvq_prefill_attention_fp4(ctypes.byref(bf.c()), *args) == kvq.KVQ_EINVAL
+    # the same arguments pass kvq_prefill_attention's checks (and stop at the device check here)
+    assert kvq._lib.kvq_prefill_attention(ctypes.byref(bf.c()), *args) != kvq.KVQ_EINVAL
+    # packed keys pass the FP4 call's checks too
+    pk = kvq.Shape(2, 32, 8)
+    args = (ctypes.byref(kvq._Calib(16, 16, 16, 16)), ctypes.byref(kvq._Cache(4096, 8 * 2304 * 4, 4)),
+            0, 1, 256, 1, 8, 512, 768, 64, 1024, 2, 2048, 1, None, 0, None, None)
+    assert kvq._lib.kvq_prefill_attention_fp4(ctypes.byref(pk.c()), *args) != kvq.KVQ_EINVAL
