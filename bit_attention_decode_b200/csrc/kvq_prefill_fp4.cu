@@ -19,11 +19,11 @@
 //
 // One CTA: one layer, one sequence, one kv head, two tiles of 32 query
 // tokens x G heads (128 MMA rows each).  Per 64-token key block:
-//   dequant warps (3): the 4 packed page tiles are bulk-copied into a staging
-//     ring; key codes are copied into the unswizzled K-major FP4 layout the
-//     MMA reads (8-row x 16-byte core matrices) and key scales into the
-//     128-row scale layout (row r's 4 scales of a 64-element K step at byte
-//     (r % 32) * 16 + (r / 32) * 4); values are dequantised to fp16.
+//   copy warp: bulk-copies the 4 packed page tiles into a staging ring.
+//   dequant warps (2): key codes are copied into the unswizzled K-major FP4
+//     layout the MMA reads (8-row x 16-byte core matrices) and key scales
+//     into the 128-row scale layout (row r's 4 scales of a 64-element K step
+//     at byte (r % 32) * 16 + (r / 32) * 4); values are dequantised to fp16.
 //   MMA warp: tcgen05.cp of the key scales into TMEM, then per tile two
 //     block-scaled MMAs (M=128, N=64, K=64) into the tile's score columns;
 //     O += P V (M=128, N=128, K=16 steps) with P read from TMEM.
@@ -51,6 +51,7 @@ constexpr int kStageN = 6;          // packed-page staging stages
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 256, kColP = 384, kColSFA = 448, kColSFB = 464;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr int kPidCap = 1024;       // page ids held in shared memory (keys up to 16384 tokens)
 
 // shared memory map (offsets from a 1024-aligned base)
 constexpr int kVBytes = kBlkTok * kD * 2;         // 16 KB fp16 value tile (128B-swizzled)
@@ -70,9 +71,13 @@ constexpr int kSmemBytes = kOffStage + kStageN * kStageBytes;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
 static_assert(2 * (kSmemAlloc + 1024) > 228 * 1024 && kSmemAlloc <= 227 * 1024, "one CTA per SM");
 
-enum { kWarpsSoftmax = 4 * kTiles, kWarpsDequant = 3 };
-constexpr int kDequantWarp0 = kWarpsSoftmax;                   // warps 8..10
-constexpr int kMmaWarp = kWarpsSoftmax + kWarpsDequant;        // warp 11
+// warps 8, 9 re-lay the keys and dequantise the values; warp 10 issues the
+// bulk copies (a copy takes the issuing thread hundreds of cycles, which a
+// warp that also dequantises would put on the critical path every block)
+enum { kWarpsSoftmax = 4 * kTiles, kWarpsDequant = 2 };
+constexpr int kDequantWarp0 = kWarpsSoftmax;                   // warps 8, 9
+constexpr int kCopyWarp = kDequantWarp0 + kWarpsDequant;       // warp 10
+constexpr int kMmaWarp = kCopyWarp + 1;                        // warp 11
 constexpr int kThreads = 32 * (kMmaWarp + 1);
 
 // byte offset of 16-byte chunk c (32 FP4 elements along K) of row `row` in an
@@ -87,9 +92,9 @@ __device__ __forceinline__ uint32_t sf_off(int row) { return (uint32_t)((row & 3
 struct Fp4Bars {
     uint64_t q_ready;                 // query tiles and scales written (count 8)
     uint64_t stage_full[kStageN];     // packed pages landed (tx bytes)
-    uint64_t stage_empty[kStageN];    // dequant warps read the stage (count 3)
-    uint64_t k_full[2];               // K tile + scales of block j written (count 3)
-    uint64_t v_full[2];               // V tile j written (count 3)
+    uint64_t stage_empty[kStageN];    // dequant warps read the stage (count 2)
+    uint64_t k_full[2];               // K tile + scales of block j written (count 2)
+    uint64_t v_full[2];               // V tile j written (count 2)
     uint64_t k_free[2];               // Q.K(j) of both tiles done (commit)
     uint64_t s_full[kTiles];          // Q.K(tile, j) done (commit)
     uint64_t s_free[kTiles];          // scores of (tile, j) loaded (count 4)
@@ -107,6 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_fp4_kernel(AttnArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ Fp4Bars bars;
+    __shared__ int32_t s_pid[kPidCap];   // the sequence's page ids, read once for every copy
 
     const int pair = blockIdx.x, b = blockIdx.y / a.Hkv, h = blockIdx.y % a.Hkv, li = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -152,6 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_fp4_kernel(AttnArgs a) {
     for (int i = threadIdx.x; i < npg; i += blockDim.x) {
         const int pg = __ldg(pt + i);
         badp |= (pg < 0 || pg >= a.num_pages);
+        if (i < kPidCap) s_pid[i] = pg;
     }
     badp = __syncthreads_or(badp);
     if (threadIdx.x == 0) {
@@ -275,19 +282,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_fp4_kernel(AttnArgs a) {
                 m8[7] = m21[21];
                 float bm = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], fmax3(m8[5], m8[6], m8[7])));
                 bm *= isig;
-                // P(j - 1) read and O(j - 1) complete before P(j) is stored or O rescaled
-                if (j > 0) {
-                    if (!mbar_wait_warp(&bars.pv_done[t][(j - 1) & 1], ((j - 1) >> 1) & 1)) {
-                        atomicOr(&bars.flags, 1);
-                        break;
+                // P.V(j - 1) must be done before O is rescaled (rare) or P(j) is
+                // stored over P(j - 1): waited for as late as possible
+                bool pv_ok = j == 0;
+                auto wait_pv = [&]() {
+                    if (!pv_ok) {
+                        pv_ok = mbar_wait_warp(&bars.pv_done[t][(j - 1) & 1], ((j - 1) >> 1) & 1);
+                        tc_fence_after();
                     }
-                    tc_fence_after();
-                }
+                    return pv_ok;
+                };
                 const bool grow = bm > m_run + kRescaleThreshold || (m_run == -INFINITY && bm > -INFINITY);
                 if (__any_sync(0xFFFFFFFFu, grow)) {
                     const float mn = grow ? bm : m_run;
                     const float al = (m_run == -INFINITY) ? 0.0f : ex2(m_run - mn);
                     if (j > 0) {
+                        if (!wait_pv()) { atomicOr(&bars.flags, 1); break; }
 #pragma unroll 1
                         for (int cc = 0; cc < 4; ++cc) {
                             float o[32];
@@ -303,59 +313,55 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_fp4_kernel(AttnArgs a) {
                 const float2 sc2 = make_float2(isig, isig), nm2 = make_float2(-m_run, -m_run);
                 float2 lsum[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
                                   make_float2(0.0f, 0.0f)};
+                uint32_t pk[32];
 #pragma unroll
-                for (int hv = 0; hv < 2; ++hv) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        const float2 x = ffma2(make_float2(s[32 * hv + 2 * c], s[32 * hv + 2 * c + 1]), sc2, nm2);
-                        float2 pp;
-                        if ((c & 3) == 3) {
-                            pp.x = poly_exp2(x.x);
-                            pp.y = poly_exp2(x.y);
-                        } else {
-                            pp.x = ex2(x.x);
-                            pp.y = ex2(x.y);
-                        }
-                        lsum[c & 3] = fadd2(lsum[c & 3], pp);
-                        pk[c] = h2(pp.x, pp.y);
-                    }
-                    tmem_st16u(tP(t) + 16 * hv + lane_addr, pk);
+                for (int c = 0; c < 32; ++c) {
+                    const float2 x = ffma2(make_float2(s[2 * c], s[2 * c + 1]), sc2, nm2);
+                    float2 pp;
+                    pp.x = ex2(x.x);
+                    pp.y = ex2(x.y);
+                    lsum[c & 3] = fadd2(lsum[c & 3], pp);
+                    pk[c] = h2(pp.x, pp.y);
                 }
+                if (!wait_pv()) { atomicOr(&bars.flags, 1); break; }
+                tmem_st16u(tP(t) + lane_addr, pk);
+                tmem_st16u(tP(t) + 16 + lane_addr, pk + 16);
                 const float2 l2 = fadd2(fadd2(lsum[0], lsum[1]), fadd2(lsum[2], lsum[3]));
                 l_run += l2.x + l2.y;
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars.p_full[t]);
             }
+        } else if (warp == kCopyWarp) {
+            // ------------------------------------------------------ copy warp
+            // block j's 4 page tiles into stage j % kStageN, once the dequant
+            // warps have read block j - kStageN out of it
+            if (lane == 0) {
+                int issued = 0;
+                for (; issued < nb; ++issued) {
+                    const int st = issued % kStageN;
+                    if (issued >= kStageN &&
+                        !mbar_wait(&bars.stage_empty[st], ((issued - kStageN) / kStageN) & 1)) {
+                        atomicOr(&bars.flags, 1);
+                        break;
+                    }
+                    const int p_lo = issued * 4, n_p = min(npg, p_lo + 4) - p_lo;
+                    mbar_arrive_expect_tx(&bars.stage_full[st], (uint32_t)n_p * kTile);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        if (k < n_p) {
+                            const int p = p_lo + k;
+                            const int pg = p < kPidCap ? s_pid[p] : __ldg(pt + p);
+                            bulk_g2s(smem + kOffStage + st * kStageBytes + k * kTile,
+                                     layer_base + ((size_t)pg * a.Hkv + h) * kTile, kTile, &bars.stage_full[st]);
+                        }
+                }
+                bars.issued = issued;
+            }
         } else if (warp < kMmaWarp) {
             // ------------------------------------------------------ dequant warps
-            const int dt = threadIdx.x - 32 * kDequantWarp0;   // 0..95
-            const bool issuer = (dt == 32 * (kWarpsDequant - 1));
-            int issued = 0;
-            int pgn[4] = {0, 0, 0, 0};
-            auto fetch_ids = [&](int j) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) pgn[k] = (j * 4 + k < npg) ? __ldg(pt + j * 4 + k) : 0;
-            };
-            auto issue = [&](int j) {
-                const int st = j % kStageN;
-                const int p_lo = j * 4, n_p = min(npg, p_lo + 4) - p_lo;
-                int pg[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) pg[k] = pgn[k];
-                fetch_ids(j + 1);
-                mbar_arrive_expect_tx(&bars.stage_full[st], (uint32_t)n_p * kTile);
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    if (k < n_p)
-                        bulk_g2s(smem + kOffStage + st * kStageBytes + k * kTile,
-                                 layer_base + ((size_t)pg[k] * a.Hkv + h) * kTile, kTile, &bars.stage_full[st]);
-            };
-            if (issuer) fetch_ids(0);
-            if (issuer)
-                for (; issued < kStageN && issued < nb; ++issued) issue(issued);
-            // items (token, half of head_dim): 128 per block over 96 threads
+            const int dt = threadIdx.x - 32 * kDequantWarp0;   // 0..63
+            // items (token, half of head_dim): 128 per block over 64 threads
             constexpr int kItems = 2 * kBlkTok, kDqThreads = 32 * kWarpsDequant;
             constexpr int kPer = (kItems + kDqThreads - 1) / kDqThreads;
             struct Staged {
@@ -386,16 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_fp4_kernel(AttnArgs a) {
                 }
                 __syncwarp();
                 if ((dt & 31) == 0) mbar_arrive(&bars.stage_empty[st]);
-                int issue_ok = 1;
-                if (issuer && issued < nb) {
-                    if (!mbar_wait(&bars.stage_empty[st], (j / kStageN) & 1)) {
-                        issue_ok = 0;
-                    } else {
-                        issue(issued);
-                        ++issued;
-                    }
-                }
-                return __shfl_sync(0xFFFFFFFFu, issue_ok, 0) != 0;
+                return true;
             };
             // key codes and scales of block j into buffer j & 1, free once
             // both tiles' Q.K(j - 2) are done; tokens past the sequence are
@@ -463,35 +460,43 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_fp4_kernel(AttnArgs a) {
                 cur = nxt;
             }
             if (!dq_ok) atomicOr(&bars.flags, 1);
-            if (issuer) bars.issued = issued;
         } else if (lane == 0) {
             // ------------------------------------------------------ MMA issuer
             constexpr uint32_t qk = fp4_idesc(kRows, kBlkTok);
             const uint32_t pv = f16_idesc(kRows, kD, true);
-            uint64_t qd[kTiles][2], kd[2][2], sfa[kTiles][2], sfb[2][2], vd[2];
+            // Descriptors are built once per operand tile; a tile, buffer or K
+            // step only moves the 14-bit start-address field (16-byte units)
+            // by a constant, which never carries out of the field for
+            // shared-memory addresses.
+            const uint64_t qd0 = nosw_desc(smem_u32(smem + kOffQ), 128, 512);
+            const uint64_t kd0 = nosw_desc(smem_u32(smem + kOffK), 128, 512);
+            const uint64_t sfa0 = nosw_desc(smem_u32(smem + kOffSFA), 128, 128);
+            const uint64_t sfb0 = nosw_desc(smem_u32(smem + kOffSFB), 128, 128);
+            const uint64_t vd0 = sw128_desc(smem_u32(smem + kOffV), kBlkTok * 128, 1024);
+            auto qd = [&](int t, int s) { return qd0 + (uint64_t)((t * kQBytes + 256 * s) >> 4); };
+            auto kd = [&](int u, int s) { return kd0 + (uint64_t)((u * kKBytes + 256 * s) >> 4); };
+            auto sfa = [&](int t, int s) { return sfa0 + (uint64_t)(((2 * t + s) * kSFBytes) >> 4); };
+            auto sfb = [&](int u, int s) { return sfb0 + (uint64_t)(((2 * u + s) * kSFBytes) >> 4); };
+            auto vd = [&](int u) { return vd0 + (uint64_t)((u * kVBytes) >> 4); };
+            // O(t) += P(t, jp) V(jp); V buffer jp & 1 is waited for by tile 0
+            auto issue_pv = [&](int t, int jp) -> bool {
+                const int pb = jp & 1;
+                if (t == 0 && !mbar_wait(&bars.v_full[pb], (jp >> 1) & 1)) return false;
+                if (!mbar_wait(&bars.p_full[t], jp & 1)) return false;
+                tc_fence_after();
 #pragma unroll
-            for (int t = 0; t < kTiles; ++t)
-#pragma unroll
-                for (int s = 0; s < 2; ++s) {
-                    qd[t][s] = nosw_desc(smem_u32(smem + kOffQ + t * kQBytes + 256 * s), 128, 512);
-                    sfa[t][s] = nosw_desc(smem_u32(smem + kOffSFA + (2 * t + s) * kSFBytes), 128, 128);
-                }
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-#pragma unroll
-                for (int s = 0; s < 2; ++s) {
-                    kd[u][s] = nosw_desc(smem_u32(smem + kOffK + u * kKBytes + 256 * s), 128, 512);
-                    sfb[u][s] = nosw_desc(smem_u32(smem + kOffSFB + (2 * u + s) * kSFBytes), 128, 128);
-                }
-                vd[u] = sw128_desc(smem_u32(smem + kOffV + u * kVBytes), kBlkTok * 128, 1024);
-            }
+                for (int s = 0; s < 4; ++s)
+                    mma_f16_ta(tO(t), tP(t) + 8 * s, vd(pb) + (uint64_t)((s * 2048) >> 4), pv, (jp | s) ? 1u : 0u);
+                mma_commit(&bars.pv_done[t][pb]);
+                return true;
+            };
             bool ok = mbar_wait(&bars.q_ready, 0);
             if (ok) {
                 tc_fence_after();
 #pragma unroll
                 for (int t = 0; t < kTiles; ++t)
 #pragma unroll
-                    for (int s = 0; s < 2; ++s) tmem_cp_scales(tmem + kColSFA + 8 * t + 4 * s, sfa[t][s]);
+                    for (int s = 0; s < 2; ++s) tmem_cp_scales(tmem + kColSFA + 8 * t + 4 * s, sfa(t, s));
             }
             for (int j = 0; ok && j <= nb; ++j) {
                 if (j < nb) {
@@ -499,35 +504,27 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_fp4_kernel(AttnArgs a) {
                     if (!mbar_wait(&bars.k_full[buf], (j >> 1) & 1)) { ok = false; break; }
                     tc_fence_after();
 #pragma unroll
-                    for (int s = 0; s < 2; ++s) tmem_cp_scales(tmem + kColSFB + 8 * buf + 4 * s, sfb[buf][s]);
-#pragma unroll
+                    for (int s = 0; s < 2; ++s) tmem_cp_scales(tmem + kColSFB + 8 * buf + 4 * s, sfb(buf, s));
+                    // tile by tile: Q.K(j) then P.V(j - 1) of tile A, then of tile
+                    // B, so that one tile's P.V is not held behind the other
+                    // tile's scores
                     for (int t = 0; t < kTiles; ++t) {
                         // the tile's scores of block j - 1 must be in registers
                         if (j >= 1 && !mbar_wait(&bars.s_free[t], (j - 1) & 1)) { ok = false; break; }
                         tc_fence_after();
 #pragma unroll
                         for (int s = 0; s < 2; ++s)
-                            mma_fp4(tS(t), qd[t][s], kd[buf][s], qk, tmem + kColSFA + 8 * t + 4 * s,
+                            mma_fp4(tS(t), qd(t, s), kd(buf, s), qk, tmem + kColSFA + 8 * t + 4 * s,
                                     tmem + kColSFB + 8 * buf + 4 * s, (uint32_t)s);
                         mma_commit(&bars.s_full[t]);
+                        if (t == kTiles - 1) mma_commit(&bars.k_free[buf]);
+                        if (j >= 1 && !issue_pv(t, j - 1)) { ok = false; break; }
                     }
                     if (!ok) break;
-                    mma_commit(&bars.k_free[buf]);
-                }
-                if (j >= 1) {
-                    const int jp = j - 1, buf = jp & 1;
-                    const uint64_t vb = vd[buf];
-                    if (!mbar_wait(&bars.v_full[buf], (jp >> 1) & 1)) { ok = false; break; }
-#pragma unroll
-                    for (int t = 0; t < kTiles; ++t) {
-                        if (!mbar_wait(&bars.p_full[t], jp & 1)) { ok = false; break; }
-                        tc_fence_after();
-#pragma unroll
-                        for (int s = 0; s < 4; ++s)
-                            mma_f16_ta(tO(t), tP(t) + 8 * s, vb + (uint64_t)((s * 2048) >> 4), pv, (jp | s) ? 1u : 0u);
-                        mma_commit(&bars.pv_done[t][buf]);
-                    }
-                    if (!ok) break;
+                } else {
+                    // after the last block: its P.V
+                    for (int t = 0; t < kTiles; ++t)
+                        if (!issue_pv(t, j - 1)) { ok = false; break; }
                 }
             }
             if (!ok) atomicOr(&bars.flags, 1);

@@ -47,6 +47,7 @@ constexpr int kBlkTok = 64;         // key tokens per block (4 pages)
 constexpr int kStageN = 3;          // packed-page staging stages
 constexpr uint32_t kTmemCols = 512; // O_A, O_B [0,256), S_A[2] [256,384), S_B[2] [384,512)
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr int kPidCap = 1024;       // page ids held in shared memory (keys up to 16384 tokens)
 
 // shared memory map (offsets from a 1024-aligned base)
 constexpr int kQBytes = kRows * kD * 2;           // 32 KB per fp16 query tile part (hi or lo)
@@ -91,6 +92,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ PrefillBars bars;
+    __shared__ int32_t s_pid[kPidCap];   // the sequence's page ids, read once for every copy
 
     const int pair = blockIdx.x, b = blockIdx.y / a.Hkv, h = blockIdx.y % a.Hkv, li = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -131,6 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
     for (int i = threadIdx.x; i < npg; i += blockDim.x) {
         const int pg = __ldg(pt + i);
         badp |= (pg < 0 || pg >= a.num_pages);
+        if (i < kPidCap) s_pid[i] = pg;
     }
     badp = __syncthreads_or(badp);
     if (threadIdx.x == 0) {
@@ -331,34 +334,27 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
             // ------------------------------------------------------ dequant warps
             const int dt = threadIdx.x - 32 * kDequantWarp0;   // 0..95
             // The copies are issued by the last dequant warp, which has the
-            // fewest dequantisation items.  The page ids of a block are read one
-            // block ahead: a page-table load ahead of each copy would otherwise
-            // put four serial L2 round trips on every block.
+            // fewest dequantisation items; page ids come from shared memory
+            // (a global load per copy would put an L2 round trip on every
+            // block).
             const bool issuer = (dt == 32 * (kWarpsDequant - 1));
             int issued = 0;
-            int pgn[4] = {0, 0, 0, 0};   // page ids of block `issued`
-            auto fetch_ids = [&](int j) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) pgn[k] = (j * 4 + k < npg) ? __ldg(pt + j * 4 + k) : 0;
-            };
             auto issue = [&](int j) {   // stage j % kStageN <- the pages of block j
                 const int st = j % kStageN;
                 const int p_lo = j * 4, n_p = min(npg, p_lo + 4) - p_lo;
-                int pg[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) pg[k] = pgn[k];
-                fetch_ids(j + 1);
                 constexpr int part = KB ? kVPart : kTile;          // bytes staged per page
                 constexpr int part0 = KB ? kBf16VCodes : 0;       // offset of that part in the tile
                 constexpr int tile = KB ? kTileBf16K : kTile;
                 mbar_arrive_expect_tx(&bars.stage_full[st], (uint32_t)n_p * part);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    if (k < n_p)
+                    if (k < n_p) {
+                        const int p = p_lo + k;
+                        const int pg = p < kPidCap ? s_pid[p] : __ldg(pt + p);
                         bulk_g2s(smem + kOffStage + st * kStageBytes + k * part,
-                                 layer_base + ((size_t)pg[k] * a.Hkv + h) * tile + part0, part, &bars.stage_full[st]);
+                                 layer_base + ((size_t)pg * a.Hkv + h) * tile + part0, part, &bars.stage_full[st]);
+                    }
             };
-            if (issuer) fetch_ids(0);
             // every stage is filled up front; a stage is refilled (block j +
             // kStageN) as soon as the three warps have read block j out of it
             if (issuer)
@@ -467,7 +463,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                     const int tkn = it >> 1, half = it & 1;
                     uint8_t* dst = Kt + half * (kBlkTok * 128);
                     if (j * kBlkTok + tkn < kv_end) {
-                        const int pg = __ldg(pt + j * 4 + (tkn >> 4));
+                        const int p = j * 4 + (tkn >> 4);
+                        const int pg = p < kPidCap ? s_pid[p] : __ldg(pt + p);
                         const uint8_t* src = layer_base + ((size_t)pg * a.Hkv + h) * kTileBf16K + (tkn & 15) * 256 +
                                              half * 128;
 #pragma unroll
