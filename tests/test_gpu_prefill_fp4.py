@@ -116,3 +116,39 @@ def test_fp4_prefill_full_config_sampled(kvq):
         for r_i, r in enumerate(rows):
             want = harness.oracle_attend_fp4q(p, li, b, qh[r_i][None], P0 + r, lens[b], cal)
             harness.check_attention(out_h[li, b, r_i], want[0], f"fp4 prefill layer {li} seq {b} row {r} bf16")
+
+
+def test_fp4_prefill_edges(kvq):
+    # one query; keys filling exactly two 64-key blocks; a zero-length sequence
+    w = _small(num_layers=1, batch=3, calib_windows=1, calib_len=64, prefill_chunk=1)
+    lens = [128, 65, 0]
+    p = harness.build_problem(kvq, w, lens=[128, 65, 1])
+    cal = harness.calib_host(p)
+    q = synth.prefill_queries(w, 0)[None]                     # [1][3][1][Hq][D]
+    q_start = torch.tensor([127, 64, 0], dtype=torch.int32)
+    out = kvq.prefill_attention(p.shape, p.calib, p.cache, q.cuda(), q_start.cuda(), p.page_table.cuda(),
+                                torch.tensor(lens, dtype=torch.int32).cuda(), out_dtype=torch.float32,
+                                qk_fp4=True).cpu().numpy()
+    for b in range(2):
+        want = harness.oracle_attend_fp4q(p, 0, b, q[0, b].float().numpy(), int(q_start[b]), lens[b], cal)
+        harness.check_attention(out[0, b], want, f"fp4 prefill edge seq {b} f32")
+    assert np.all(out[0, 2] == 0)
+
+
+def test_fp4_prefill_device_faults_are_flagged(kvq):
+    w = _small(num_layers=1, batch=2, calib_windows=1, calib_len=64, prefill_chunk=32)
+    p = harness.build_problem(kvq, w, lens=[96, 96])
+    cal = harness.calib_host(p)
+    q = synth.prefill_queries(w, 0)[None]
+    q_start = torch.tensor([64, 64], dtype=torch.int32)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pt = p.page_table.clone()
+    pt[1, 2] = p.num_pages + 3                                 # outside the pool
+    out = kvq.prefill_attention(p.shape, p.calib, p.cache, q.cuda(), q_start.cuda(), pt.cuda(), p.lens.cuda(),
+                                out_dtype=torch.float32, status=status, qk_fp4=True)
+    torch.cuda.synchronize()
+    assert status.item() & kvq.DEV_BAD_PAGE
+    out = out.cpu().numpy()
+    assert np.all(out[0, 1] == 0)
+    want = harness.oracle_attend_fp4q(p, 0, 0, q[0, 0].float().numpy(), 64, 96, cal)
+    harness.check_attention(out[0, 0], want, "fp4 prefill beside a bad page f32")
