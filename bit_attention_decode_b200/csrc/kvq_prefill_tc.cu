@@ -12,10 +12,11 @@
 // the kv head times its 32 tokens (row = head * 32 + token), so each
 // dequantised key/value block feeds 8 query heads x 32 tokens.  Per 64-token
 // key block (4 pages):
-//   dequant warps (3): bulk-copy the 4 packed page tiles into a staging
-//     ring, dequantise to fp16 (E2M1 x E4M3 is exact in fp16) into a K tile
-//     (K-major) and a V tile (MN-major), both in the 128-byte-swizzled
-//     canonical layouts the MMA reads; rows past the sequence are zeros.
+//   copy warp: bulk-copies the 4 packed page tiles into a staging ring.
+//   dequant warps (2): dequantise to fp16 (E2M1 x E4M3 is exact in fp16)
+//     into a K tile (K-major) and a V tile (MN-major), both in the
+//     128-byte-swizzled canonical layouts the MMA reads; rows past the
+//     sequence are zeros.
 //   MMA warp (1 elected thread): for each tile, S = Q_hi K^T + Q_lo K^T
 //     (M=128, N=64, K=16 steps; the query is split into fp16 hi + lo parts
 //     so its rounding does not reach the scores) into one of the tile's two
@@ -62,17 +63,21 @@ constexpr int kOffStage = kOffV + 2 * kVBytes;    // kStageN stages
 constexpr int kSmemBytes = kOffStage + kStageN * kStageBytes;
 constexpr int kSmemAlloc = kSmemBytes + 1024;     // room to align the base
 
-enum { kWarpsSoftmax = 4 * kTiles, kWarpsDequant = 3 };
-constexpr int kDequantWarp0 = kWarpsSoftmax;                   // warps 8..10
-constexpr int kMmaWarp = kWarpsSoftmax + kWarpsDequant;        // warp 11
+// warps 8, 9 dequantise; warp 10 only issues the bulk copies (a copy costs
+// the issuing thread hundreds of cycles, which would otherwise sit on a
+// dequant warp's path every block)
+enum { kWarpsSoftmax = 4 * kTiles, kWarpsDequant = 2 };
+constexpr int kDequantWarp0 = kWarpsSoftmax;                   // warps 8, 9
+constexpr int kCopyWarp = kDequantWarp0 + kWarpsDequant;       // warp 10
+constexpr int kMmaWarp = kCopyWarp + 1;                        // warp 11
 constexpr int kThreads = 32 * (kMmaWarp + 1);
 
 struct PrefillBars {
     uint64_t q_ready;                 // both softmax warpgroups wrote their query tiles (count 8)
     uint64_t stage_full[kStageN];     // packed pages landed (tx bytes)
-    uint64_t stage_empty[kStageN];    // dequant warps read the stage (count 3)
-    uint64_t k_full[2];               // K tile j%2 written (count 3)
-    uint64_t v_full[2];               // V tile j%2 written (count 3)
+    uint64_t stage_empty[kStageN];    // dequant warps read the stage (count 2)
+    uint64_t k_full[2];               // K tile j%2 written (count 2)
+    uint64_t v_full[2];               // V tile j%2 written (count 2)
     uint64_t s_full[kTiles][2];       // QK(tile, j) done (commit)
     uint64_t p_full[kTiles][2];       // P(tile, j) stored in TMEM, O rescaled (count 4)
     uint64_t pv_done[kTiles][2];      // PV(tile, j) done (commit)
@@ -330,44 +335,47 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars.p_full[t][u]);
             }
-        } else if (warp < kMmaWarp) {
-            // ------------------------------------------------------ dequant warps
-            const int dt = threadIdx.x - 32 * kDequantWarp0;   // 0..95
-            // The copies are issued by the last dequant warp, which has the
-            // fewest dequantisation items; page ids come from shared memory
-            // (a global load per copy would put an L2 round trip on every
-            // block).
-            const bool issuer = (dt == 32 * (kWarpsDequant - 1));
-            int issued = 0;
-            auto issue = [&](int j) {   // stage j % kStageN <- the pages of block j
-                const int st = j % kStageN;
-                const int p_lo = j * 4, n_p = min(npg, p_lo + 4) - p_lo;
+        } else if (warp == kCopyWarp) {
+            // ------------------------------------------------------ copy warp
+            // block j's page tiles (the value parts only for bf16 keys) into
+            // stage j % kStageN, once the dequant warps have read block
+            // j - kStageN out of it; page ids come from shared memory
+            if (lane == 0) {
                 constexpr int part = KB ? kVPart : kTile;          // bytes staged per page
                 constexpr int part0 = KB ? kBf16VCodes : 0;       // offset of that part in the tile
                 constexpr int tile = KB ? kTileBf16K : kTile;
-                mbar_arrive_expect_tx(&bars.stage_full[st], (uint32_t)n_p * part);
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    if (k < n_p) {
-                        const int p = p_lo + k;
-                        const int pg = p < kPidCap ? s_pid[p] : __ldg(pt + p);
-                        bulk_g2s(smem + kOffStage + st * kStageBytes + k * part,
-                                 layer_base + ((size_t)pg * a.Hkv + h) * tile + part0, part, &bars.stage_full[st]);
+                int issued = 0;
+                for (; issued < nb; ++issued) {
+                    const int st = issued % kStageN;
+                    if (issued >= kStageN &&
+                        !mbar_wait(&bars.stage_empty[st], ((issued - kStageN) / kStageN) & 1)) {
+                        atomicOr(&bars.flags, 1);
+                        break;
                     }
-            };
-            // every stage is filled up front; a stage is refilled (block j +
-            // kStageN) as soon as the three warps have read block j out of it
-            if (issuer)
-                for (; issued < kStageN && issued < nb; ++issued) issue(issued);
-            // items (token, half of head_dim): 128 per block over 96 threads
+                    const int p_lo = issued * 4, n_p = min(npg, p_lo + 4) - p_lo;
+                    mbar_arrive_expect_tx(&bars.stage_full[st], (uint32_t)n_p * part);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        if (k < n_p) {
+                            const int p = p_lo + k;
+                            const int pg = p < kPidCap ? s_pid[p] : __ldg(pt + p);
+                            bulk_g2s(smem + kOffStage + st * kStageBytes + k * part,
+                                     layer_base + ((size_t)pg * a.Hkv + h) * tile + part0, part, &bars.stage_full[st]);
+                        }
+                }
+                bars.issued = issued;
+            }
+        } else if (warp < kMmaWarp) {
+            // ------------------------------------------------------ dequant warps
+            const int dt = threadIdx.x - 32 * kDequantWarp0;   // 0..63
+            // items (token, half of head_dim): 128 per block over 64 threads
             constexpr int kItems = 2 * kBlkTok, kDqThreads = 32 * kWarpsDequant;
             constexpr int kPer = (kItems + kDqThreads - 1) / kDqThreads;
             struct Staged {
                 uint4 kc[kPer][2], vc[kPer][2];
                 uint32_t ks[kPer], vs[kPer][4];
             };
-            // read block j's codes and scales out of its stage, release the
-            // stage and (issuer) refill it with block j + kStageN
+            // read block j's codes and scales out of its stage and release it
             auto load_block = [&](int j, Staged& S) -> bool {
                 const int st = j % kStageN;
                 if (!mbar_wait_warp(&bars.stage_full[st], (j / kStageN) & 1)) return false;
@@ -401,16 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                 }
                 __syncwarp();
                 if ((dt & 31) == 0) mbar_arrive(&bars.stage_empty[st]);
-                int issue_ok = 1;
-                if (issuer && issued < nb) {   // issued == j + kStageN
-                    if (!mbar_wait(&bars.stage_empty[st], (j / kStageN) & 1)) {
-                        issue_ok = 0;
-                    } else {
-                        issue(issued);
-                        ++issued;
-                    }
-                }
-                return __shfl_sync(0xFFFFFFFFu, issue_ok, 0) != 0;
+                return true;
             };
             // keys of block j into K buffer j & 1, free once both tiles'
             // Q.K(j - 2) are done (the commit after the last MMA covers all)
@@ -546,7 +545,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                 }
             }
             if (!dq_ok) atomicOr(&bars.flags, 1);
-            if (issuer) bars.issued = issued;
         } else if (lane == 0) {
             // ------------------------------------------------------ MMA issuer
             // Descriptors are built once; a k-step only advances the 14-bit
