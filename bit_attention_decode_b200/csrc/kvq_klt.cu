@@ -291,29 +291,39 @@ __global__ void klt_finalize_kernel(float* __restrict__ gk, float* __restrict__ 
 }
 
 // ------------------------------------------------------------------ append
-// Keys of the KLT cache: grid (tiles of 64 tokens, Hkv, nlayers).  Smoothing
-// y = k * inv_s, the transform y' = U^T y (klt_tile), then the NVFP4
-// quantiser of the append (absmax -> E4M3 scale -> reciprocal -> E2M1, each
-// step one fp32 rounding) and the scatter to the token's slot.  Thread
-// (tg, dg) holds dims 8dg..8dg+7 of 4 tokens; the two threads of a 16-block
-// (dg, dg ^ 1) are neighbouring lanes and share its absmax by a shuffle.
+// Keys of the KLT cache: grid (CTAs per (layer, head), Hkv, nlayers), 128
+// threads, two CTAs per SM; each CTA loads the basis once and walks tiles of
+// 64 tokens (one CTA's tile load overlaps the other's transform).  Smoothing y = k * inv_s,
+// the transform y' = U^T y (one fp32 FMA chain per output over c = 0..127),
+// then the NVFP4 quantiser of the append (absmax -> E4M3 scale -> reciprocal
+// -> E2M1, each step one fp32 rounding) and the scatter to the token's slot.
+//
+// Thread (warp w, lane l) holds 8 tokens (8 (2w + l / 16) .. + 7) x 8 dims
+// (4 (l % 16) .. + 3 and 64 + 4 (l % 16) .. + 3): per step c it reads 8
+// token values (the same for a half-warp) and two runs of 4 basis values
+// (contiguous over a quarter-warp), 16 shared-memory wavefronts for 64 FMAs,
+// which keeps shared memory and the FMA pipe in balance.  The 4 lanes of a
+// 16-block are neighbours and share its absmax by two shuffles.
 __device__ __forceinline__ uint32_t klt_e2m1x2(float hi, float lo) {
     uint16_t r;
     asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u16.u8 %0, t; }" : "=h"(r) : "f"(hi), "f"(lo));
     return r;
 }
 
-constexpr size_t kKltAppendSmem = kKltTileSmem + 128 * sizeof(float) + 64 * sizeof(int64_t) + 16;
+constexpr int kKltTok = 64;   // tokens per append tile
+constexpr size_t kKltAppendSmem =
+    (size_t)kD * kD * sizeof(float) + (size_t)kD * kKltTok * sizeof(float) + 128 * sizeof(float) +
+    kKltTok * sizeof(int64_t) + 16;
 
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(128, 2)
 klt_append_keys_kernel(const T* __restrict__ k, const int64_t* __restrict__ slots, int num_tokens, int Hkv,
                        const float* __restrict__ inv_s, const float* __restrict__ U, const float* __restrict__ gk,
                        uint8_t* __restrict__ cache, int64_t layer_stride, int num_pages, int32_t* __restrict__ status) {
     extern __shared__ __align__(16) float sm[];
-    float* Us = sm;
-    float* Yt = Us + kD * kD;
-    float* rtab = Yt + kD * 64;
+    float* Us = sm;                              // [c][i]
+    float* Yt = Us + kD * kD;                    // [c][token]
+    float* rtab = Yt + kD * kKltTok;
     int64_t* sslot = reinterpret_cast<int64_t*>(rtab + 128);
     const int h = blockIdx.y, li = blockIdx.z;
     klt_load_basis(Us, U + ((size_t)li * Hkv + h) * kD * kD);
@@ -327,17 +337,19 @@ klt_append_keys_kernel(const T* __restrict__ k, const int64_t* __restrict__ slot
     const float* inv = inv_s + ((size_t)li * Hkv + h) * kD;
     const int64_t num_slots = (int64_t)num_pages * kPage;
     uint8_t* layer_cache = cache + (size_t)li * layer_stride;
-    const int tg = threadIdx.x >> 4, dg = threadIdx.x & 15;
-    const int ntiles = (num_tokens + 63) / 64;
-    // the basis is loaded once; the CTA walks tiles of its (layer, head)
+    const int lane = threadIdx.x & 31;
+    const int tgi = 2 * (threadIdx.x >> 5) + (lane >> 4);   // token group: tokens 8 tgi .. + 7
+    const int dl = lane & 15;                               // dims 4 dl .. + 3 and 64 + 4 dl .. + 3
+    const int ntiles = (num_tokens + kKltTok - 1) / kKltTok;
     for (int tile_i = blockIdx.x; tile_i < ntiles; tile_i += gridDim.x) {
-        const int t0 = tile_i * 64;
+        const int t0 = tile_i * kKltTok;
         __syncthreads();     // the previous tile's Yt and slots are consumed
-        if (threadIdx.x < 64) sslot[threadIdx.x] = (t0 + threadIdx.x < num_tokens) ? __ldg(slots + t0 + threadIdx.x) : -1;
-        // rows of 8 elements: 64 tokens x 16 groups; neighbouring lanes take
+        if (threadIdx.x < kKltTok)
+            sslot[threadIdx.x] = (t0 + threadIdx.x < num_tokens) ? __ldg(slots + t0 + threadIdx.x) : -1;
+        // rows of 8 elements: 128 tokens x 16 groups; neighbouring lanes take
         // neighbouring tokens, so the transposed stores hit distinct banks
-        for (int e = threadIdx.x; e < 64 * 16; e += blockDim.x) {
-            const int r = e & 63, c8 = (e >> 6) * 8;
+        for (int e = threadIdx.x; e < kKltTok * 16; e += blockDim.x) {
+            const int r = e & (kKltTok - 1), c8 = (e / kKltTok) * 8;
             float x[8];
             if (t0 + r < num_tokens) {
                 load8(k + (((size_t)li * num_tokens + t0 + r) * Hkv + h) * kD + c8, x);
@@ -348,32 +360,51 @@ klt_append_keys_kernel(const T* __restrict__ k, const int64_t* __restrict__ slot
                 for (int j = 0; j < 8; ++j) x[j] = 0.0f;
             }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) Yt[(c8 + j) * 64 + r] = x[j];
+            for (int j = 0; j < 8; ++j) Yt[(c8 + j) * kKltTok + r] = x[j];
         }
         __syncthreads();
-        float acc[4][8];
-        klt_tile(Yt, Us, tg, dg, acc);
+        float acc[8][8];
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            float m = 0.0f;
+        for (int a = 0; a < 8; ++a)
 #pragma unroll
-            for (int b = 0; b < 8; ++b) m = fmaxf(m, fabsf(acc[a][b]));
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));       // the other half of the 16-block
-            const uint32_t sf = e4m3_rn(__fmul_rn(m, enc));
-            const float r = rtab[sf & 0x7Fu];
-            uint32_t w = 0;
+            for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
+#pragma unroll 2
+        for (int c = 0; c < kD; ++c) {
+            const float4 y0 = *reinterpret_cast<const float4*>(Yt + c * kKltTok + 8 * tgi);
+            const float4 y1 = *reinterpret_cast<const float4*>(Yt + c * kKltTok + 8 * tgi + 4);
+            const float4 u0 = *reinterpret_cast<const float4*>(Us + c * kD + 4 * dl);
+            const float4 u1 = *reinterpret_cast<const float4*>(Us + c * kD + 64 + 4 * dl);
+            const float y[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+            const float u[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                w |= klt_e2m1x2(__fmul_rn(acc[a][2 * j + 1], r), __fmul_rn(acc[a][2 * j], r)) << (8 * j);
-            const int tt = 4 * tg + a;
+            for (int a = 0; a < 8; ++a)
+#pragma unroll
+                for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(u[b], y[a], acc[a][b]);
+        }
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+            const int tt = 8 * tgi + a;
             const int64_t slot = sslot[tt];
-            if (slot >= num_slots) {
-                if (dg == 0) set_status(status, KVQ_DEV_BAD_SLOT);
-            } else if (slot >= 0) {
-                uint8_t* tile = layer_cache + ((size_t)(slot >> 4) * Hkv + h) * kTile;
-                const int off = (int)(slot & 15);
-                *reinterpret_cast<uint32_t*>(tile + kKCodes + off * 64 + 4 * dg) = w;
-                if ((dg & 1) == 0) tile[kKScales + off * 8 + (dg >> 1)] = (uint8_t)sf;
+#pragma unroll
+            for (int gi = 0; gi < 2; ++gi) {
+                // this lane's 4 dims of block 4 gi + dl / 4; the block's 4 lanes are neighbours
+                float m = fmaxf(fmaxf(fabsf(acc[a][4 * gi]), fabsf(acc[a][4 * gi + 1])),
+                                fmaxf(fabsf(acc[a][4 * gi + 2]), fabsf(acc[a][4 * gi + 3])));
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+                const uint32_t sf = e4m3_rn(__fmul_rn(m, enc));
+                const float r = rtab[sf & 0x7Fu];
+                const uint32_t w = klt_e2m1x2(__fmul_rn(acc[a][4 * gi + 1], r), __fmul_rn(acc[a][4 * gi], r)) |
+                                   (klt_e2m1x2(__fmul_rn(acc[a][4 * gi + 3], r), __fmul_rn(acc[a][4 * gi + 2], r)) << 8);
+                if (slot >= num_slots) {
+                    if (dl == 0 && gi == 0) set_status(status, KVQ_DEV_BAD_SLOT);
+                } else if (slot >= 0) {
+                    uint8_t* tile = layer_cache + ((size_t)(slot >> 4) * Hkv + h) * kTile;
+                    const int off = (int)(slot & 15);
+                    // dims 64 gi + 4 dl .. + 3: code bytes 32 gi + 2 dl, + 1
+                    *reinterpret_cast<uint16_t*>(tile + kKCodes + off * 64 + 32 * gi + 2 * dl) = (uint16_t)w;
+                    if ((dl & 3) == 0) tile[kKScales + off * 8 + 4 * gi + (dl >> 2)] = (uint8_t)sf;
+                }
             }
         }
     }
@@ -390,7 +421,7 @@ kvq_status append_klt_keys(const kvq_shape& s, const kvq_calib& c, const kvq_cac
     // about two CTAs per SM in all; each walks tiles of its (layer, head)
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const long ntiles = (num_tokens + 63) / 64;
+    const long ntiles = (num_tokens + kKltTok - 1) / kKltTok;
     const long per = (2L * sms + (long)H * nlayers - 1) / ((long)H * nlayers);
     const dim3 grid((unsigned)(ntiles < per ? ntiles : (per < 1 ? 1 : per)), H, nlayers);
     cudaError_t e;
@@ -398,14 +429,14 @@ kvq_status append_klt_keys(const kvq_shape& s, const kvq_calib& c, const kvq_cac
         e = cudaFuncSetAttribute(klt_append_keys_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kKltAppendSmem);
         if (e != cudaSuccess) return KVQ_ECUDA;
-        klt_append_keys_kernel<float><<<grid, 256, kKltAppendSmem, st>>>((const float*)k, slots, num_tokens, H, inv,
+        klt_append_keys_kernel<float><<<grid, 128, kKltAppendSmem, st>>>((const float*)k, slots, num_tokens, H, inv,
                                                                        U, gk, base, cache.layer_stride_bytes,
                                                                        cache.num_pages, status);
     } else {
         e = cudaFuncSetAttribute(klt_append_keys_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kKltAppendSmem);
         if (e != cudaSuccess) return KVQ_ECUDA;
-        klt_append_keys_kernel<__nv_bfloat16><<<grid, 256, kKltAppendSmem, st>>>(
+        klt_append_keys_kernel<__nv_bfloat16><<<grid, 128, kKltAppendSmem, st>>>(
             (const __nv_bfloat16*)k, slots, num_tokens, H, inv, U, gk, base, cache.layer_stride_bytes,
             cache.num_pages, status);
     }
