@@ -212,6 +212,38 @@ def ncu_traffic():
         return None
 
 
+def fp32_fma_peak_tflops():
+    """FP32 FMA peak from unit counts and clocks: 128 FMA lanes per SM per
+    clock x SMs x the maximum SM clock (148 x 128 x 1.965 GHz = 37.2 TFMA/s
+    on B200)."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        h = pynvml.nvmlDeviceGetHandleByIndex(torch.cuda.current_device())
+        mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+    except Exception:
+        mhz = 1965
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return sms * 128 * mhz * 1e6 / 1e12
+
+
+def append_entry(wl, peak_hbm):
+    """The bulk append's line: HBM-bound, except with the KLT, whose key
+    transform (16,384 FMAs per token-head) makes it bound by the FP32 FMA pipe."""
+    ms = statistics.median(wl.append_ms)
+    gbs = wl.append_bytes / (ms / 1e3) / 1e9
+    d = {"kernel": "kvq quantize-append (bulk prefix, one layer per launch)", "alg_bytes_per_launch": wl.append_bytes,
+         "achieved": gbs, "unit": "GB/s", "frac": gbs / peak_hbm, "bound": "hbm"}
+    if wl.klt:
+        fma = wl.prefix_tokens * wl.w.num_kv_heads * 128 * 128      # the key transform, per launch
+        tfma = fma / (ms / 1e3) / 1e12
+        pk = fp32_fma_peak_tflops()
+        d.update({"bound": "alu", "alu_achieved": tfma, "alu_peak": pk, "alu_unit": "TFMA/s", "alu_frac": tfma / pk,
+                  "alu_peak_source": "derived: SMs x 128 FP32 FMA lanes x max SM clock",
+                  "alg_fma_per_launch": fma})
+    return d
+
+
 # ------------------------------------------------------------------ workload
 class Ragged:
     """Device-resident ragged decode workload (one replica)."""
@@ -708,11 +740,7 @@ def main():
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
                          "kernel": "kvq decode (+split combine)", "alg_bytes_per_launch": dec_bytes},
-            "append": {"kernel": "kvq quantize-append (bulk prefix, one layer per launch)",
-                       "alg_bytes_per_launch": wl.append_bytes,
-                       "achieved": wl.append_bytes / (statistics.median(wl.append_ms) / 1e3) / 1e9,
-                       "unit": "GB/s",
-                       "frac": wl.append_bytes / (statistics.median(wl.append_ms) / 1e3) / 1e9 / peak},
+            "append": append_entry(wl, peak),
             "gpu_launches": wl.launches_per_step * args.steps,
             "clocks": clocks}
     if not args.no_e2e:
