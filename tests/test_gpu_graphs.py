@@ -1,4 +1,4 @@
-"""The hot path under CUDA-graph capture.
+"""The hot path under CUDA-graph capture and on concurrent streams.
 
 A serving loop captures a decode step once and replays it with new inputs
 copied into the captured buffers.  Every call of the library is stream-ordered
@@ -7,7 +7,8 @@ token per sequence into every layer, then decode every layer (split-K with
 the combine on this small batch) -- and a chunked prefill (fp16 and FP4 Q.K)
 are captured with torch.cuda.CUDAGraph and replayed.  Each replay must equal
 the eager call on a copy of the cache bit for bit: the same kernels in the
-same launch shapes, deterministic reductions.
+same launch shapes, deterministic reductions.  Two problems run at once on two
+streams give their sequential results bit for bit (the library keeps no state).
 """
 import dataclasses
 
@@ -105,3 +106,32 @@ def test_prefill_graph_replay_matches_eager(kvq, fp4):
         g.replay()
         torch.cuda.synchronize()
         assert torch.equal(out_buf, want)
+
+
+def test_concurrent_streams_match_sequential(kvq):
+    # the library keeps no state: two problems decoded (and prefilled) at the
+    # same time on two streams give the sequential results bit for bit
+    w = _small(num_layers=2, batch=3, calib_windows=1, calib_len=64, prefill_chunk=32)
+    probs = [harness.build_problem(kvq, w, lens=[40 + 30 * i, 90, 200 - 50 * i]) for i in range(2)]
+    qd = torch.stack([synth.decode_queries(w, l, 0, "cuda") for l in range(2)])
+    qp = torch.stack([synth.prefill_queries(w, l, "cuda") for l in range(2)])
+
+    def run(p):
+        ln = p.lens.cuda()
+        d = kvq.decode_attention(p.shape, p.calib, p.cache, qd, p.page_table.cuda(), ln, out_dtype=torch.float32)
+        qs = (ln - 32).clamp_min(0).to(torch.int32)
+        f = kvq.prefill_attention(p.shape, p.calib, p.cache, qp, qs, p.page_table.cuda(), ln,
+                                  out_dtype=torch.float32)
+        return d, f
+
+    want = [run(p) for p in probs]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in probs]
+    got = []
+    for p, s in zip(probs, streams):
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            got.append(run(p))
+    torch.cuda.synchronize()
+    for (d0, f0), (d1, f1) in zip(want, got):
+        assert torch.equal(d0, d1) and torch.equal(f0, f1)
