@@ -100,3 +100,36 @@ def test_chunked_prefill(kvq):
         for r_i, r in enumerate(rows):
             want = harness.oracle_attend(p, li, b, qh[r_i][None], P0 + r, lens[b], cal)
             harness.check_attention(out_h[li, b, r_i], want[0], f"prefill layer {li} seq {b} row {r} bf16")
+
+
+@pytest.mark.parametrize("variant", ["klt", "bf16_keys"])
+def test_ragged_variants_full_size(kvq, variant):
+    # the ragged workload (36 layers, 64 sequences of 1024..8192 tokens) with
+    # the static per-head KLT (bench.py --klt) or the mixed cache of bf16 keys
+    # and NVFP4 values (bench.py --k-format bf16), as the bench launches them:
+    # one step appended into all 36 layers, then all 36 layers decoded.
+    # Codes and scales bit for bit and attention rows within tolerance, on
+    # sampled (layer, sequence) pairs.
+    w = synth.WORKLOADS["ragged"]
+    lens = synth.ragged_lengths(w)
+    order = torch.argsort(lens)
+    sample_seqs = sorted({int(order[0]), int(order[-1]), int(order[len(order) // 2])})
+    keep = {(l, b) for l in (0, 35) for b in sample_seqs}
+    p = harness.build_problem(kvq, w, lens=lens, extra_tokens=1, gen_device="cuda", keep=keep, keep_tails=True,
+                              klt=(variant == "klt"), k_format=(1 if variant == "bf16_keys" else 0))
+    cal = harness.calib_host(p)
+    tk, tv = p.tails
+    slots = synth.slot_mapping(p.page_table, torch.arange(w.batch), lens.long()).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvq.quantize_append(p.shape, p.calib, p.cache, tk[0].contiguous(), tv[0].contiguous(), slots, status=status)
+    seq_lens = (lens + 1).to(torch.int32)
+    q = torch.stack([synth.decode_queries(w, l, 0, "cuda") for l in range(w.num_layers)])
+    out = kvq.decode_attention(p.shape, p.calib, p.cache, q, p.page_table.cuda(), seq_lens.cuda(),
+                               out_dtype=torch.bfloat16, status=status).float().cpu().numpy()
+    assert status.item() == 0
+    qh = q.float().cpu().numpy()
+    for (li, b) in sorted(keep):
+        n = int(seq_lens[b])
+        assert_codes_equal(p, li, b, n, cal)
+        want = harness.oracle_attend(p, li, b, qh[li, b][None], n - 1, n, cal)
+        harness.check_attention(out[li, b], want[0], f"ragged {variant} layer {li} seq {b} len {n} bf16")
