@@ -135,3 +135,23 @@ def test_concurrent_streams_match_sequential(kvq):
     torch.cuda.synchronize()
     for (d0, f0), (d1, f1) in zip(want, got):
         assert torch.equal(d0, d1) and torch.equal(f0, f1)
+
+
+def test_noalloc_decode_graph_replay(kvq):
+    # the allocation-free entry point under capture: its first call (which
+    # looks up the static scratch array) is made before the capture
+    w = _small(num_layers=2, batch=3, calib_windows=1, calib_len=64)
+    lens = torch.tensor([40, 77, 130], dtype=torch.int32)
+    p = harness.build_problem(kvq, w, lens=lens)
+    pt, ln = p.page_table.cuda(), lens.cuda()
+    q_buf = torch.stack([synth.decode_queries(w, l, 0, "cuda") for l in range(2)])
+    out_buf = torch.empty(q_buf.shape, dtype=torch.float32, device="cuda")
+    kvq.decode_attention_noalloc(p.shape, p.calib, p.cache, q_buf, pt, ln, out_buf)   # before capture
+    g = _capture(lambda: kvq.decode_attention_noalloc(p.shape, p.calib, p.cache, q_buf, pt, ln, out_buf))
+    for step in (1, 2):
+        q = torch.stack([synth.decode_queries(w, l, step, "cuda") for l in range(2)])
+        want = kvq.decode_attention(p.shape, p.calib, p.cache, q, pt, ln, out_dtype=torch.float32)
+        q_buf.copy_(q)
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out_buf, want)
