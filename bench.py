@@ -436,23 +436,30 @@ class Prefix:
                                   workspace=self.ws)
 
 
+def nvtx(name: str):
+    """An NVTX range (for filtering a profiler capture to the timed steps)."""
+    return torch.cuda.nvtx.range(name)
+
+
 def time_two_kernels(first, second, warmup: int, steps: int, world: int):
     """Time steps of first() + second() with events around each call."""
     st = torch.cuda.current_stream()
-    for _ in range(warmup):
-        first()
-        second()
+    with nvtx("warmup"):
+        for _ in range(warmup):
+            first()
+            second()
     torch.cuda.synchronize()
     barrier(world)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(st)
-    for i in range(steps):
-        ev[i][0].record(st)
-        first()
-        ev[i][1].record(st)
-        second()
-        ev[i][2].record(st)
+    with nvtx("timed steps"):
+        for i in range(steps):
+            ev[i][0].record(st)
+            first()
+            ev[i][1].record(st)
+            second()
+            ev[i][2].record(st)
     t1.record(st)
     torch.cuda.synchronize()
     barrier(world)
@@ -461,10 +468,11 @@ def time_two_kernels(first, second, warmup: int, steps: int, world: int):
 
 def time_device(wl: Ragged, warmup: int, steps: int, world: int):
     st = torch.cuda.current_stream()
-    for i in range(warmup):
-        s = i % wl.S
-        wl.append(s)
-        wl.decode(s)
+    with nvtx("warmup"):
+        for i in range(warmup):
+            s = i % wl.S
+            wl.append(s)
+            wl.decode(s)
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
@@ -472,13 +480,16 @@ def time_device(wl: Ragged, warmup: int, steps: int, world: int):
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dec_bytes = 0
     t0.record(st)
-    for i in range(steps):
-        s = (warmup + i) % wl.S
-        wl.append(s)
-        ev[i][0].record(st)
-        wl.decode(s)
-        ev[i][1].record(st)
-        dec_bytes += wl.decode_bytes(s)
+    with nvtx("timed steps"):
+        for i in range(steps):
+            s = (warmup + i) % wl.S
+            with nvtx(f"step {i}: append"):
+                wl.append(s)
+            ev[i][0].record(st)
+            with nvtx(f"step {i}: decode"):
+                wl.decode(s)
+            ev[i][1].record(st)
+            dec_bytes += wl.decode_bytes(s)
     t1.record(st)
     torch.cuda.synchronize()
     barrier(world)
