@@ -10,7 +10,7 @@
 // and the online softmax.  Every dequantised E2M1 x E4M3 product is exact in
 // fp16; the query is split into fp16 hi + lo columns (its rounding would
 // otherwise reach the scores at ~1e-2), the probabilities are rounded once to
-// fp16 (relative error <= 2^-12 per weight), and everything accumulates in
+// fp16 (relative error <= 2^-11 per weight), and everything accumulates in
 // fp32.
 //
 // Work unit (one CTA): one layer, one sequence, one split of its pages, all
@@ -30,7 +30,7 @@
 
 namespace kvq {
 
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // ------------------------------------------------------------------ primitives
@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
     float o[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
-    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.0f, l_b = 0.0f;
+    float m_h = -INFINITY, l_h = 0.0f;       // running reference and sum of head c
 
     if (warp == Hkv) {
         // ---------------------------------------------------------- producer
@@ -229,7 +229,10 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
         // ---------------------------------------------------------- consumer
         const int h = warp;
         const int G = a.G;
-        const int jq = g & 3;                 // query head of this lane's B-fragment column
+        // B-fragment column g of Q.K: head g >> 1, its hi part for even g and
+        // its lo part for odd g, so score columns 2c and 2c + 1 are the two
+        // parts of head c and a lane adds them without a shuffle
+        const int jq = g >> 1;
         const bool head_ok = jq < G;
         // query prologue: lane (g, c) holds dims 32c..32c+31 of head jq
         float qv[32];
@@ -301,16 +304,14 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
                     // bf16 hi + lo: 16 significant bits of the query
                     const uint32_t hv = pack_bf2(x0, x1);
                     const float2 f = unpack_bf2(hv);
-                    qb[2 * s + r] = (g < 4) ? hv : pack_bf2(x0 - f.x, x1 - f.y);
+                    qb[2 * s + r] = (g & 1) ? pack_bf2(x0 - f.x, x1 - f.y) : hv;
                 } else {
                     const uint32_t hv = pack_h2(x0, x1);
                     const float2 f = unpack_h2(hv);
-                    qb[2 * s + r] = (g < 4) ? hv : pack_h2(x0 - f.x, x1 - f.y);
+                    qb[2 * s + r] = (g & 1) ? pack_h2(x0 - f.x, x1 - f.y) : hv;
                 }
             }
-        const int ha = 2 * (c & 1), hb = ha + 1;   // heads of this lane's score columns
-        const float isg_a = __shfl_sync(kFull, isig, ha * 4);
-        const float isg_b = __shfl_sync(kFull, isig, hb * 4);
+        const float isg = __shfl_sync(kFull, isig, 8 * c);   // head c's normalisation (lane g = 2c)
 
         const uint8_t* my_tile = smem + h * kTB;
         for (int i = 0; i < n; ++i) {
@@ -382,14 +383,12 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
             }
 #pragma unroll
             for (int k = 0; k < 4; ++k) sacc[k] += sacc2[k];
-            // hi + lo columns -> full scores of heads ha, hb for tokens g, g + 8
-            float s0 = sacc[0] + __shfl_xor_sync(kFull, sacc[0], 2);
-            float s1 = sacc[1] + __shfl_xor_sync(kFull, sacc[1], 2);
-            float s2 = sacc[2] + __shfl_xor_sync(kFull, sacc[2], 2);
-            float s3 = sacc[3] + __shfl_xor_sync(kFull, sacc[3], 2);
+            // hi + lo columns -> scores of head c for tokens g, g + 8
+            float s0 = sacc[0] + sacc[1];
+            float s1 = sacc[2] + sacc[3];
             if (nvalid < kPage) {
-                if (g >= nvalid) s0 = s1 = -INFINITY;
-                if (g + 8 >= nvalid) s2 = s3 = -INFINITY;
+                if (g >= nvalid) s0 = -INFINITY;
+                if (g + 8 >= nvalid) s1 = -INFINITY;
                 // stale slots past the end may hold anything: zero their value scales
                 const uint32_t m01 = ((2 * c < nvalid) ? 0xFFFFu : 0u) | ((2 * c + 1 < nvalid) ? 0xFFFF0000u : 0u);
                 const uint32_t m89 = ((2 * c + 8 < nvalid) ? 0xFFFFu : 0u) | ((2 * c + 9 < nvalid) ? 0xFFFF0000u : 0u);
@@ -399,38 +398,42 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
                 vs01 = e4m3x2_to_f16x2(vs01);
                 vs89 = e4m3x2_to_f16x2(vs89);
             }
-            // ---- online softmax (exp2 domain)
-            float pm_a = fmaxf(s0, s2), pm_b = fmaxf(s1, s3);
+            // ---- online softmax (exp2 domain) with a lazy reference: m moves
+            // only when a score of this page exceeds it by more than 8 (a
+            // weight above 2^8), so most pages skip the cross-lane max and the
+            // rescale.  Any common reference gives the same o / l; bounding the
+            // weights by 2^8 keeps them, scaled by 2^7, inside fp16.
+            const float lm = fmaxf(s0, s1) * isg;
+            if (__any_sync(kFull, lm > m_h + 8.0f)) {
+                float pm = lm;
 #pragma unroll
-            for (int x = 4; x < 32; x <<= 1) {
-                pm_a = fmaxf(pm_a, __shfl_xor_sync(kFull, pm_a, x));
-                pm_b = fmaxf(pm_b, __shfl_xor_sync(kFull, pm_b, x));
-            }
-            pm_a *= isg_a;
-            pm_b *= isg_b;
-            const float mn_a = fmaxf(m_a, pm_a), mn_b = fmaxf(m_b, pm_b);
-            if (__any_sync(kFull, (mn_a > m_a) || (mn_b > m_b))) {
-                const float al_a = fast_exp2(m_a - mn_a), al_b = fast_exp2(m_b - mn_b);
-                l_a *= al_a;
-                l_b *= al_b;
+                for (int x = 4; x < 32; x <<= 1) pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, x));
+                const float mn = fmaxf(m_h, pm);
+                const float al = fast_exp2(m_h - mn);
+                l_h *= al;
+                // output columns 2c, 2c + 1 are heads 2c, 2c + 1 (zero for c >= 2)
+                const float al_a = __shfl_sync(kFull, al, (lane & ~3) | ((2 * c) & 3));
+                const float al_b = __shfl_sync(kFull, al, (lane & ~3) | ((2 * c + 1) & 3));
 #pragma unroll
                 for (int t = 0; t < 8; ++t) {
                     o[t][0] *= al_a; o[t][2] *= al_a;
                     o[t][1] *= al_b; o[t][3] *= al_b;
                 }
-                m_a = mn_a;
-                m_b = mn_b;
+                m_h = mn;
             }
-            // probabilities scaled by 2^15 for the fp16 operand
-            const float ca = 15.0f - m_a, cb = 15.0f - m_b;
-            const float p0 = fast_exp2(fmaf(s0, isg_a, ca)), p1 = fast_exp2(fmaf(s1, isg_b, cb));
-            const float p2 = fast_exp2(fmaf(s2, isg_a, ca)), p3 = fast_exp2(fmaf(s3, isg_b, cb));
-            l_a += p0 + p2;
-            l_b += p1 + p3;
-            // P (fp16, relative rounding <= 2^-12) as the B operand: [tokens] x
-            // [4 heads | 4 zero columns], via an 8x8 transpose
-            const uint32_t m0 = (c < 2) ? pack_h2(p0, p1) : 0u, m1 = (c < 2) ? pack_h2(p2, p3) : 0u;
-            const uint32_t pb0 = movmatrix_t(m0), pb1 = movmatrix_t(m1);
+            // weights (<= 2^8 against the reference) scaled by 2^7 for the fp16 operand
+            const float ca = 7.0f - m_h;
+            const float p0 = fast_exp2(fmaf(s0, isg, ca)), p1 = fast_exp2(fmaf(s1, isg, ca));
+            l_h += p0 + p1;
+            // P (fp16, relative rounding <= 2^-11) as the B operand [tokens] x
+            // [4 heads | 4 zero columns].  Lane (g, c) holds M[g][2c] = P(g, c),
+            // M[g][2c + 1] = P(g + 8, c); after the 8x8 transpose lane (r, c)
+            // holds P(2c, r/2), P(2c + 1, r/2) for even r and the same tokens
+            // + 8 for odd r, so b0 comes from lane (2g, c) and b1 from (2g + 1, c)
+            const uint32_t tp = movmatrix_t(pack_h2(p0, p1));
+            const uint32_t t0 = __shfl_sync(kFull, tp, (((2 * g) & 7) << 2) | c);
+            const uint32_t t1 = __shfl_sync(kFull, tp, (((2 * g + 1) & 7) << 2) | c);
+            const uint32_t pb0 = (g < 4) ? t0 : 0u, pb1 = (g < 4) ? t1 : 0u;
             // ---- O^T += V^T P : rows = dims 16g + 2t (+1), k = tokens
             const uint32_t w0[2] = {v0.x, v0.y}, w1[2] = {v1.x, v1.y};
             const uint32_t w2[2] = {v2.x, v2.y}, w3[2] = {v3.x, v3.y};
@@ -471,8 +474,7 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
     const bool dead = poison || timed_out;
 #pragma unroll
     for (int x = 4; x < 32; x <<= 1) {
-        l_a += __shfl_xor_sync(kFull, l_a, x);
-        l_b += __shfl_xor_sync(kFull, l_b, x);
+        l_h += __shfl_xor_sync(kFull, l_h, x);
     }
 #pragma unroll
     for (int t = 0; t < 8; ++t)
@@ -482,6 +484,9 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
     const int h = warp;
     const bool first = c < 2;
     const int head = first ? 2 * c : 2 * (c - 2) + 1;
+    // head's sum and reference live in lanes (g, head)
+    const float l = __shfl_sync(kFull, l_h, (lane & ~3) | head);
+    const float m = __shfl_sync(kFull, m_h, (lane & ~3) | head);
     if (head >= a.G) return;
     float r[16];
 #pragma unroll
@@ -489,8 +494,6 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
         r[2 * t] = first ? o[t][0] : o[t][1];
         r[2 * t + 1] = first ? o[t][2] : o[t][3];
     }
-    const float l = first ? l_a : l_b;
-    const float m = first ? m_a : m_b;
     const int hq = h * a.G + head;
     if (a.splits == 1) {
         const float sc = (dead || l == 0.0f) ? 0.0f : __ldg(a.gv + li) / l;

@@ -97,7 +97,7 @@ def test_fp4_prefill_query_quantisation_error(kvq, capsys):
 
 
 def test_fp4_prefill_full_config_sampled(kvq):
-    # the prefill workload (32 sequences, 512-token chunks after 8192 cached
+    # the prefill workload (8 sequences of 32 query heads, 512-token chunks after 8192 cached
     # tokens, 36 layers) in the bench's launch, sampled rows against the oracle
     w = synth.WORKLOADS["prefill"]
     B, Tq, P0 = w.batch, w.prefill_chunk, w.context
