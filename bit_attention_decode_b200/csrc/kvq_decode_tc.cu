@@ -58,11 +58,6 @@ __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
 __device__ __forceinline__ float2 unpack_bf2(uint32_t a) {
     return make_float2(__uint_as_float(a << 16), __uint_as_float(a & 0xFFFF0000u));
 }
-__device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
-    uint32_t d;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
-    return d;
-}
 __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
     __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
     return *reinterpret_cast<uint32_t*>(&r);
@@ -213,15 +208,20 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
         // ---------------------------------------------------------- producer
         if (lane == 0 && !poison) {
             int i = 0;
+            int st = 0;
+            uint32_t ph = 0;          // parity of round i / kST
             for (; i < n; ++i) {
-                const int st = i % kST;
-                if (i >= kST && !mbar_wait(&empty[st], ((i / kST) - 1) & 1)) {
+                if (i >= kST && !mbar_wait(&empty[st], ph ^ 1u)) {
                     atomicOr(&s_flags, 1);
                     break;
                 }
                 const int pg = __ldg(pt + i);
                 mbar_arrive_expect_tx(&full[st], page_bytes);
                 bulk_g2s(smem + st * page_bytes, layer_base + (size_t)pg * page_bytes, page_bytes, &full[st]);
+                if (++st == kST) {
+                    st = 0;
+                    ph ^= 1u;
+                }
             }
             s_issued = i;
         }
@@ -314,9 +314,10 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
         const float isg = __shfl_sync(kFull, isig, 8 * c);   // head c's normalisation (lane g = 2c)
 
         const uint8_t* my_tile = smem + h * kTB;
+        int st = 0;
+        uint32_t ph = 0;              // parity of round i / kST
         for (int i = 0; i < n; ++i) {
-            const int st = i % kST;
-            if (!mbar_wait(&full[st], (i / kST) & 1)) {
+            if (!mbar_wait(&full[st], ph)) {
                 atomicOr(&s_flags, 1);
                 break;
             }
@@ -426,14 +427,14 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
             const float p0 = fast_exp2(fmaf(s0, isg, ca)), p1 = fast_exp2(fmaf(s1, isg, ca));
             l_h += p0 + p1;
             // P (fp16, relative rounding <= 2^-11) as the B operand [tokens] x
-            // [4 heads | 4 zero columns].  Lane (g, c) holds M[g][2c] = P(g, c),
-            // M[g][2c + 1] = P(g + 8, c); after the 8x8 transpose lane (r, c)
-            // holds P(2c, r/2), P(2c + 1, r/2) for even r and the same tokens
-            // + 8 for odd r, so b0 comes from lane (2g, c) and b1 from (2g + 1, c)
-            const uint32_t tp = movmatrix_t(pack_h2(p0, p1));
-            const uint32_t t0 = __shfl_sync(kFull, tp, (((2 * g) & 7) << 2) | c);
-            const uint32_t t1 = __shfl_sync(kFull, tp, (((2 * g + 1) & 7) << 2) | c);
-            const uint32_t pb0 = (g < 4) ? t0 : 0u, pb1 = (g < 4) ? t1 : 0u;
+            // [4 heads | 4 zero columns]: lane (g, c) needs tokens 2c, 2c + 1
+            // (b0) and 2c + 8, 2c + 9 (b1) of head g, held by lanes (2c, g)
+            // and (2c + 1, g) as their (token, token + 8) pairs
+            const uint32_t pp = pack_h2(p0, p1);
+            const uint32_t x = __shfl_sync(kFull, pp, (c << 3) | (g & 3));
+            const uint32_t y = __shfl_sync(kFull, pp, (c << 3) | 4 | (g & 3));
+            const uint32_t pb0 = (g < 4) ? __byte_perm(x, y, 0x5410) : 0u;
+            const uint32_t pb1 = (g < 4) ? __byte_perm(x, y, 0x7632) : 0u;
             // ---- O^T += V^T P : rows = dims 16g + 2t (+1), k = tokens
             const uint32_t w0[2] = {v0.x, v0.y}, w1[2] = {v1.x, v1.y};
             const uint32_t w2[2] = {v2.x, v2.y}, w3[2] = {v3.x, v3.y};
@@ -453,6 +454,10 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
                 for (int j = 0; j < 4; ++j)
                     mma16816(o[4 * wi + j], hmul2(rl01[j], vs01), hmul2(rh01[j], vs01), hmul2(rl89[j], vs89),
                              hmul2(rh89[j], vs89), pb0, pb1);
+            }
+            if (++st == kST) {
+                st = 0;
+                ph ^= 1u;
             }
         }
     }
