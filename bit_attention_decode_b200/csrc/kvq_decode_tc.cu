@@ -312,6 +312,7 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
                 }
             }
         const float isg = __shfl_sync(kFull, isig, 8 * c);   // head c's normalisation (lane g = 2c)
+        float thr = -INFINITY;   // raw-score threshold (m + 8) / isg past which m moves
 
         const uint8_t* my_tile = smem + h * kTB;
         int st = 0;
@@ -404,15 +405,15 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
             // weight above 2^8), so most pages skip the cross-lane max and the
             // rescale.  Any common reference gives the same o / l; bounding the
             // weights by 2^8 keeps them, scaled by 2^7, inside fp16.
-            const float lm = fmaxf(s0, s1) * isg;
-            if (__any_sync(kFull, lm > m_h + 8.0f)) {
+            const float lm = fmaxf(s0, s1);
+            if (__any_sync(kFull, lm > thr)) {
                 float pm = lm;
 #pragma unroll
                 for (int x = 4; x < 32; x <<= 1) pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, x));
-                const float mn = fmaxf(m_h, pm);
+                const float mn = fmaxf(m_h, pm * isg);
                 const float al = fast_exp2(m_h - mn);
                 l_h *= al;
-                // output columns 2c, 2c + 1 are heads 2c, 2c + 1 (zero for c >= 2)
+                // output columns 2c, 2c + 1 are heads (2c) & 3, (2c + 1) & 3
                 const float al_a = __shfl_sync(kFull, al, (lane & ~3) | ((2 * c) & 3));
                 const float al_b = __shfl_sync(kFull, al, (lane & ~3) | ((2 * c + 1) & 3));
 #pragma unroll
@@ -421,20 +422,20 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
                     o[t][1] *= al_b; o[t][3] *= al_b;
                 }
                 m_h = mn;
+                thr = (mn + 8.0f) * __frcp_rn(isg);   // exact: isg is a power of two
             }
             // weights (<= 2^8 against the reference) scaled by 2^7 for the fp16 operand
             const float ca = 7.0f - m_h;
             const float p0 = fast_exp2(fmaf(s0, isg, ca)), p1 = fast_exp2(fmaf(s1, isg, ca));
             l_h += p0 + p1;
             // P (fp16, relative rounding <= 2^-11) as the B operand [tokens] x
-            // [4 heads | 4 zero columns]: lane (g, c) needs tokens 2c, 2c + 1
-            // (b0) and 2c + 8, 2c + 9 (b1) of head g, held by lanes (2c, g)
-            // and (2c + 1, g) as their (token, token + 8) pairs
+            // [4 heads | the same 4 heads again]: lane (g, c) needs tokens 2c,
+            // 2c + 1 (b0) and 2c + 8, 2c + 9 (b1) of head g & 3, held by lanes
+            // (2c, g & 3) and (2c + 1, g & 3) as their (token, token + 8) pairs
             const uint32_t pp = pack_h2(p0, p1);
             const uint32_t x = __shfl_sync(kFull, pp, (c << 3) | (g & 3));
             const uint32_t y = __shfl_sync(kFull, pp, (c << 3) | 4 | (g & 3));
-            const uint32_t pb0 = (g < 4) ? __byte_perm(x, y, 0x5410) : 0u;
-            const uint32_t pb1 = (g < 4) ? __byte_perm(x, y, 0x7632) : 0u;
+            const uint32_t pb0 = __byte_perm(x, y, 0x5410), pb1 = __byte_perm(x, y, 0x7632);
             // ---- O^T += V^T P : rows = dims 16g + 2t (+1), k = tokens
             const uint32_t w0[2] = {v0.x, v0.y}, w1[2] = {v1.x, v1.y};
             const uint32_t w2[2] = {v2.x, v2.y}, w3[2] = {v3.x, v3.y};
@@ -481,11 +482,8 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
     for (int x = 4; x < 32; x <<= 1) {
         l_h += __shfl_xor_sync(kFull, l_h, x);
     }
-#pragma unroll
-    for (int t = 0; t < 8; ++t)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) o[t][k] += __shfl_xor_sync(kFull, o[t][k], 2);
-    // lane (g, c) writes dims 16g..16g+15 of one head: c < 2 -> head 2c, else head 2(c-2)+1
+    // lane (g, c) writes dims 16g..16g+15 of one head: c < 2 -> head 2c (its
+    // column 2c), else head 2(c-2)+1 (its column 2c + 1, which repeats it)
     const int h = warp;
     const bool first = c < 2;
     const int head = first ? 2 * c : 2 * (c - 2) + 1;
