@@ -143,6 +143,27 @@ def test_long_sequence_many_splits(kvq):
     harness.check_attention(out[0, 0], want[0], "5000 tokens f32")
 
 
+@pytest.mark.parametrize("scale", [1.0 / 64, 3.0])
+def test_flat_and_peaked_softmax(kvq, scale):
+    # The decode keeps a lazy softmax reference that moves only when a score
+    # passes it by more than 8 (log2 units).  A near-uniform softmax (queries
+    # x 1/64: the reference never moves after the first page) and a peaked
+    # one (x 3: it moves often, by large steps) both match the oracle, on a
+    # split sequence (partials merged by the combine) and on unsplit ones.
+    w = small(num_layers=2, batch=3, calib_windows=1, calib_len=64)
+    lens = [3000, 45, 700]
+    p = harness.build_problem(kvq, w, lens=lens)
+    cal = harness.oracle_calibration(p)
+    q = torch.stack([synth.decode_queries(w, l, 0) for l in p.layers]).float() * scale
+    out = kvq.decode_attention(p.shape, p.calib, p.cache, q.cuda(), p.page_table.cuda(), p.lens.cuda(),
+                               out_dtype=torch.float32).cpu().numpy()
+    qh = q.numpy()
+    for li in range(2):
+        for b, n in enumerate(lens):
+            want = harness.oracle_attend(p, li, b, qh[li, b][None], n - 1, n, cal)
+            harness.check_attention(out[li, b], want[0], f"query x {scale} layer {li} seq {b}")
+
+
 def test_page_order_does_not_change_results(kvq):
     w = small(num_layers=1, batch=3, calib_windows=1, calib_len=64)
     lens = [40, 200, 77]
