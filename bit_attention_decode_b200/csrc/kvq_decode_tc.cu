@@ -326,7 +326,7 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
             const int nvalid = min(kPage, len - (p0 + i) * kPage);
             uint2 v0, v1, v2, v3;
             uint32_t vs01, vs89;
-            // ---- S = K q~ : tokens (rows) x [4 heads hi | 4 heads lo] (cols);
+            // ---- S = K q~ : tokens (rows) x [hi, lo of head 0, ..., hi, lo of head 3] (cols);
             // two accumulators (even / odd words) halve the dependent MMA chain
             float sacc[4] = {0.0f, 0.0f, 0.0f, 0.0f}, sacc2[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             if constexpr (KB) {
