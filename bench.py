@@ -569,8 +569,6 @@ def time_e2e(wl: Ragged, steps: int, world: int):
 def oracle_sample(seconds: float, layers=None):
     """Time the oracle on (layer, sequence) units of a ragged decode step until
     `seconds` pass; returns (tokens/s extrapolated to the full step, sample text)."""
-    import numpy as np
-
     import oracle
     import synth
     w = synth.WORKLOADS["ragged"]

@@ -30,7 +30,6 @@ copy of exactly the tensor the library saw.
 from __future__ import annotations
 
 import dataclasses
-import math
 from typing import Optional
 
 import torch
