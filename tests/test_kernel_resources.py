@@ -26,8 +26,12 @@ _spec.loader.exec_module(_build)
 SOURCES = ["kvq_decode_tc.cu", "kvq_quant.cu", "kvq_prefill_tc.cu", "kvq_prefill_fp4.cu", "kvq_klt.cu"]
 
 
+def _nvcc():
+    return _build.NVCC if os.path.exists(_build.NVCC) else shutil.which("nvcc")
+
+
 def _report(src, out_dir):
-    r = subprocess.run([_build.NVCC, *_build.FLAGS, "-Xptxas", "-v", "-c", os.path.join(_build.CSRC, src),
+    r = subprocess.run([_nvcc(), *_build.FLAGS, "-Xptxas", "-v", "-c", os.path.join(_build.CSRC, src),
                         "-o", os.path.join(out_dir, src + ".o")], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
     entries, cur = {}, None
@@ -50,7 +54,7 @@ def _report(src, out_dir):
 
 @pytest.fixture(scope="module")
 def resources():
-    if not os.path.exists(_build.NVCC) and shutil.which("nvcc") is None:
+    if _nvcc() is None:
         pytest.skip("nvcc not available")
     with tempfile.TemporaryDirectory() as d:
         with concurrent.futures.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
