@@ -96,7 +96,7 @@ class Problem:
 
 def build_problem(kvq, w: synth.Workload, lens, layers=None, extra_tokens: int = 0, shuffle: bool = True,
                   keep_host=True, device="cuda", gen_device="cpu", keep=None, all_layers_one_call=False,
-                  keep_tails=False, native=False, k_format=0, klt=False):
+                  keep_tails=False, native=False, k_format=0, klt=False, exclude_pos0=True):
     """Calibrate, then append each sequence's first lens[b] tokens.
 
     keep:      optional set of (layer index, sequence) whose host copies are kept
@@ -107,7 +107,14 @@ def build_problem(kvq, w: synth.Workload, lens, layers=None, extra_tokens: int =
                device, as tails_k/v [extra][nl][B][Hkv][D].
     native:    calibrate the keys in their native basis (no smoothing).
     k_format:  1 for the mixed cache (bf16 keys, NVFP4 values).
-    klt:       smoothing plus the static per-head KLT (kvq.calibrate_klt).
+    klt:       smoothing plus the static per-head KLT.  The library runs on the
+               oracle's own calibration (fp64 eigh basis rounded to fp32, its
+               smoothing and tensor scales), written into a caller-owned
+               Calibration, so no value the oracle reads comes from the
+               device.  kvq_calibrate_klt itself is checked as a calibration
+               in tests/test_gpu_klt.py.
+    exclude_pos0: leave position 0 of every window out of the smoothing
+               absmax (and of the KLT's second moment).
     """
     layers = list(range(w.num_layers)) if layers is None else list(layers)
     lens = torch.as_tensor(lens, dtype=torch.int32)
@@ -118,12 +125,19 @@ def build_problem(kvq, w: synth.Workload, lens, layers=None, extra_tokens: int =
     kc = torch.stack([x[0] for x in wins])
     vc = torch.stack([x[1] for x in wins])
     del wins
+    klt_cal = klt_U = None
     if klt:
-        calib = kvq.calibrate_klt(shape, kc.to(device).contiguous(), vc.to(device).contiguous())
+        kh, vh = kc.float().cpu().numpy(), vc.float().cpu().numpy()
+        s_o, inv_o, klt_U, _ = oracle.calibrate_klt(kh, vh, exclude_pos0=exclude_pos0)
+        gk_o, gv_o = oracle.klt_tensor_scales(kh, vh, inv_o, klt_U)
+        klt_cal = (s_o, inv_o, gk_o, gv_o)
+        calib = kvq.Calibration(*(torch.from_numpy(np.ascontiguousarray(x)).to(device) for x in klt_cal),
+                                k_klt=torch.from_numpy(klt_U).to(device))
     elif native:
         calib = kvq.calibrate_native(shape, kc.to(device).contiguous(), vc.to(device).contiguous())
     else:
-        calib = kvq.calibrate_smoothing(shape, kc.to(device).contiguous(), vc.to(device).contiguous())
+        calib = kvq.calibrate_smoothing(shape, kc.to(device).contiguous(), vc.to(device).contiguous(),
+                                        exclude_pos0=exclude_pos0)
     page_table, num_pages = synth.build_page_table(w, lens + extra_tokens, shuffle=shuffle)
     cache = kvq.new_cache(shape, num_pages, device)
     seqs = {}
@@ -162,17 +176,33 @@ def build_problem(kvq, w: synth.Workload, lens, layers=None, extra_tokens: int =
     p.native = native
     p.k_format = k_format
     p.klt = klt
+    p.klt_U = klt_U            # [nl][Hkv][128][128] fp32, the oracle's basis (klt only)
+    p.klt_cal = klt_cal
+    p.exclude_pos0 = exclude_pos0
     return p
 
 
 def oracle_calibration(p: Problem):
-    return oracle.calibrate(p.k_calib, p.v_calib, exclude_pos0=True, hadamard=p.w.hadamard,
-                            smooth=not getattr(p, "native", False))
+    """The oracle's calibration of the problem: (s, inv_s, g_K, g_V)."""
+    if getattr(p, "klt", False):
+        return p.klt_cal
+    return oracle.calibrate(p.k_calib, p.v_calib, exclude_pos0=getattr(p, "exclude_pos0", True),
+                            hadamard=p.w.hadamard, smooth=not getattr(p, "native", False))
 
 
 def calib_host(p: Problem):
+    """The library's calibration arrays, read back from the device."""
     return (p.calib.k_smooth.cpu().numpy(), p.calib.k_inv_smooth.cpu().numpy(),
             p.calib.k_gscale.cpu().numpy(), p.calib.v_gscale.cpu().numpy())
+
+
+def checked_calibration(p: Problem):
+    """The oracle's calibration, after checking the library's bit for bit
+    against it; every oracle comparison then runs on the oracle's values."""
+    cal = oracle_calibration(p)
+    for got, want, name in zip(calib_host(p), cal, ("s", "inv_s", "g_K", "g_V")):
+        np.testing.assert_array_equal(got, want, err_msg=f"calibration {name}")
+    return cal
 
 
 def oracle_sequence(p: Problem, li: int, b: int, n: int, cal):
@@ -184,8 +214,8 @@ def oracle_sequence(p: Problem, li: int, b: int, n: int, cal):
         vc, vsf = oracle.quantize_rows(v[:n], gv[li])
         return {"kc": oracle.round_bf16(k[:n]), "ksf": None, "vc": vc, "vsf": vsf}
     if getattr(p, "klt", False):
-        # smoothing, then the device's KLT basis in the fixed FMA order
-        U = p.calib.k_klt[li].cpu().numpy()
+        # smoothing, then the oracle's KLT basis in the fixed FMA order
+        U = p.klt_U[li]
         y = oracle.transform_keys(k[:n], inv[li])
         yk = np.stack([oracle.klt_apply(y[:, h], U[h]) for h in range(y.shape[1])], axis=1)
         kc, ksf = oracle.quantize_rows(yk, gk[li])
@@ -195,7 +225,8 @@ def oracle_sequence(p: Problem, li: int, b: int, n: int, cal):
 
 
 def oracle_attend(p: Problem, li: int, b: int, q_rows: np.ndarray, q_start: int, n: int, cal):
-    """Oracle attention of q_rows [Tq][Hq][D] over the first n tokens."""
+    """Oracle attention of q_rows [Tq][Hq][D] over the first n tokens
+    (cal: the oracle's calibration, oracle_calibration)."""
     s, inv, gk, gv = cal
     qz = oracle_sequence(p, li, b, n, cal)
     vx = oracle.dequantize_rows(qz["vc"], qz["vsf"], gv[li])
@@ -205,7 +236,7 @@ def oracle_attend(p: Problem, li: int, b: int, q_rows: np.ndarray, q_start: int,
     kx = oracle.dequantize_rows(qz["kc"], qz["ksf"], gk[li])
     if getattr(p, "klt", False):
         # the query rotated to match: q~ = U^T (q * s) per kv head, in fp64
-        U = p.calib.k_klt[li].cpu().numpy().astype(np.float64)
+        U = p.klt_U[li].astype(np.float64)
         G = q_rows.shape[1] // U.shape[0]
         qs = np.asarray(q_rows, np.float64) * np.repeat(np.asarray(s[li], np.float64), G, axis=0)[None]
         qt = np.einsum("thc,hci->thi", qs, np.repeat(U, G, axis=0))
@@ -215,14 +246,14 @@ def oracle_attend(p: Problem, li: int, b: int, q_rows: np.ndarray, q_start: int,
 
 def oracle_attend_fp4q(p: Problem, li: int, b: int, q_rows: np.ndarray, q_start: int, n: int, cal):
     """Oracle of the FP4 Q.K prefill: the query in the keys' basis (smoothing,
-    rotation or the device's KLT basis), quantised to NVFP4 per row by the
+    rotation or the oracle's KLT basis), quantised to NVFP4 per row by the
     oracle, dequantised exactly, then attended in fp64 against the
     dequantised cache."""
     s, inv, gk, gv = cal
     qz = oracle_sequence(p, li, b, n, cal)
     kx = oracle.dequantize_rows(qz["kc"], qz["ksf"], gk[li])
     vx = oracle.dequantize_rows(qz["vc"], qz["vsf"], gv[li])
-    U = p.calib.k_klt[li].cpu().numpy() if getattr(p, "klt", False) else None
+    U = p.klt_U[li] if getattr(p, "klt", False) else None
     y = oracle.query_rows_fp4(q_rows, s[li], hadamard=bool(p.w.hadamard) and U is None, U=U)
     qx = oracle.dequantize_query(*oracle.quantize_query(y))
     return oracle.attention_x(qx, q_start, kx, vx)

@@ -3,7 +3,8 @@ the bench uses, on sampled outputs the oracle computes one by one.
 
 Calibration is compared in full; codes and scales bit for bit on sampled
 (layer, sequence) pairs; attention rows within the tolerance of
-tests/harness.py.
+tests/harness.py, for bf16 output (the bench's) and for fp32 output at the
+strict max-abs bound (the same launch with the other output type).
 """
 import numpy as np
 import pytest
@@ -36,13 +37,15 @@ def test_prefix_append_and_one_decode_step(kvq, name):
     for (li, b) in sorted(keep):
         assert_codes_equal(p, li, b, w.context, cal)
     q = torch.stack([synth.decode_queries(w, l, 0, "cuda") for l in range(w.num_layers)])
-    out = kvq.decode_attention(p.shape, p.calib, p.cache, q, p.page_table.cuda(), p.lens.cuda(),
-                               out_dtype=torch.bfloat16).float().cpu().numpy()
+    outs = {tag: kvq.decode_attention(p.shape, p.calib, p.cache, q, p.page_table.cuda(), p.lens.cuda(),
+                                      out_dtype=dt).float().cpu().numpy()
+            for dt, tag in ((torch.bfloat16, "bf16"), (torch.float32, "f32"))}
     qh = q.float().cpu().numpy()
     n = w.context
     for (li, b) in sorted(keep):
         want = harness.oracle_attend(p, li, b, qh[li, b][None], n - 1, n, cal)
-        harness.check_attention(out[li, b], want[0], f"{name} layer {li} seq {b} bf16")
+        for tag, out in outs.items():
+            harness.check_attention(out[li, b], want[0], f"{name} layer {li} seq {b} {tag}")
 
 
 def test_ragged_decode_64_steps(kvq):
@@ -69,14 +72,17 @@ def test_ragged_decode_64_steps(kvq):
         out = kvq.decode_attention(p.shape, p.calib, p.cache, q, pt, seq_lens.cuda(), out_dtype=torch.bfloat16,
                                    status=status)
         if s in (0, S // 2 - 1, S - 1):
-            out = out.float().cpu().numpy()
+            outs = {"bf16": out.float().cpu().numpy(),
+                    "f32": kvq.decode_attention(p.shape, p.calib, p.cache, q, pt, seq_lens.cuda(),
+                                                out_dtype=torch.float32, status=status).cpu().numpy()}
             qh = q.float().cpu().numpy()
             for (li, b) in sorted(keep):
                 n = int(seq_lens[b])
                 if s == S - 1:
                     assert_codes_equal(p, li, b, n, cal)
                 want = harness.oracle_attend(p, li, b, qh[li, b][None], n - 1, n, cal)
-                harness.check_attention(out[li, b], want[0], f"ragged step {s} layer {li} seq {b} len {n} bf16")
+                for tag, o in outs.items():
+                    harness.check_attention(o[li, b], want[0], f"ragged step {s} layer {li} seq {b} len {n} {tag}")
     torch.cuda.synchronize()
     assert status.item() == 0
 
@@ -91,15 +97,19 @@ def test_chunked_prefill(kvq):
     cal = check_calibration(p)
     q = torch.stack([synth.prefill_queries(w, l, "cuda") for l in range(w.num_layers)])   # [L][B][Tq][Hq][D]
     q_start = torch.full((B,), P0, dtype=torch.int32, device="cuda")
-    out = kvq.prefill_attention(p.shape, p.calib, p.cache, q, q_start, p.page_table.cuda(), p.lens.cuda(),
-                                out_dtype=torch.bfloat16)
     rows = [0, 1, 255, Tq - 1]
-    out_h = out[:, :, rows].float().cpu().numpy()
+    outs = {}
+    for dt, tag in ((torch.bfloat16, "bf16"), (torch.float32, "f32")):
+        out = kvq.prefill_attention(p.shape, p.calib, p.cache, q, q_start, p.page_table.cuda(), p.lens.cuda(),
+                                    out_dtype=dt)
+        outs[tag] = out[:, :, rows].float().cpu().numpy()
+        del out
     for (li, b) in sample:
         qh = q[li, b, rows].float().cpu().numpy()
         for r_i, r in enumerate(rows):
             want = harness.oracle_attend(p, li, b, qh[r_i][None], P0 + r, lens[b], cal)
-            harness.check_attention(out_h[li, b, r_i], want[0], f"prefill layer {li} seq {b} row {r} bf16")
+            for tag, out_h in outs.items():
+                harness.check_attention(out_h[li, b, r_i], want[0], f"prefill layer {li} seq {b} row {r} {tag}")
 
 
 @pytest.mark.parametrize("variant", ["klt", "bf16_keys"])
@@ -109,7 +119,9 @@ def test_ragged_variants_full_size(kvq, variant):
     # and NVFP4 values (bench.py --k-format bf16), as the bench launches them:
     # one step appended into all 36 layers, then all 36 layers decoded.
     # Codes and scales bit for bit and attention rows within tolerance, on
-    # sampled (layer, sequence) pairs.
+    # sampled (layer, sequence) pairs.  The KLT variant runs on the oracle's
+    # calibration (its eigh basis, smoothing and tensor scales written into
+    # the Calibration), so the oracle reads no device value.
     w = synth.WORKLOADS["ragged"]
     lens = synth.ragged_lengths(w)
     order = torch.argsort(lens)
@@ -117,19 +129,21 @@ def test_ragged_variants_full_size(kvq, variant):
     keep = {(l, b) for l in (0, 35) for b in sample_seqs}
     p = harness.build_problem(kvq, w, lens=lens, extra_tokens=1, gen_device="cuda", keep=keep, keep_tails=True,
                               klt=(variant == "klt"), k_format=(1 if variant == "bf16_keys" else 0))
-    cal = harness.calib_host(p)
+    cal = harness.checked_calibration(p)
     tk, tv = p.tails
     slots = synth.slot_mapping(p.page_table, torch.arange(w.batch), lens.long()).cuda()
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     kvq.quantize_append(p.shape, p.calib, p.cache, tk[0].contiguous(), tv[0].contiguous(), slots, status=status)
     seq_lens = (lens + 1).to(torch.int32)
     q = torch.stack([synth.decode_queries(w, l, 0, "cuda") for l in range(w.num_layers)])
-    out = kvq.decode_attention(p.shape, p.calib, p.cache, q, p.page_table.cuda(), seq_lens.cuda(),
-                               out_dtype=torch.bfloat16, status=status).float().cpu().numpy()
+    outs = {tag: kvq.decode_attention(p.shape, p.calib, p.cache, q, p.page_table.cuda(), seq_lens.cuda(),
+                                      out_dtype=dt, status=status).float().cpu().numpy()
+            for dt, tag in ((torch.bfloat16, "bf16"), (torch.float32, "f32"))}
     assert status.item() == 0
     qh = q.float().cpu().numpy()
     for (li, b) in sorted(keep):
         n = int(seq_lens[b])
         assert_codes_equal(p, li, b, n, cal)
         want = harness.oracle_attend(p, li, b, qh[li, b][None], n - 1, n, cal)
-        harness.check_attention(out[li, b], want[0], f"ragged {variant} layer {li} seq {b} len {n} bf16")
+        for tag, out in outs.items():
+            harness.check_attention(out[li, b], want[0], f"ragged {variant} layer {li} seq {b} len {n} {tag}")

@@ -97,6 +97,29 @@ def test_native_basis_keys(kvq, hadamard):
             harness.check_attention(out[li, b], want[0], f"native layer {li} seq {b} len {n}")
 
 
+@pytest.mark.parametrize("hadamard", [False, True])
+def test_sink_included_smoothing(kvq, hadamard):
+    # "NVFP4 attention cache on W4A4 Qwen3-8B", results table row "K: same
+    # smoothing, but sink token included in the absmax" (observation 2):
+    # kvq_calibrate_smoothing with exclude_pos0 = 0, then append and decode
+    w = small(num_layers=2, batch=3, calib_windows=2, calib_len=64, hadamard=hadamard)
+    lens = [9, 140, 301]
+    p = harness.build_problem(kvq, w, lens=lens, exclude_pos0=False)
+    cal = harness.checked_calibration(p)
+    # the sink (x40) now sets the absmax of its channels
+    s_ex = oracle.calibrate(p.k_calib, p.v_calib, exclude_pos0=True, hadamard=hadamard)[0]
+    assert np.all(cal[0] >= s_ex) and np.any(cal[0] > s_ex)
+    for li in range(2):
+        for b, n in enumerate(lens):
+            assert_codes_equal(p, li, b, n, cal)
+    for dt, tag in ((torch.float32, "f32"), (torch.bfloat16, "bf16")):
+        q, out = decode_all(kvq, p, out_dtype=dt)
+        for li in range(2):
+            for b, n in enumerate(lens):
+                want = harness.oracle_attend(p, li, b, q[li, b][None], n - 1, n, cal)
+                harness.check_attention(out[li, b], want[0], f"sink-included layer {li} seq {b} {tag}")
+
+
 @pytest.mark.parametrize("name", ["tiny", "qwen3_8b"])
 def test_mixed_cache_bf16_keys(kvq, name):
     # "NVFP4 attention cache on W4A4 Qwen3-8B", results table row "NVFP4 V

@@ -41,7 +41,7 @@ def test_fp4_prefill_ragged(kvq, variant):
     P0, Tq = [100, 33], 80
     lens = [n + Tq for n in P0]
     p = harness.build_problem(kvq, w, lens=lens, klt=(variant == "klt"))
-    cal = harness.calib_host(p)
+    cal = harness.checked_calibration(p)
     q = torch.stack([synth.prefill_queries(w, l) for l in p.layers])        # [nl][B][Tq][Hq][D]
     q_start = torch.tensor(P0, dtype=torch.int32)
     for dt, tag in ((torch.float32, "f32"), (torch.bfloat16, "bf16")):
@@ -59,7 +59,7 @@ def test_fp4_prefill_bf16_query_and_small_groups(kvq):
     P0, Tq = [7, 130], 40
     lens = [n + Tq for n in P0]
     p = harness.build_problem(kvq, w, lens=lens)
-    cal = harness.calib_host(p)
+    cal = harness.checked_calibration(p)
     q = synth.prefill_queries(w, 0)[None].to(torch.bfloat16)
     out = _run(kvq, p, q, torch.tensor(P0, dtype=torch.int32), torch.float32)
     for b in range(2):
@@ -74,7 +74,7 @@ def test_fp4_prefill_query_quantisation_error(kvq, capsys):
     P0, Tq = [200, 64], 64
     lens = [n + Tq for n in P0]
     p = harness.build_problem(kvq, w, lens=lens)
-    cal = harness.calib_host(p)
+    cal = harness.checked_calibration(p)
     q = torch.stack([synth.prefill_queries(w, l) for l in p.layers])
     out = _run(kvq, p, q, torch.tensor(P0, dtype=torch.int32), torch.float32)
     err_q, err_x, ref = [], [], []
@@ -104,18 +104,22 @@ def test_fp4_prefill_full_config_sampled(kvq):
     sample = [(0, 0), (35, B - 1)]
     lens = [P0 + Tq] * B
     p = harness.build_problem(kvq, w, lens=lens, gen_device="cuda", keep=set(sample))
-    cal = harness.calib_host(p)
+    cal = harness.checked_calibration(p)
     q = torch.stack([synth.prefill_queries(w, l, "cuda") for l in range(w.num_layers)])
     q_start = torch.full((B,), P0, dtype=torch.int32, device="cuda")
-    out = kvq.prefill_attention(p.shape, p.calib, p.cache, q, q_start, p.page_table.cuda(), p.lens.cuda(),
-                                out_dtype=torch.bfloat16, qk_fp4=True)
     rows = [0, 1, 255, Tq - 1]
-    out_h = out[:, :, rows].float().cpu().numpy()
+    outs = {}
+    for dt, tag in ((torch.bfloat16, "bf16"), (torch.float32, "f32")):
+        out = kvq.prefill_attention(p.shape, p.calib, p.cache, q, q_start, p.page_table.cuda(), p.lens.cuda(),
+                                    out_dtype=dt, qk_fp4=True)
+        outs[tag] = out[:, :, rows].float().cpu().numpy()
+        del out
     for (li, b) in sample:
         qh = q[li, b, rows].float().cpu().numpy()
         for r_i, r in enumerate(rows):
             want = harness.oracle_attend_fp4q(p, li, b, qh[r_i][None], P0 + r, lens[b], cal)
-            harness.check_attention(out_h[li, b, r_i], want[0], f"fp4 prefill layer {li} seq {b} row {r} bf16")
+            for tag, out_h in outs.items():
+                harness.check_attention(out_h[li, b, r_i], want[0], f"fp4 prefill layer {li} seq {b} row {r} {tag}")
 
 
 def test_fp4_prefill_edges(kvq):
@@ -123,7 +127,7 @@ def test_fp4_prefill_edges(kvq):
     w = _small(num_layers=1, batch=3, calib_windows=1, calib_len=64, prefill_chunk=1)
     lens = [128, 65, 0]
     p = harness.build_problem(kvq, w, lens=[128, 65, 1])
-    cal = harness.calib_host(p)
+    cal = harness.checked_calibration(p)
     q = synth.prefill_queries(w, 0)[None]                     # [1][3][1][Hq][D]
     q_start = torch.tensor([127, 64, 0], dtype=torch.int32)
     out = kvq.prefill_attention(p.shape, p.calib, p.cache, q.cuda(), q_start.cuda(), p.page_table.cuda(),
@@ -138,7 +142,7 @@ def test_fp4_prefill_edges(kvq):
 def test_fp4_prefill_device_faults_are_flagged(kvq):
     w = _small(num_layers=1, batch=2, calib_windows=1, calib_len=64, prefill_chunk=32)
     p = harness.build_problem(kvq, w, lens=[96, 96])
-    cal = harness.calib_host(p)
+    cal = harness.checked_calibration(p)
     q = synth.prefill_queries(w, 0)[None]
     q_start = torch.tensor([64, 64], dtype=torch.int32)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
