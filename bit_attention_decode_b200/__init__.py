@@ -29,7 +29,7 @@ PAGE_SIZE = 16
 TILE_BYTES = 2304
 
 KVQ_OK, KVQ_EINVAL, KVQ_ECUDA, KVQ_EUNSUPPORTED, KVQ_EWORKSPACE = 0, 1, 2, 3, 4
-DEV_BAD_PAGE, DEV_BAD_SLOT, DEV_BAD_LEN, DEV_TIMEOUT = 1, 2, 4, 8
+DEV_BAD_PAGE, DEV_BAD_SLOT, DEV_BAD_LEN, DEV_TIMEOUT, DEV_BAD_WORKSPACE = 1, 2, 4, 8, 16
 KVQ_F32, KVQ_BF16 = 0, 1
 K_NVFP4, K_BF16 = 0, 1          # kvq_shape.k_format: packed keys, or bf16 keys (mixed cache)
 
@@ -258,6 +258,13 @@ def quantize_append(shape: Shape, calib: Calibration, cache: PagedCache, k: torc
                                     slot_mapping.data_ptr(), T, _ptr(status), _stream()), "kvq_quantize_append")
 
 
+def new_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A workspace for decode_attention / prefill_attention: zero-filled, as
+    the split merge's counters at its start must be before the first call
+    (every call leaves them zero, so it can be reused for any later call)."""
+    return torch.zeros(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
 def decode_workspace_bytes(shape: Shape, nlayers: int, batch: int, max_pages_per_seq: int) -> int:
     return int(_lib.kvq_decode_workspace_bytes(ctypes.byref(shape.c()), nlayers, batch, max_pages_per_seq))
 
@@ -275,7 +282,7 @@ def decode_attention(shape: Shape, calib: Calibration, cache: PagedCache, q: tor
         out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
     need = decode_workspace_bytes(shape, nl, B, maxp)
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        workspace = new_workspace(need, q.device)
     _need_cuda(q, page_table, seq_lens, out, workspace, status)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_lib.kvq_decode_attention(ctypes.byref(shape.c()), ctypes.byref(calib.c()), ctypes.byref(cache.c()),
@@ -323,7 +330,7 @@ def prefill_attention(shape: Shape, calib: Calibration, cache: PagedCache, q: to
         out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
     need = prefill_workspace_bytes(shape, nl, B, Tq)
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        workspace = new_workspace(need, q.device)
     _need_cuda(q, q_start, page_table, seq_lens, out, workspace, status)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     name = "kvq_prefill_attention_fp4" if qk_fp4 else "kvq_prefill_attention"

@@ -7,6 +7,14 @@ namespace kvq {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kPartialStride = 132;  // floats per split partial: m, l, pad, pad, o[128]
+// The first bytes of every attention workspace: one arrival counter per
+// (layer, sequence) unit of a split decode.  They must hold zeros before the
+// first call and every decode leaves them zero (the last split of a unit
+// resets its counter), so a workspace is zero-filled once, when allocated.
+// Splits are used only below one wave of (layer, sequence) units (fewer than
+// 296), so 1024 counters always suffice.
+constexpr size_t kWsHeader = 4096;
+constexpr int kWsCounters = (int)(kWsHeader / sizeof(unsigned));
 
 struct AttnArgs {
     const uint8_t* cache;      // layer layer0
@@ -25,6 +33,7 @@ struct AttnArgs {
     int batch, q_len;
     void* out;
     float* partials;           // decode with splits > 1
+    unsigned* counters;        // decode with splits > 1: [nl][B] arrivals (workspace header)
     int splits, pps;
     int32_t* status;
 };

@@ -1,5 +1,6 @@
-// kvq_decode.cu -- host side of the attention calls (split plan, argument
-// block, launches) and the log-sum-exp combine of the decode splits.
+// kvq_decode.cu -- host side of the attention calls: split plan, workspace
+// layout, argument block, launches.  (The log-sum-exp merge of the decode
+// splits runs inside the decode kernel, in the last split of each unit.)
 //
 // The query carries the key smoothing: q~ = q * s (then H q~ / sqrt(128)
 // when keys are rotated), so q~ . T(k) = q . k -- "NVFP4 attention cache on
@@ -14,35 +15,6 @@
 #include "kvq_attn.cuh"
 
 namespace kvq {
-
-// Log-sum-exp merge of the split partials in split order.  A poisoned split
-// (bad page or length) zeroes the row.  grid (batch * Hq, nlayers), block 128.
-template <typename TO>
-__global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ partials, int splits,
-                                                      const float* __restrict__ gv, TO* __restrict__ out,
-                                                      int rows) {
-    const int row = blockIdx.x, li = blockIdx.y, d = threadIdx.x;
-    const float* base = partials + ((size_t)li * rows + row) * splits * kPartialStride;
-    float M = -INFINITY;
-    bool poison = false;
-    for (int s = 0; s < splits; ++s) {
-        const float ms = base[(size_t)s * kPartialStride];
-        poison |= (ms == INFINITY);
-        M = fmaxf(M, ms);
-    }
-    float L = 0.0f, acc = 0.0f;
-    if (!poison && M != -INFINITY) {
-        for (int s = 0; s < splits; ++s) {
-            const float* p = base + (size_t)s * kPartialStride;
-            const float w = (p[0] == -INFINITY) ? 0.0f : exp2f(p[0] - M);
-            L += w * p[1];
-            acc += w * p[4 + d];
-        }
-    }
-    const float r = (poison || L == 0.0f) ? 0.0f : acc / L * __ldg(gv + li);
-    TO* dst = out + ((size_t)li * rows + row) * kD + d;
-    if constexpr (sizeof(TO) == 4) *dst = r; else *dst = __float2bfloat16_rn(r);
-}
 
 // ------------------------------------------------------------------ host side
 DecodePlan decode_plan(const kvq_shape& s, int nlayers, int batch, int max_pages) {
@@ -80,7 +52,9 @@ DecodePlan decode_plan(const kvq_shape& s, int nlayers, int batch, int max_pages
     return {pps, splits};
 }
 
-// workspace: split partials, then (KLT cache) the transformed queries
+// Workspace of a decode: the counter header (kWsHeader bytes, zero between
+// calls), the split partials, then (KLT cache) the transformed queries.  No
+// workspace at all when neither partials nor queries are needed.
 static size_t partial_bytes(const kvq_shape& s, int nlayers, int batch, int max_pages) {
     DecodePlan p = decode_plan(s, nlayers, batch, max_pages);
     if (p.splits == 1) return 0;
@@ -90,8 +64,10 @@ static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 size_t decode_workspace(const kvq_shape& s, int nlayers, int batch, int max_pages) {
     const size_t part = partial_bytes(s, nlayers, batch, max_pages);
-    if (!s.use_klt) return part;
-    return align256(part) + (size_t)nlayers * batch * s.num_q_heads * kD * sizeof(float);
+    if (part == 0 && !s.use_klt) return 0;
+    size_t n = kWsHeader + align256(part);
+    if (s.use_klt) n += (size_t)nlayers * batch * s.num_q_heads * kD * sizeof(float);
+    return n;
 }
 
 static AttnArgs make_args(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cache, int layer0,
@@ -128,13 +104,15 @@ kvq_status decode(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cache
     a.splits = p.splits;
     a.pps = p.pages_per_split;
     a.q_len = 1;
-    a.partials = reinterpret_cast<float*>(ws);
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    a.counters = reinterpret_cast<unsigned*>(wsb);
+    a.partials = wsb ? reinterpret_cast<float*>(wsb + kWsHeader) : nullptr;
     bool qb = q_dtype == KVQ_BF16;
     const bool ob = out_dtype == KVQ_BF16;
+    if (p.splits > 1 && (long)nlayers * batch > kWsCounters) return KVQ_EINVAL;   // not reached by the plan
     if (s.use_klt) {
         // the queries, rotated by the KLT (and smoothed), go through the workspace
-        float* qt = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
-                                             align256(partial_bytes(s, nlayers, batch, max_pages)));
+        float* qt = reinterpret_cast<float*>(wsb + kWsHeader + align256(partial_bytes(s, nlayers, batch, max_pages)));
         const kvq_status r = klt_queries(s, c, layer0, nlayers, q, q_dtype, batch, qt, st);
         if (r != KVQ_OK) return r;
         a.q = qt;
@@ -142,18 +120,14 @@ kvq_status decode(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cache
         qb = false;
     }
     if (launch_decode_tc(a, nlayers, qb, ob, st) != cudaSuccess) return KVQ_ECUDA;
-    if (p.splits > 1) {
-        dim3 g2(batch * s.num_q_heads, nlayers);
-        if (ob) combine_kernel<__nv_bfloat16><<<g2, kD, 0, st>>>(a.partials, p.splits, a.gv, (__nv_bfloat16*)out, batch * s.num_q_heads);
-        else combine_kernel<float><<<g2, kD, 0, st>>>(a.partials, p.splits, a.gv, (float*)out, batch * s.num_q_heads);
-    }
     return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ECUDA;
 }
 
 size_t prefill_workspace(const kvq_shape& s, int nlayers, int batch, int q_len) {
-    // KLT cache: the rotated queries
+    // KLT cache: the rotated queries, after the header a decode's counters
+    // use (untouched here, so one workspace can serve both calls)
     if (!s.use_klt) return 0;
-    return (size_t)nlayers * batch * q_len * s.num_q_heads * kD * sizeof(float);
+    return kWsHeader + (size_t)nlayers * batch * q_len * s.num_q_heads * kD * sizeof(float);
 }
 
 kvq_status prefill(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cache, int layer0, int nlayers,
@@ -166,7 +140,7 @@ kvq_status prefill(const kvq_shape& s, const kvq_calib& c, const kvq_cache& cach
     bool qb = q_dtype == KVQ_BF16;
     const bool ob = out_dtype == KVQ_BF16;
     if (s.use_klt) {
-        float* qt = reinterpret_cast<float*>(ws);
+        float* qt = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kWsHeader);
         const kvq_status r = klt_queries(s, c, layer0, nlayers, q, q_dtype, batch * q_len, qt, st);
         if (r != KVQ_OK) return r;
         a.q = qt;

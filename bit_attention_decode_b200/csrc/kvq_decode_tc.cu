@@ -71,6 +71,10 @@ __device__ __forceinline__ float2 unpack_h2(uint32_t a) {
 }
 __device__ __forceinline__ uint32_t bcast_lo(uint32_t h2) { return (h2 & 0xFFFFu) | (h2 << 16); }
 __device__ __forceinline__ uint32_t bcast_hi(uint32_t h2) { return (h2 & 0xFFFF0000u) | (h2 >> 16); }
+// barrier of the consumer warps alone (the producer warp has exited)
+__device__ __forceinline__ void consumers_sync(int threads) {
+    asm volatile("bar.sync 1, %0;" ::"r"(threads) : "memory");
+}
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -125,6 +129,72 @@ __device__ __forceinline__ void store16(__nv_bfloat16* p, const float* x) {
     reinterpret_cast<uint4*>(p)[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
+// ------------------------------------------------------------------ split merge
+// Log-sum-exp merge of one query head's split partials (m: reference in log2
+// units, INFINITY for a poisoned split, -INFINITY for an empty one; l: sum of
+// weights; o: weighted values) in split order, scaled by g_V / l; a lane
+// handles 4 dims.  A poisoned or empty row is written as zeros.
+__device__ __forceinline__ void store4(float* p, const float* r) {
+    *reinterpret_cast<float4*>(p) = make_float4(r[0], r[1], r[2], r[3]);
+}
+__device__ __forceinline__ void store4(__nv_bfloat16* p, const float* r) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf2(r[0], r[1]), pack_bf2(r[2], r[3]));
+}
+template <typename TO>
+__device__ __forceinline__ void merge_store(const float* m, const float* l, const float4* o, int n, float gv,
+                                            TO* dst) {
+    float M = -INFINITY;
+    bool poison = false;
+    for (int sp = 0; sp < n; ++sp) {
+        poison |= (m[sp] == INFINITY);
+        M = fmaxf(M, m[sp]);
+    }
+    float L = 0.0f, acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (!poison && M != -INFINITY) {
+        for (int sp = 0; sp < n; ++sp) {
+            const float w = (m[sp] == -INFINITY) ? 0.0f : exp2f(m[sp] - M);
+            L += w * l[sp];
+            acc[0] += w * o[sp].x;
+            acc[1] += w * o[sp].y;
+            acc[2] += w * o[sp].z;
+            acc[3] += w * o[sp].w;
+        }
+    }
+    float r[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) r[k] = (poison || L == 0.0f) ? 0.0f : acc[k] / L * gv;
+    store4(dst, r);
+}
+// the same for any number of splits, read from the partials in two passes
+template <typename TO>
+__device__ __forceinline__ void merge_store_n(const float* base, int n, int lane, float gv, TO* dst) {
+    float M = -INFINITY;
+    bool poison = false;
+    for (int sp = 0; sp < n; ++sp) {
+        const float ms = __ldcg(base + (size_t)sp * kPartialStride);
+        poison |= (ms == INFINITY);
+        M = fmaxf(M, ms);
+    }
+    float L = 0.0f, acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (!poison && M != -INFINITY) {
+        for (int sp = 0; sp < n; ++sp) {
+            const float* ps = base + (size_t)sp * kPartialStride;
+            const float ms = __ldcg(ps);
+            const float w = (ms == -INFINITY) ? 0.0f : exp2f(ms - M);
+            L += w * __ldcg(ps + 1);
+            const float4 ov = __ldcg(reinterpret_cast<const float4*>(ps + 4) + lane);
+            acc[0] += w * ov.x;
+            acc[1] += w * ov.y;
+            acc[2] += w * ov.z;
+            acc[3] += w * ov.w;
+        }
+    }
+    float r[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) r[k] = (poison || L == 0.0f) ? 0.0f : acc[k] / L * gv;
+    store4(dst, r);
+}
+
 // ------------------------------------------------------------------ kernel
 // grid (splits, nlayers, batch); block 32 * (Hkv + 1); dynamic smem
 // kStages * Hkv * 2304 + barriers.
@@ -138,6 +208,8 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ int s_flags;    // 1: a bounded wait gave up
     __shared__ int s_issued;   // pages the producer issued
+    __shared__ int s_last;     // split merge: this CTA is the unit's last split to finish
+    __shared__ int s_badp;     // the producer met a page id outside the pool
 
     const int Hkv = a.Hkv;
     const uint32_t page_bytes = (uint32_t)Hkv * kTB;
@@ -178,23 +250,19 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
     if (threadIdx.x == 0) {
         s_flags = 0;
         s_issued = 0;
+        s_badp = 0;
         for (int s = 0; s < kST; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], Hkv);
         }
         mbar_fence_init();
-    }
-    int badp = 0;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const int pg = __ldg(pt + i);
-        badp |= (pg < 0 || pg >= a.num_pages);
-    }
-    badp = __syncthreads_or(badp);
-    if (threadIdx.x == 0) {
         if (bad_len && split == 0) set_status(a.status, KVQ_DEV_BAD_LEN);
-        if (badp) set_status(a.status, KVQ_DEV_BAD_PAGE);
     }
-    const bool poison = bad_len || badp;
+    __syncthreads();
+    // page ids are checked by the producer as it issues the copies (no
+    // up-front pass over the page table delays the first copy); a unit with a
+    // bad page is poisoned and its output discarded at the end
+    const bool poison = bad_len;
     const uint8_t* layer_base = a.cache + (size_t)li * a.layer_stride;
 
     // consumer state (kept in registers across the final barrier)
@@ -210,20 +278,33 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
             int i = 0;
             int st = 0;
             uint32_t ph = 0;          // parity of round i / kST
+            bool bad = false;
             for (; i < n; ++i) {
                 if (i >= kST && !mbar_wait(&empty[st], ph ^ 1u)) {
                     atomicOr(&s_flags, 1);
                     break;
                 }
                 const int pg = __ldg(pt + i);
-                mbar_arrive_expect_tx(&full[st], page_bytes);
-                bulk_g2s(smem + st * page_bytes, layer_base + (size_t)pg * page_bytes, page_bytes, &full[st]);
+                bad |= (pg < 0 || pg >= a.num_pages);
+                if (bad) {
+                    // a page outside the pool, here or earlier: nothing is
+                    // copied; the stage completes empty so the consumers
+                    // move on, and the unit's result is discarded
+                    mbar_arrive(&full[st]);
+                } else {
+                    mbar_arrive_expect_tx(&full[st], page_bytes);
+                    bulk_g2s(smem + st * page_bytes, layer_base + (size_t)pg * page_bytes, page_bytes, &full[st]);
+                }
                 if (++st == kST) {
                     st = 0;
                     ph ^= 1u;
                 }
             }
             s_issued = i;
+            if (bad) {
+                s_badp = 1;
+                set_status(a.status, KVQ_DEV_BAD_PAGE);
+            }
         }
     } else if (!poison) {
         // ---------------------------------------------------------- consumer
@@ -477,7 +558,7 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
     if (warp >= Hkv) return;
 
     // ------------------------------------------------------------------ epilogue
-    const bool dead = poison || timed_out;
+    const bool dead = poison || timed_out || s_badp != 0;
 #pragma unroll
     for (int x = 4; x < 32; x <<= 1) {
         l_h += __shfl_xor_sync(kFull, l_h, x);
@@ -490,26 +571,82 @@ __global__ void __launch_bounds__(288, 2) decode_tc_kernel(AttnArgs a) {
     // head's sum and reference live in lanes (g, head)
     const float l = __shfl_sync(kFull, l_h, (lane & ~3) | head);
     const float m = __shfl_sync(kFull, m_h, (lane & ~3) | head);
-    if (head >= a.G) return;
-    float r[16];
+    if (head < a.G) {
+        float r[16];
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-        r[2 * t] = first ? o[t][0] : o[t][1];
-        r[2 * t + 1] = first ? o[t][2] : o[t][3];
-    }
-    const int hq = h * a.G + head;
-    if (a.splits == 1) {
-        const float sc = (dead || l == 0.0f) ? 0.0f : __ldg(a.gv + li) / l;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) r[k] *= sc;
-        store16(reinterpret_cast<TO*>(a.out) + (((size_t)li * a.batch + b) * a.Hq + hq) * kD + 16 * g, r);
-    } else {
-        float* part = a.partials + ((((size_t)li * a.batch + b) * a.Hq + hq) * a.splits + split) * kPartialStride;
-        if (g == 0) {
-            part[0] = dead ? INFINITY : m;
-            part[1] = l;
+        for (int t = 0; t < 8; ++t) {
+            r[2 * t] = first ? o[t][0] : o[t][1];
+            r[2 * t + 1] = first ? o[t][2] : o[t][3];
         }
-        store16(part + 4 + 16 * g, r);
+        const int hq = h * a.G + head;
+        if (a.splits == 1) {
+            // (a poisoned unit may have computed on stale stages: select, not scale)
+            const bool zero = dead || l == 0.0f;
+            const float sc = zero ? 0.0f : __ldg(a.gv + li) / l;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) r[k] = zero ? 0.0f : r[k] * sc;
+            store16(reinterpret_cast<TO*>(a.out) + (((size_t)li * a.batch + b) * a.Hq + hq) * kD + 16 * g, r);
+        } else {
+            float* part = a.partials + ((((size_t)li * a.batch + b) * a.Hq + hq) * a.splits + split) * kPartialStride;
+            if (g == 0) {
+                part[0] = dead ? INFINITY : m;
+                part[1] = l;
+            }
+            store16(part + 4 + 16 * g, r);
+        }
+    }
+    if (a.splits == 1) return;
+
+    // ---- split merge, fused: the last split of a (layer, sequence) unit to
+    // arrive merges the partials of all its splits, in split order (so the
+    // result does not depend on which split came last), and resets the
+    // unit's arrival counter for the next call.
+    consumers_sync(32 * Hkv);                          // every partial of this CTA is written
+    if (threadIdx.x == 0) {
+        __threadfence();                               // ... and visible, before the arrival
+        unsigned* ctr = a.counters + (size_t)li * a.batch + b;
+        const unsigned old = atomicAdd(ctr, 1u);
+        const bool last = old + 1u == (unsigned)a.splits;
+        if (last) atomicExch(ctr, 0u);
+        // a counter that did not start at zero: the workspace header was not zero-filled
+        if (old >= (unsigned)a.splits) set_status(a.status, KVQ_DEV_BAD_WORKSPACE);
+        s_last = last;
+    }
+    consumers_sync(32 * Hkv);
+    if (!s_last) return;
+    __threadfence();
+    // warp h merges the G query heads of kv head h; lane covers dims 4 lane .. 4 lane + 3
+    const float gvl = __ldg(a.gv + li);
+    const size_t row0 = ((size_t)li * a.batch + b) * a.Hq + (size_t)h * a.G;   // first query head of the warp
+    TO* dst0 = reinterpret_cast<TO*>(a.out) + row0 * kD + 4 * lane;
+    if (a.splits == 2) {
+        // every load of the merge issued at once: one round trip to L2
+        float mv[4][2], lv[4][2];
+        float4 ov[4][2];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int sp = 0; sp < 2; ++sp) {
+                mv[j][sp] = -INFINITY;
+                lv[j][sp] = 0.0f;
+                ov[j][sp] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                if (j < a.G) {
+                    const float* ps = a.partials + ((row0 + j) * 2 + sp) * kPartialStride;
+                    mv[j][sp] = __ldcg(ps);
+                    lv[j][sp] = __ldcg(ps + 1);
+                    ov[j][sp] = __ldcg(reinterpret_cast<const float4*>(ps + 4) + lane);
+                }
+            }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (j >= a.G) break;
+            merge_store<TO>(mv[j], lv[j], ov[j], 2, gvl, dst0 + (size_t)j * kD);
+        }
+    } else {
+        for (int j = 0; j < a.G; ++j) {
+            const float* base = a.partials + (row0 + j) * a.splits * kPartialStride;
+            merge_store_n<TO>(base, a.splits, lane, gvl, dst0 + (size_t)j * kD);
+        }
     }
 }
 

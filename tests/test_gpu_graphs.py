@@ -60,8 +60,7 @@ def test_decode_step_graph_replay_matches_eager(kvq):
     q_buf = torch.empty_like(qs[0])
     len_buf = torch.empty(B, dtype=torch.int32, device="cuda")
     out_buf = torch.empty(q_buf.shape, dtype=torch.float32, device="cuda")
-    ws = torch.empty(max(1, kvq.decode_workspace_bytes(p.shape, nl, B, pt.shape[1])), dtype=torch.uint8,
-                     device="cuda")
+    ws = kvq.new_workspace(kvq.decode_workspace_bytes(p.shape, nl, B, pt.shape[1]))
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
 
     def step():
