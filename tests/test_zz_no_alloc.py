@@ -38,11 +38,9 @@ def _compare(kvq, p, step, out_dtype):
     kvq.decode_attention_noalloc(p.shape, p.calib, p.cache, q, pt, lens, out, status=status)
     torch.cuda.synchronize()
     assert status.item() == 0
-    tag = "bf16" if out_dtype == torch.bfloat16 else "f32"
-    for li in range(len(p.layers)):
-        for b in range(len(p.lens)):
-            harness.check_attention(out[li, b].float().cpu().numpy(), ref[li, b].float().cpu().numpy(),
-                                    f"noalloc layer {li} seq {b} {tag}")
+    # the same kernels with the same split plan, only the scratch differs:
+    # the results are identical
+    assert torch.equal(out, ref), (out - ref).abs().max().item()
 
 
 def test_noalloc_matches_workspace_decode_on_consecutive_calls(kvq):
@@ -56,12 +54,28 @@ def test_noalloc_matches_workspace_decode_on_consecutive_calls(kvq):
 
 
 def test_noalloc_rejects_problems_beyond_the_scratch(kvq):
-    import ctypes
-    # few (layer, sequence) units over very long sequences: many splits
-    shape = kvq.Shape(8, 32, 8)
-    need = kvq.decode_workspace_bytes(shape, 8, 22, 16384)
+    # few (layer, sequence) units over very long page tables: many splits,
+    # more partials than the static array holds.  Every buffer is real and
+    # sized for the problem (a 4-page cache, sequences of one token), so
+    # even a launch would stay in bounds; the call must refuse it.
+    L, B, maxp = 8, 22, 16384
+    shape = kvq.Shape(L, 32, 8)
+    need = kvq.decode_workspace_bytes(shape, L, B, maxp)
     assert need > kvq.NOALLOC_SCRATCH_BYTES
-    st = kvq._lib.kvq_decode_attention_noalloc(
-        ctypes.byref(shape.c()), ctypes.byref(kvq._Calib(16, 16, 16, 16)),
-        ctypes.byref(kvq._Cache(4096, 8 * 2304 * 4, 4)), 0, 8, 256, 1, 512, 16384, 768, 22, 1024, 1, None, None)
-    assert st == kvq.KVQ_EWORKSPACE
+    calib = kvq.new_calibration(shape)
+    calib.k_smooth.fill_(1.0)
+    calib.k_inv_smooth.fill_(1.0)
+    calib.k_gscale.fill_(1.0)
+    calib.v_gscale.fill_(1.0)
+    cache = kvq.new_cache(shape, 4)
+    cache.data.zero_()
+    q = torch.zeros(L, B, 32, 128, dtype=torch.float32, device="cuda")
+    pt = torch.zeros(B, maxp, dtype=torch.int32, device="cuda")
+    lens = torch.ones(B, dtype=torch.int32, device="cuda")
+    out = torch.full((L, B, 32, 128), 7.0, dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    with pytest.raises(kvq.KVQError) as e:
+        kvq.decode_attention_noalloc(shape, calib, cache, q, pt, lens, out, status=status)
+    assert e.value.status == kvq.KVQ_EWORKSPACE
+    torch.cuda.synchronize()
+    assert status.item() == 0 and torch.all(out == 7.0)     # nothing was launched
