@@ -35,12 +35,20 @@ constexpr float kInvSqrt128 = 0.08838834764831845f;
 constexpr float kTensorRange = 2688.0f;
 
 // ---------------------------------------------------------------- formats
-// Two fp32 values -> one byte of two E2M1 codes (hi -> high nibble).
-__device__ __forceinline__ uint32_t e2m1x2_rn(float hi, float lo) {
-    uint16_t r;
-    asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u16.u8 %0, t; }"
-        : "=h"(r) : "f"(hi), "f"(lo));
-    return r;
+// Eight fp32 values as four pairs -> four bytes of E2M1 codes, round to
+// nearest even, saturating at 6, sign kept: pair i -> byte i, its .x in the
+// low nibble.  Every quantiser of the library (the append, the KLT key
+// append, the FP4 query of the prefill) converts through this routine, and
+// kvq_round_e2m1 exposes it for an exhaustive check.
+__device__ __forceinline__ uint32_t e2m1x8_rn(float2 a, float2 b, float2 c, float2 d) {
+    uint32_t w;
+    asm("{ .reg .b8 b0, b1, b2, b3;\n"
+        "  cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1; cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n"
+        "  cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5; cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n"
+        "  mov.b32 %0, {b0, b1, b2, b3}; }"
+        : "=r"(w)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
+    return w;
 }
 
 // One fp32 value -> E4M3 code (round-to-nearest-even, saturating).

@@ -304,12 +304,6 @@ __global__ void klt_finalize_kernel(float* __restrict__ gk, float* __restrict__ 
 // (contiguous over a quarter-warp), 16 shared-memory wavefronts for 64 FMAs,
 // which keeps shared memory and the FMA pipe in balance.  The 4 lanes of a
 // 16-block are neighbours and share its absmax by two shuffles.
-__device__ __forceinline__ uint32_t klt_e2m1x2(float hi, float lo) {
-    uint16_t r;
-    asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u16.u8 %0, t; }" : "=h"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-
 constexpr int kKltTok = 64;   // tokens per append tile
 constexpr size_t kKltAppendSmem =
     (size_t)kD * kD * sizeof(float) + (size_t)kD * kKltTok * sizeof(float) + 128 * sizeof(float) +
@@ -394,8 +388,11 @@ klt_append_keys_kernel(const T* __restrict__ k, const int64_t* __restrict__ slot
                 m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
                 const uint32_t sf = e4m3_rn(__fmul_rn(m, enc));
                 const float r = rtab[sf & 0x7Fu];
-                const uint32_t w = klt_e2m1x2(__fmul_rn(acc[a][4 * gi + 1], r), __fmul_rn(acc[a][4 * gi], r)) |
-                                   (klt_e2m1x2(__fmul_rn(acc[a][4 * gi + 3], r), __fmul_rn(acc[a][4 * gi + 2], r)) << 8);
+                // two code bytes (the other two pairs of the routine are unused)
+                const uint32_t w =
+                    e2m1x8_rn(make_float2(__fmul_rn(acc[a][4 * gi], r), __fmul_rn(acc[a][4 * gi + 1], r)),
+                              make_float2(__fmul_rn(acc[a][4 * gi + 2], r), __fmul_rn(acc[a][4 * gi + 3], r)),
+                              make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)) & 0xFFFFu;
                 if (slot >= num_slots) {
                     if (dl == 0 && gi == 0) set_status(status, KVQ_DEV_BAD_SLOT);
                 } else if (slot >= 0) {

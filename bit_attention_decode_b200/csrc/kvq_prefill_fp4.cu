@@ -238,10 +238,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_fp4_kernel(AttnArgs a) {
                     const uint32_t sc = e4m3_rn(__fmul_rn(am, enc));
                     const float d = __fmul_rn(e4m3_to_f32(sc), g);
                     const float rr = d == 0.0f ? 0.0f : __frcp_rn(d);
-                    uint32_t w[2] = {0u, 0u};
+                    float2 z[8];
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        w[k >> 2] |= e2m1x2_rn(__fmul_rn(y[2 * k + 1], rr), __fmul_rn(y[2 * k], rr)) << (8 * (k & 3));
+                    for (int k = 0; k < 8; ++k) z[k] = make_float2(__fmul_rn(y[2 * k], rr), __fmul_rn(y[2 * k + 1], rr));
+                    const uint32_t w[2] = {e2m1x8_rn(z[0], z[1], z[2], z[3]), e2m1x8_rn(z[4], z[5], z[6], z[7])};
                     // 16 codes = 8 bytes at byte 8 * blk of the row
                     *reinterpret_cast<uint2*>(qt + fp4_off(r, blk >> 1) + (blk & 1) * 8) = make_uint2(w[0], w[1]);
                     sfw[blk >> 2] |= sc << (8 * (blk & 3));

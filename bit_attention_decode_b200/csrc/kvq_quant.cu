@@ -85,19 +85,6 @@ __global__ void calib_finalize_gscale_kernel(float* __restrict__ gk, float* __re
 }
 
 // ------------------------------------------------------------------ quantise
-// Eight fp32 pairs -> four bytes of E2M1 codes: pair i -> byte i, its .x in
-// the low nibble.
-__device__ __forceinline__ uint32_t e2m1x8_rn(float2 a, float2 b, float2 c, float2 d) {
-    uint32_t w;
-    asm("{ .reg .b8 b0, b1, b2, b3;\n"
-        "  cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1; cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n"
-        "  cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5; cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n"
-        "  mov.b32 %0, {b0, b1, b2, b3}; }"
-        : "=r"(w)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
-    return w;
-}
-
 // One 16-element block: E4M3 block scale from the absmax, then E2M1 codes.
 // enc = 1/(6 g); rtab[c] = 1/(val(c) g) for every scale code c (0 where the
 // product is zero), both computed once per tensor.
@@ -316,9 +303,23 @@ append_kernel(const T* __restrict__ k, const T* __restrict__ v, const int64_t* _
 }
 
 // ------------------------------------------------------------------ utilities
+// Each thread converts 8 consecutive inputs with the quantisers' own
+// e2m1x8_rn: even inputs go through the low-nibble operand, odd ones through
+// the high-nibble operand (a caller checks both by converting x and x + 1).
 __global__ void round_e2m1_kernel(const float* __restrict__ x, uint8_t* __restrict__ out, int64_t n) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-        out[i] = (uint8_t)(e2m1x2_rn(0.0f, x[i]) & 0xFu);
+    const int64_t groups = (n + 7) / 8;
+    for (int64_t gi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; gi < groups;
+         gi += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i0 = 8 * gi;
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = (i0 + k < n) ? x[i0 + k] : 0.0f;
+        const uint32_t w = e2m1x8_rn(make_float2(v[0], v[1]), make_float2(v[2], v[3]), make_float2(v[4], v[5]),
+                                     make_float2(v[6], v[7]));
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (i0 + k < n) out[i0 + k] = (uint8_t)((w >> (4 * k)) & 0xFu);
+    }
 }
 
 __global__ void round_e4m3_kernel(const float* __restrict__ x, uint8_t* __restrict__ out, int64_t n) {

@@ -81,7 +81,9 @@ enum {
     KVQ_DEV_BAD_PAGE = 1,   /* page-table entry outside [0, num_pages)      */
     KVQ_DEV_BAD_SLOT = 2,   /* slot_mapping entry beyond the cache          */
     KVQ_DEV_BAD_LEN = 4,    /* seq_len < 0, or beyond max_pages_per_seq*16  */
-    KVQ_DEV_TIMEOUT = 8     /* a bounded wait on a copy gave up             */
+    KVQ_DEV_TIMEOUT = 8,    /* a bounded wait on a copy gave up             */
+    KVQ_DEV_BAD_WORKSPACE = 16 /* the workspace's counter header was not    */
+                               /* zero-filled (see kvq_decode_attention)    */
 };
 
 enum { KVQ_F32 = 0, KVQ_BF16 = 1 };
@@ -221,7 +223,7 @@ kvq_status kvq_quantize_append(const kvq_shape* shape, const kvq_calib* calib, c
                                int32_t dtype, const int64_t* slot_mapping, int32_t num_tokens,
                                int32_t* dev_status, void* stream);
 
-/* Workspace bytes kvq_decode_attention needs for these sizes. */
+/* Workspace bytes kvq_decode_attention needs for these sizes (0: none). */
 size_t kvq_decode_workspace_bytes(const kvq_shape* shape, int32_t nlayers, int32_t batch,
                                   int32_t max_pages_per_seq);
 
@@ -235,7 +237,8 @@ size_t kvq_decode_workspace_bytes(const kvq_shape* shape, int32_t nlayers, int32
  * memory-bound on the 4-bit cache, as QServe's fused kernels are ([P3]
  * Kernels field): split-K over the pages of each sequence, dequantisation in
  * registers, online softmax with scale 1/sqrt(128), P.V, and a log-sum-exp
- * merge of the splits.
+ * merge of the splits (in the same launch: the last split of each (layer,
+ * sequence) to finish merges the partials of all of them, in split order).
  *
  *   q            [nlayers][batch][Hq][128], q_dtype, post-RoPE queries.
  *   page_table   [batch][max_pages_per_seq] int32 page ids (shared by all
@@ -243,12 +246,21 @@ size_t kvq_decode_workspace_bytes(const kvq_shape* shape, int32_t nlayers, int32
  *   seq_lens     [batch] int32 cached tokens attended by each sequence
  *                (0 gives a zero output row).
  *   out          [nlayers][batch][Hq][128], out_dtype.
- *   workspace    >= kvq_decode_workspace_bytes(...) bytes, 16-byte aligned;
- *                scratch for split partials, contents undefined after.
+ *   workspace    >= kvq_decode_workspace_bytes(...) bytes, 16-byte aligned
+ *                (may be NULL when that is 0).  Its first 4096 bytes are
+ *                arrival counters of the split merge: they must hold zeros
+ *                before the first call, and every call leaves them zero, so
+ *                zero-fill a workspace once when allocating it (one buffer
+ *                may then serve any sequence of decode and prefill calls).
+ *                The rest is scratch (split partials, rotated queries) whose
+ *                contents are undefined after the call.  A counter found
+ *                non-zero sets KVQ_DEV_BAD_WORKSPACE.  Calls that share a
+ *                workspace must not overlap on the GPU.
  * With KVQ_K_BF16 keys the query is used as given (no smoothing, no
  * rotation, no key tensor scale): scores are q . k / sqrt(128).
  * Errors: KVQ_EINVAL / KVQ_EWORKSPACE on the host; KVQ_DEV_BAD_PAGE and
- * KVQ_DEV_BAD_LEN on the device (the affected rows are written as zeros).
+ * KVQ_DEV_BAD_LEN on the device (the affected rows are written as zeros),
+ * KVQ_DEV_BAD_WORKSPACE (see workspace).
  */
 kvq_status kvq_decode_attention(const kvq_shape* shape, const kvq_calib* calib, const kvq_cache* cache,
                                 int32_t layer0, int32_t nlayers, const void* q, int32_t q_dtype,
@@ -257,7 +269,9 @@ kvq_status kvq_decode_attention(const kvq_shape* shape, const kvq_calib* calib, 
                                 void* workspace, size_t workspace_bytes, int32_t* dev_status,
                                 void* stream);
 
-/* Workspace bytes kvq_prefill_attention needs for these sizes. */
+/* Workspace bytes kvq_prefill_attention needs for these sizes (0: none;
+ * only a KLT cache needs one).  The workspace follows the rules of
+ * kvq_decode_attention's: its first 4096 bytes are left untouched. */
 size_t kvq_prefill_workspace_bytes(const kvq_shape* shape, int32_t nlayers, int32_t batch,
                                    int32_t q_len);
 
@@ -316,17 +330,21 @@ kvq_status kvq_prefill_attention_fp4(const kvq_shape* shape, const kvq_calib* ca
  * cudaMalloc's implicit device-wide synchronisation).  The pages have no
  * counterpart to this call; it exists only for such callers.
  *
- * Same arguments, results and errors as kvq_decode_attention.  The split-K
- * scratch is a static device array of KVQ_NOALLOC_SCRATCH_BYTES inside the
- * library, reserved on every GPU that loads it until the process exits; the
- * call allocates nothing.  A problem whose kvq_decode_workspace_bytes exceeds
- * that size returns KVQ_EWORKSPACE and launches nothing.
- *   - The first call on a device looks up the array's device address (once
- *     per device, with that device current); make that first call before
- *     any stream capture.
+ * Same arguments, results and errors as kvq_decode_attention, whose host
+ * checks run first.  The split-K scratch is a static device array of
+ * KVQ_NOALLOC_SCRATCH_BYTES inside the library, reserved on every GPU that
+ * loads it until the process exits; the call allocates nothing.  A problem
+ * whose kvq_decode_workspace_bytes exceeds that size returns KVQ_EWORKSPACE
+ * (after the argument checks) and launches nothing.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and keeps it for that device's context; make that
+ *     first call before any stream capture.  After a cudaDeviceReset the
+ *     next call looks the address up again: make it outside a capture too.
  *   - The array is shared by all calls on a device and keeps the last
- *     call's contents; the decode writes every partial before reading it, so
- *     no clearing is needed.  Calls whose GPU work overlaps (other streams,
+ *     call's contents.  It starts zero-filled (a static device array), which
+ *     is what the split merge's counters at its start need, and each call
+ *     leaves those counters zero again; the decode writes every partial
+ *     before reading it.  Calls whose GPU work overlaps (other streams,
  *     other host threads) race on the array: serialise them.
  */
 #define KVQ_NOALLOC_SCRATCH_BYTES (16u << 20)
@@ -338,11 +356,14 @@ kvq_status kvq_decode_attention_noalloc(const kvq_shape* shape, const kvq_calib*
                                         int32_t* dev_status, void* stream);
 
 /*
- * Elementwise format conversions with the kernels' own rounding routines
- * (the ones kvq_quantize_append uses), for checking them against a
- * reference.  x: [n] fp32 device array; codes: [n] bytes, one code per byte
- * (E2M1 in the low nibble; E4M3 as a byte).  Round-to-nearest-even,
- * saturating, sign kept.
+ * Elementwise format conversions with the kernels' own rounding routines,
+ * for checking them against a reference: kvq_round_e2m1 goes through the
+ * E2M1 routine every quantiser uses (the append, the KLT key append and the
+ * FP4 query of kvq_prefill_attention_fp4), eight values per call with even
+ * positions in its low-nibble operand and odd ones in its high-nibble
+ * operand; kvq_round_e4m3 through the E4M3 routine of the block scales.
+ * x: [n] fp32 device array; codes: [n] bytes, one code per byte (E2M1 in the
+ * low nibble; E4M3 as a byte).  Round-to-nearest-even, saturating, sign kept.
  */
 kvq_status kvq_round_e2m1(const float* x, uint8_t* codes, int64_t n, void* stream);
 kvq_status kvq_round_e4m3(const float* x, uint8_t* codes, int64_t n, void* stream);
