@@ -6,6 +6,10 @@ head_dim 128, batch 64 with lengths uniform on [1024, 8192], a paged NVFP4
 cache of 16-token pages in shuffled order.  One step = append one new token
 per sequence into every layer (kvq_quantize_append) + one decode of every
 layer (kvq_decode_attention).  The 64 steps of the workload are cycled.
+After the headline, the line's "secondary" entry carries the kernel numbers
+of the other workloads (chunked prefill with fp16 and FP4 Q.K, the qwen3_8b
+and hadamard prefix workloads), each measured with a few steps in the same
+run.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
 
@@ -35,6 +39,11 @@ FALLBACK_HBM_GBS = 6650.0
 TOKEN_LAYER_BYTES = 1152          # packed K+V codes and scales of 8 heads
 TOKEN_LAYER_BYTES_BF16K = 2624    # mixed cache: bf16 keys (8 x 256 B) + packed values (8 x 72 B)
 QO_BYTES_PER_SEQ_LAYER = 32 * 128 * 2 * 2   # bf16 query in + bf16 output
+# what the kernels compute in ("dtype" of the JSON line)
+DECODE_DTYPE = ("fp16 mma operands (exact e2m1 x e4m3 dequant, query split hi + lo, P rounded to fp16), "
+                "f32 accumulate")
+PREFILL_DTYPE_F16 = "fp16 tcgen05 operands (exact dequant, query split hi + lo, P fp16), f32 accumulate"
+PREFILL_DTYPE_FP4 = "nvfp4 Q.K (query quantised per row) + fp16 P.V, f32 accumulate"
 
 
 def parse():
@@ -56,6 +65,9 @@ def parse():
     ap.add_argument("--source-sha", action="store_true",
                     help="print the hash of the decode kernel's sources (the key of the committed ncu counters) and exit")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the other workloads' kernel numbers (prefill fp16 / FP4 Q.K, qwen3_8b, hadamard) "
+                         "measured after the headline")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--layers", type=int, default=36,
                     help="layers of the ragged workload (36; fewer only for profiling captures)")
@@ -194,18 +206,14 @@ def decode_source_sha() -> str:
 
 
 def ncu_traffic():
-    """Per-launch DRAM bytes of the decode kernel from the committed ncu summary,
-    or None when the kernel sources changed since that capture."""
-    path = os.path.join(ROOT, "profiles", "decode_ragged_ncu.md")
+    """Per-launch DRAM bytes of the decode kernel from the committed ncu
+    counters (profiles/decode_ragged_ncu.json), or None when the kernel's
+    sources changed since that capture."""
+    path = os.path.join(ROOT, "profiles", "decode_ragged_ncu.json")
     try:
-        sha = decode_source_sha()
-        vals = {}
         with open(path) as f:
-            for line in f:
-                if ":" in line and line.strip().startswith("- "):
-                    k, v = line.strip()[2:].split(":", 1)
-                    vals[k.strip()] = v.strip()
-        if vals.get("kernel_source_sha256_16") != sha:
+            vals = json.load(f)
+        if vals.get("kernel_source_sha256_16") != decode_source_sha():
             return None
         return float(vals["dram_bytes_per_full_launch"])
     except (OSError, KeyError, ValueError):
@@ -292,17 +300,8 @@ class Ragged:
             kvq.quantize_append(self.shape, self.calib, self.cache, kc_all, vc_all, prefix_slots, layer0=l)
             del ks, vs
             if l == L - 1:
-                # time the bulk append on the last layer: re-appending the same
-                # tokens rewrites identical bytes; launches go back to back so
-                # the queue never drains between them
-                torch.cuda.synchronize()
-                ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
-                ev[0].record()
-                for r in range(6):
-                    kvq.quantize_append(self.shape, self.calib, self.cache, kc_all, vc_all, prefix_slots, layer0=l)
-                    ev[r + 1].record()
-                torch.cuda.synchronize()
-                self.append_ms = [ev[r].elapsed_time(ev[r + 1]) for r in range(1, 6)]
+                # the last layer's prefix, kept to time the bulk append (time_bulk_append)
+                self.bulk = (kc_all, vc_all, prefix_slots, l)
             del kc_all, vc_all
         self.q = torch.stack([torch.stack([synth.decode_queries(w, l, s, dev) for l in range(L)])
                               for s in range(S)])                             # [S][L][B][Hq][D]
@@ -310,13 +309,27 @@ class Ragged:
         self.page_table_dev = self.page_table.to(dev)
         self.out = torch.empty(L, B, w.num_q_heads, D, dtype=torch.bfloat16, device=dev)
         need = kvq.decode_workspace_bytes(self.shape, L, B, self.page_table.shape[1])
-        self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-        # append (+ KLT keys) and decode (+ KLT queries), plus a combine when split
-        part = kvq.decode_workspace_bytes(kvq.Shape(L, w.num_q_heads, w.num_kv_heads), L, B, self.page_table.shape[1])
-        self.launches_per_step = (4 if klt else 2) + (1 if part else 0)
+        self.ws = kvq.new_workspace(need, dev)
+        # append (+ KLT keys) and decode (+ KLT queries); a split decode merges in the same launch
+        self.launches_per_step = 4 if klt else 2
         torch.cuda.synchronize()
         # bulk append of each layer's prefix (read bf16 K and V, write codes + scales)
         self.append_bytes = self.prefix_tokens * (2 * w.num_kv_heads * D * 2 + self.tlb)
+
+    def time_bulk_append(self, reps: int = 6):
+        """CUDA-event times of the bulk prefix append of one layer (1.54 GB moved
+        at 36 layers x 64 sequences): re-appending the same tokens rewrites
+        identical bytes; launches go back to back so the queue never drains."""
+        kc_all, vc_all, slots, l = self.bulk
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        ev[0].record()
+        for r in range(reps):
+            self.kvq.quantize_append(self.shape, self.calib, self.cache, kc_all, vc_all, slots, layer0=l)
+            ev[r + 1].record()
+        torch.cuda.synchronize()
+        # the first launch is a warm-up
+        self.append_ms = [ev[r].elapsed_time(ev[r + 1]) for r in range(1, reps)]
 
     def decode_bytes(self, s: int) -> int:
         valid = int(self.lens.sum()) + self.B * (s + 1)
@@ -422,8 +435,8 @@ class Prefix:
         self.pt = self.page_table.to(dev)
         self.out = torch.empty(L, B, w.num_q_heads, D, dtype=torch.bfloat16, device=dev)
         need = kvq.decode_workspace_bytes(self.shape, L, B, self.page_table.shape[1])
-        self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-        self.launches = 2 + (1 if need else 0)
+        self.ws = kvq.new_workspace(need, dev)
+        self.launches = 2
         self.append_bytes = L * B * T * (2 * H * D * 2 + TOKEN_LAYER_BYTES)
         self.decode_bytes = L * B * T * TOKEN_LAYER_BYTES + L * B * QO_BYTES_PER_SEQ_LAYER
         torch.cuda.synchronize()
@@ -623,77 +636,136 @@ def config_block(wl=None):
             "parallelism": "replicas (independent sequences per GPU)"}
 
 
-def other_workload(args, kvq, synth, rank, world):
-    """One JSON line for the chunked-prefill or prefix workloads."""
-    peak_hbm, hbm_kind = measured_peak()
+def tensor_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             pk = json.load(f)
-        peak_tf, tf_kind = float(pk["bf16_tflops"]), "measured (cuBLAS bf16 burst; fp16 runs at the same rate)"
-        peak_tf_sus = float(pk.get("bf16_tflops_sustained", peak_tf))
+        return (float(pk["bf16_tflops"]), float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                "measured (cuBLAS bf16 burst; fp16 runs at the same rate)")
     except (OSError, KeyError, ValueError):
-        peak_tf, tf_kind, peak_tf_sus = 1590.0, "fallback", 1400.0
+        return 1590.0, 1400.0, "fallback"
+
+
+def measure_prefill(kvq, synth, layers, k_format, qk_fp4, warm, steps, world):
+    """Chunked causal prefill: per-step times of the chunk append and of the
+    prefill launch, and the prefill kernel's roofline entry."""
+    wl = Prefill(kvq, synth, layers, k_format=k_format, qk_fp4=qk_fp4)
+    total, app_ms, pre_ms = time_two_kernels(wl.append, wl.attend, warm, steps, world)
+    peak_tf, peak_tf_sus, tf_kind = tensor_peaks()
+    pre = statistics.mean(pre_ms)
+    achieved = wl.flops / (pre / 1e3) / 1e12
+    if qk_fp4:
+        # half the algorithmic flops (Q.K) run on FP4 operands at 4x the bf16 rate
+        # (nominal 9 vs 2.25 PFLOP/s dense), half (P.V) on fp16 at the bf16 rate:
+        # the mix's peak is 2 / (1/4 + 1) = 1.6x the bf16 one
+        peak_tf, peak_tf_sus = 1.6 * peak_tf, 1.6 * peak_tf_sus
+        tf_kind += "; x1.6 for the FP4 Q.K / fp16 P.V mix (FP4 = 4x bf16, nominal ratio)"
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+            "frac": achieved / peak_tf, "frac_of_sustained": achieved / peak_tf_sus, "traffic": None,
+            "peak_source": tf_kind,
+            "kernel": "kvq prefill fp4 Q.K (tcgen05 mxf4nvf4 + f16)" if qk_fp4 else "kvq prefill (tcgen05)",
+            "alg_flops_per_launch": wl.flops,
+            "note": "algorithmic flops count 4 per attended (query head, key, dim)" +
+                    ("" if qk_fp4 else "; the kernel issues 1.5x that on the tensor pipe (query hi + lo)")}
+    out = {"total_ms": total, "append_ms": statistics.mean(app_ms), "prefill_ms": pre, "roofline": roof,
+           "tokens": wl.B * wl.Tq * steps, "L": wl.L, "k_format": wl.k_format}
+    del wl
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_prefix(kvq, synth, name, layers, warm, steps, world):
+    """Prefix workload (qwen3_8b or hadamard): per-step times of the bulk
+    append of every layer's prefix and of one decode step of every layer."""
+    wl = Prefix(kvq, synth, name, layers)
+    total, app_ms, dec_ms = time_two_kernels(wl.append, wl.decode, warm, steps, world)
+    peak_hbm, hbm_kind = measured_peak()
+    app, dec = statistics.mean(app_ms), statistics.mean(dec_ms)
+    out = {"total_ms": total, "append_ms": app, "decode_ms": dec, "B": wl.B, "T": wl.T, "L": wl.L,
+           "hadamard": wl.w.hadamard, "launches": wl.launches,
+           "decode": {"achieved": wl.decode_bytes / (dec / 1e3) / 1e9, "peak": peak_hbm, "unit": "GB/s",
+                      "frac": wl.decode_bytes / (dec / 1e3) / 1e9 / peak_hbm, "peak_source": hbm_kind,
+                      "alg_bytes_per_launch": wl.decode_bytes, "ms": dec},
+           "append": {"achieved": wl.append_bytes / (app / 1e3) / 1e9, "unit": "GB/s",
+                      "frac": wl.append_bytes / (app / 1e3) / 1e9 / peak_hbm,
+                      "alg_bytes_per_launch": wl.append_bytes, "ms": app}}
+    del wl
+    torch.cuda.empty_cache()
+    return out
+
+
+PREFILL_METRIC = "NVFP4-KV chunked causal prefill tokens/s; achieved tensor TFLOP/s vs B200 peak"
+PREFILL_WORKLOAD = ("chunked prefill: {L} layers, batch 8, 8192 cached + 512-token causal chunk, 32 q / 8 kv "
+                    "heads, head_dim 128")
+PREFIX_WORKLOAD = "{name}: {L} layers, batch {B} x {T} tokens; one step = quantise-append of the whole prefix + " \
+                  "one decode step"
+
+
+def other_workload(args, kvq, synth, rank, world):
+    """One JSON line for the chunked-prefill or prefix workloads."""
     warm = max(3, args.warmup)
     clock = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if args.workload == "prefill":
-        wl = Prefill(kvq, synth, args.layers, k_format=1 if args.k_format == "bf16" else 0, qk_fp4=args.qk == "fp4")
-        total, app_ms, pre_ms = time_two_kernels(wl.append, wl.attend, warm, args.steps, world)
+        qk_fp4 = args.qk == "fp4"
+        r = measure_prefill(kvq, synth, args.layers, 1 if args.k_format == "bf16" else 0, qk_fp4, warm,
+                            args.steps, world)
         clocks = clock.stop() if clock else None
-        total = max_over_ranks(total, world)
-        tokens = world * wl.B * wl.Tq * args.steps
-        pre = statistics.mean(pre_ms)
-        achieved = wl.flops / (pre / 1e3) / 1e12
-        if wl.qk_fp4:
-            # half the algorithmic flops (Q.K) run on FP4 operands at 4x the bf16 rate
-            # (nominal 9 vs 2.25 PFLOP/s dense), half (P.V) on fp16 at the bf16 rate:
-            # the mix's peak is 2 / (1/4 + 1) = 1.6x the bf16 one
-            peak_tf, peak_tf_sus = 1.6 * peak_tf, 1.6 * peak_tf_sus
-            tf_kind += "; x1.6 for the FP4 Q.K / fp16 P.V mix (FP4 = 4x bf16, nominal ratio)"
-        line = {"metric": "NVFP4-KV chunked causal prefill tokens/s; achieved tensor TFLOP/s vs B200 peak",
-                "value": tokens / (total / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-                "warmup": warm, "ms_per_step": total / args.steps, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "data": "synthetic",
-                "dtype": ("nvfp4 Q.K (query quantised per row) + f16 P.V, f32 accumulate" if wl.qk_fp4
-                          else "f16 mma (q split hi+lo), f32 accumulate"),
-                "config": {"workload": f"chunked prefill: {wl.L} layers, batch 8, 8192 cached + 512-token causal "
-                                       "chunk, 32 q / 8 kv heads, head_dim 128", "layers": wl.L,
-                           "kv_cache": "mixed: bf16 keys, nvfp4 values" if wl.k_format else "nvfp4",
-                           "qk": "fp4" if wl.qk_fp4 else "fp16"},
-                "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
-                             "frac": achieved / peak_tf, "frac_of_sustained": achieved / peak_tf_sus,
-                             "traffic": None, "peak_source": tf_kind,
-                             "kernel": "kvq prefill fp4 Q.K (tcgen05 mxf4nvf4 + f16)" if wl.qk_fp4
-                             else "kvq prefill (tcgen05)", "alg_flops_per_launch": wl.flops,
-                             "note": "algorithmic flops count 4 per attended (query head, key, dim)" +
-                                     ("" if wl.qk_fp4 else "; the kernel issues 1.5x that on the tensor pipe "
-                                                           "(query hi + lo)")},
-                "append_ms": statistics.mean(app_ms), "prefill_ms": pre, "gpu_launches": 2 * args.steps,
-                "clocks": clocks}
-    else:
-        wl = Prefix(kvq, synth, args.workload, args.layers)
-        total, app_ms, dec_ms = time_two_kernels(wl.append, wl.decode, warm, args.steps, world)
-        clocks = clock.stop() if clock else None
-        total = max_over_ranks(total, world)
-        app, dec = statistics.mean(app_ms), statistics.mean(dec_ms)
-        line = {"metric": METRIC, "value": world * wl.B * args.steps / (total / 1e3), "unit": "tokens/s",
+        total = max_over_ranks(r["total_ms"], world)
+        line = {"metric": PREFILL_METRIC, "value": world * r["tokens"] / (total / 1e3), "unit": "tokens/s",
                 "n_gpus": world, "steps": args.steps, "warmup": warm, "ms_per_step": total / args.steps,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "data": "synthetic",
+                "dtype": (PREFILL_DTYPE_FP4 if qk_fp4 else PREFILL_DTYPE_F16),
+                "config": {"workload": PREFILL_WORKLOAD.format(L=r["L"]), "layers": r["L"],
+                           "kv_cache": "mixed: bf16 keys, nvfp4 values" if r["k_format"] else "nvfp4",
+                           "qk": "fp4" if qk_fp4 else "fp16"},
+                "roofline": r["roofline"], "append_ms": r["append_ms"], "prefill_ms": r["prefill_ms"],
+                "gpu_launches": 2 * args.steps, "clocks": clocks}
+    else:
+        r = measure_prefix(kvq, synth, args.workload, args.layers, warm, args.steps, world)
+        clocks = clock.stop() if clock else None
+        total = max_over_ranks(r["total_ms"], world)
+        roof = dict(r["decode"], bound="hbm", traffic=None, kernel="kvq decode (split merge fused)")
+        line = {"metric": METRIC, "value": world * r["B"] * args.steps / (total / 1e3), "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": warm, "ms_per_step": total / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": DECODE_DTYPE,
                 "data": "synthetic",
-                "config": {"workload": f"{args.workload}: {wl.L} layers, batch {wl.B} x {wl.T} tokens; one step = "
-                                       "quantise-append of the whole prefix + one decode step",
-                           "hadamard": wl.w.hadamard},
-                "roofline": {"bound": "hbm", "achieved": wl.decode_bytes / (dec / 1e3) / 1e9, "peak": peak_hbm,
-                             "unit": "GB/s", "frac": wl.decode_bytes / (dec / 1e3) / 1e9 / peak_hbm, "traffic": None,
-                             "peak_source": hbm_kind, "kernel": "kvq decode", "alg_bytes_per_launch": wl.decode_bytes},
-                "append": {"achieved": wl.append_bytes / (app / 1e3) / 1e9, "unit": "GB/s",
-                           "frac": wl.append_bytes / (app / 1e3) / 1e9 / peak_hbm, "alg_bytes_per_launch":
-                           wl.append_bytes, "ms": app},
-                "decode_ms": dec, "gpu_launches": wl.launches * args.steps, "clocks": clocks}
+                "config": {"workload": PREFIX_WORKLOAD.format(name=args.workload, L=r["L"], B=r["B"], T=r["T"]),
+                           "hadamard": r["hadamard"]},
+                "roofline": roof, "append": r["append"], "decode_ms": r["decode_ms"],
+                "gpu_launches": r["launches"] * args.steps, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def secondary_workloads(kvq, synth, warm=3, steps=5):
+    """The other workloads' kernel numbers, measured in the same run as the
+    headline (each with its own clock samples), so they sit on the record
+    beside it: the chunked prefill with fp16 and with FP4 Q.K (36 layers,
+    batch 8, 8192 + 512 tokens) and the qwen3_8b and hadamard prefix
+    workloads (bulk append + one decode step).  Each workload is freed before
+    the next one is built."""
+    out = {}
+    for key, qk_fp4 in (("prefill_fp16_qk", False), ("prefill_fp4_qk", True)):
+        clock = ClockSampler(torch.cuda.current_device())
+        r = measure_prefill(kvq, synth, 36, 0, qk_fp4, warm, steps, 1)
+        roof = r["roofline"]
+        out[key] = {"workload": PREFILL_WORKLOAD.format(L=r["L"]), "steps": steps, "warmup": warm,
+                    "prefill_ms": r["prefill_ms"], "append_ms": r["append_ms"],
+                    "tflops": roof["achieved"], "peak": roof["peak"], "frac": roof["frac"],
+                    "frac_of_sustained": roof["frac_of_sustained"], "peak_source": roof["peak_source"],
+                    "dtype": PREFILL_DTYPE_FP4 if qk_fp4 else PREFILL_DTYPE_F16, "clocks": clock.stop()}
+    for name in ("qwen3_8b", "hadamard"):
+        clock = ClockSampler(torch.cuda.current_device())
+        r = measure_prefix(kvq, synth, name, 36, warm, steps, 1)
+        out[name] = {"workload": PREFIX_WORKLOAD.format(name=name, L=r["L"], B=r["B"], T=r["T"]),
+                     "steps": steps, "warmup": warm,
+                     "decode": {k: r["decode"][k] for k in ("ms", "achieved", "frac", "unit")},
+                     "append": {k: r["append"][k] for k in ("ms", "achieved", "frac", "unit")},
+                     "clocks": clock.stop()}
+    return out
 
 
 def main():
@@ -705,19 +777,23 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        vals = []
-        spent_total = 0.0
+        # each step: one bounded sample of the workload -- the oracle on
+        # (layer, sequence) units of one layer of a ragged decode step
+        vals, spent = [], []
         sample = ""
         for i in range(args.warmup + args.steps):
-            v, sample, spent = oracle_sample(max(1.0, args.cpu_seconds / 4), layers=[i % 36])
+            v, sample, sp = oracle_sample(max(1.0, args.cpu_seconds / 4), layers=[i % 36])
             if i >= args.warmup:
                 vals.append(v)
-                spent_total += spent
+                spent.append(sp)
         value = statistics.median(vals)
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": 64 / value * 1e3, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": config_block(), "impl": "reference",
+                "warmup": args.warmup, "ms_per_step": statistics.mean(spent) * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64 (fp32 quantiser, fp64 attention)",
+                "data": "synthetic", "config": config_block(), "impl": "reference",
+                "step": "one bounded sample: the oracle on (layer, sequence) units of one layer of a ragged "
+                        "decode step; value = its token-layer rate expressed as tokens/s of the whole step",
+                "full_step_ms_extrapolated": 64 / value * 1e3,
                 "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores(), "kind": "oracle",
                                  "sample": "per step: " + sample},
                 "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -734,6 +810,7 @@ def main():
     sys.stderr.write(f"[bench] setup {time.time() - t_setup:.1f} s, {wl.num_pages} pages, "
                      f"cache {wl.cache.data.numel() / 1e9:.2f} GB\n")
     clock = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    wl.time_bulk_append()
     total_ms, dec_ms, dec_bytes = time_device(wl, max(3, args.warmup), args.steps, world)
     clocks = clock.stop() if clock else None
     total_ms = max_over_ranks(total_ms, world)
@@ -745,10 +822,11 @@ def main():
     traffic = ncu_traffic() if wl.k_format == 0 and not wl.klt else None
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_block(wl),
+            "scaling": "weak", "vs_baseline": None, "dtype": DECODE_DTYPE, "data": "synthetic",
+            "config": config_block(wl),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
-                         "kernel": "kvq decode (+split combine)", "alg_bytes_per_launch": dec_bytes},
+                         "kernel": "kvq decode (split merge fused)", "alg_bytes_per_launch": dec_bytes},
             "append": append_entry(wl, peak),
             "gpu_launches": wl.launches_per_step * args.steps,
             "clocks": clocks}
@@ -757,9 +835,11 @@ def main():
         e_ms = max_over_ranks(e_ms, world)
         line["e2e"] = {"value": world * wl.B * args.steps / (e_ms / 1e3), "unit": "tokens/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del wl
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_secondary:
+        line["secondary"] = secondary_workloads(kvq, synth)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        del wl
-        torch.cuda.empty_cache()
         v, sample, _ = oracle_sample(args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores(), "kind": "oracle",
                                 "sample": sample}
