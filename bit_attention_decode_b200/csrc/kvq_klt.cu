@@ -216,20 +216,36 @@ __device__ __forceinline__ void klt_tile(const float* __restrict__ Yt, const flo
 
 constexpr size_t kKltTileSmem = (size_t)kD * kD * sizeof(float) + (size_t)kD * 64 * sizeof(float);
 
-// 8 consecutive elements (16-byte aligned for bf16, 32 for fp32) as fp32
-__device__ __forceinline__ void load8(const float* p, float* x) {
-    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-}
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float* x) {
-    const uint4 t = *reinterpret_cast<const uint4*>(p);
-    const uint32_t w[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        x[2 * j] = __uint_as_float(w[j] << 16);
-        x[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+// Eight consecutive key elements of one token, as loaded from global memory
+// (kept raw in registers until they are smoothed and transposed).
+template <typename T>
+struct Raw8;
+template <>
+struct Raw8<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float* p) {
+        a = __ldg(reinterpret_cast<const float4*>(p));
+        b = __ldg(reinterpret_cast<const float4*>(p) + 1);
     }
-}
+    __device__ __forceinline__ void zero() { a = b = make_float4(0.0f, 0.0f, 0.0f, 0.0f); }
+    __device__ __forceinline__ void unpack(float* x) const {
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    }
+};
+template <>
+struct Raw8<__nv_bfloat16> {
+    uint4 v;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { v = __ldg(reinterpret_cast<const uint4*>(p)); }
+    __device__ __forceinline__ void zero() { v = make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ void unpack(float* x) const {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            x[2 * j] = __uint_as_float(w[j] << 16);
+            x[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+    }
+};
 
 // Load U of (l, h) into shared memory.
 __device__ __forceinline__ void klt_load_basis(float* Us, const float* __restrict__ U) {
@@ -335,28 +351,41 @@ klt_append_keys_kernel(const T* __restrict__ k, const int64_t* __restrict__ slot
     const int tgi = 2 * (threadIdx.x >> 5) + (lane >> 4);   // token group: tokens 8 tgi .. + 7
     const int dl = lane & 15;                               // dims 4 dl .. + 3 and 64 + 4 dl .. + 3
     const int ntiles = (num_tokens + kKltTok - 1) / kKltTok;
-    for (int tile_i = blockIdx.x; tile_i < ntiles; tile_i += gridDim.x) {
+    // The next tile's key rows and slots are loaded one tile ahead, into
+    // registers, so their global-memory latency overlaps this tile's
+    // transform.  Rows of 8 elements: 64 tokens x 16 groups; neighbouring
+    // lanes take neighbouring tokens, so the transposed stores hit distinct
+    // banks.
+    constexpr int kRowLoads = kKltTok * 16 / 128;
+    static_assert(kRowLoads * 128 == kKltTok * 16, "128 threads");
+    const int rr = threadIdx.x & (kKltTok - 1), cg = threadIdx.x >> 6;   // token, first 8-group
+    Raw8<T> raw[kRowLoads];
+    int64_t nslot = -1;
+    auto fetch = [&](int tile_i) {
         const int t0 = tile_i * kKltTok;
-        __syncthreads();     // the previous tile's Yt and slots are consumed
+        const bool live = tile_i < ntiles && t0 + rr < num_tokens;
+#pragma unroll
+        for (int e = 0; e < kRowLoads; ++e) {
+            if (live) raw[e].load(k + (((size_t)li * num_tokens + t0 + rr) * Hkv + h) * kD + (cg + 2 * e) * 8);
+            else raw[e].zero();
+        }
         if (threadIdx.x < kKltTok)
-            sslot[threadIdx.x] = (t0 + threadIdx.x < num_tokens) ? __ldg(slots + t0 + threadIdx.x) : -1;
-        // rows of 8 elements: 128 tokens x 16 groups; neighbouring lanes take
-        // neighbouring tokens, so the transposed stores hit distinct banks
-        for (int e = threadIdx.x; e < kKltTok * 16; e += blockDim.x) {
-            const int r = e & (kKltTok - 1), c8 = (e / kKltTok) * 8;
+            nslot = (tile_i < ntiles && t0 + threadIdx.x < num_tokens) ? __ldg(slots + t0 + threadIdx.x) : -1;
+    };
+    fetch(blockIdx.x);
+    for (int tile_i = blockIdx.x; tile_i < ntiles; tile_i += gridDim.x) {
+        __syncthreads();     // the previous tile's Yt and slots are consumed
+        if (threadIdx.x < kKltTok) sslot[threadIdx.x] = nslot;
+#pragma unroll
+        for (int e = 0; e < kRowLoads; ++e) {
+            const int c8 = (cg + 2 * e) * 8;
             float x[8];
-            if (t0 + r < num_tokens) {
-                load8(k + (((size_t)li * num_tokens + t0 + r) * Hkv + h) * kD + c8, x);
+            raw[e].unpack(x);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) x[j] = __fmul_rn(x[j], __ldg(inv + c8 + j));
-            } else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) x[j] = 0.0f;
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) Yt[(c8 + j) * kKltTok + r] = x[j];
+            for (int j = 0; j < 8; ++j) Yt[(c8 + j) * kKltTok + rr] = __fmul_rn(x[j], __ldg(inv + c8 + j));
         }
         __syncthreads();
+        fetch(tile_i + gridDim.x);
         float acc[8][8];
 #pragma unroll
         for (int a = 0; a < 8; ++a)
