@@ -10,25 +10,31 @@
 // One CTA: one layer, one sequence, one kv head, and two tiles (A, B) of 32
 // query tokens each.  A tile's 128 MMA rows are the G <= 4 query heads of
 // the kv head times its 32 tokens (row = head * 32 + token), so each
-// dequantised key/value block feeds 8 query heads x 32 tokens.  Per 64-token
-// key block (4 pages):
-//   copy warp: bulk-copies the 4 packed page tiles into a staging ring.
-//   dequant warps (2): dequantise to fp16 (E2M1 x E4M3 is exact in fp16)
-//     into a K tile (K-major) and a V tile (MN-major), both in the
-//     128-byte-swizzled canonical layouts the MMA reads; rows past the
-//     sequence are zeros.
-//   MMA warp (1 elected thread): for each tile, S = Q_hi K^T + Q_lo K^T
-//     (M=128, N=64, K=16 steps; the query is split into fp16 hi + lo parts
-//     so its rounding does not reach the scores) into one of the tile's two
-//     TMEM score buffers, then O += P V (M=128, N=128) with P read from TMEM.
+// dequantised key/value block feeds 8 query heads x 32 tokens.  Keys are
+// taken in blocks of 128 tokens (8 pages), so every MMA has N = 128: at that
+// shape an MMA's shared-memory operand reads (A and B, 4 KB each per 16-deep
+// step) keep pace with its math, where N = 64 would leave the tensor pipe
+// waiting on shared memory.  Per block:
+//   dequant warps (3): read the block's packed page tiles straight from
+//     global memory (one block ahead, in registers), dequantise to fp16
+//     (E2M1 x E4M3 is exact in fp16) into a K tile (K-major, two buffers)
+//     and a V tile (MN-major, one buffer), both in the 128-byte-swizzled
+//     canonical layouts the MMA reads; rows past the sequence are zeros.
+//   MMA warp (1 elected thread): per tile, S = Q_hi K^T + Q_lo K^T (M = 128,
+//     N = 128, K = 16 steps; the query is split into fp16 hi + lo parts so
+//     its rounding does not reach the scores) into the tile's score columns;
+//     then O += P V (M = 128, N = 128) with P read from TMEM.  Order per
+//     block: QK_A, QK_B, PV_A, PV_B; a tile's next QK is issued only after
+//     its previous PV has completed (P lives in the score columns).
 //   softmax warpgroups (one per tile; a thread owns one TMEM lane = row):
-//     causal mask on diagonal blocks only, running max with lazy rescaling
-//     (the output in TMEM is rescaled only when the max grows by more than
-//     2^8), probabilities rounded once to fp16 and stored back over the
-//     first 32 columns of their own score buffer as the A operand of P V.
-// The two tiles ping-pong: while one warpgroup works on its scores, the
-// tensor pipe runs the other tile's MMAs.  TMEM: O_A, O_B (128 columns each),
-// S_A[2], S_B[2] (64 each) = 512 columns.
+//     causal mask on diagonal blocks only, a lazy softmax reference (it
+//     moves, and the output in TMEM is rescaled in one round trip, only when
+//     a block's max passes it by more than 2^12), probabilities rounded once
+//     to fp16 and stored back over the first 64 columns of the tile's score
+//     buffer as the A operand of P V.
+// TMEM: O_A, O_B (128 columns each), S_A, S_B (128 each) = 512 columns.
+// Shared memory: the query tiles (hi, lo per tile) 128 KB, two K tiles 64 KB,
+// one V tile 32 KB.
 // All hand-offs are mbarriers with bounded waits; a wait that runs out sets
 // KVQ_DEV_TIMEOUT, the CTA writes zeros and frees its TMEM.
 #include "kvq_attn.cuh"
@@ -44,60 +50,133 @@ namespace {
 constexpr int kRows = 128;          // MMA M of one tile: 4 heads x 32 query tokens
 constexpr int kQTok = 32;           // query tokens per tile
 constexpr int kTiles = 2;           // query tiles per CTA (A, B)
-constexpr int kBlkTok = 64;         // key tokens per block (4 pages)
-constexpr int kStageN = 3;          // packed-page staging stages
-constexpr uint32_t kTmemCols = 512; // O_A, O_B [0,256), S_A[2] [256,384), S_B[2] [384,512)
-constexpr float kRescaleThreshold = 8.0f;   // log2 units
-constexpr int kPidCap = 1024;       // page ids held in shared memory (keys up to 16384 tokens)
+constexpr int kBlkTok = 128;        // key tokens per block (8 pages)
+constexpr int kBlkPages = kBlkTok / kPage;
+constexpr uint32_t kTmemCols = 512; // O_A, O_B [0,256), S_A [256,384), S_B [384,512)
+// The softmax reference moves only when a block's max passes it by more than
+// kRescaleThreshold (log2 units); the probabilities are scaled by
+// 2^kPScaleLog2, so they stay below 2^(12 + 3) = 2^15, inside fp16, and a
+// weight 2^-17 of the row's largest is still a normal fp16 number.
+constexpr float kRescaleThreshold = 12.0f;
+constexpr float kPScaleLog2 = 3.0f;
+constexpr int kPidCap = 256;        // page ids held in shared memory (keys up to 4096 tokens)
 
 // shared memory map (offsets from a 1024-aligned base)
 constexpr int kQBytes = kRows * kD * 2;           // 32 KB per fp16 query tile part (hi or lo)
-constexpr int kKBytes = kBlkTok * kD * 2;         // 16 KB per fp16 key tile
-constexpr int kVBytes = kBlkTok * kD * 2;         // 16 KB per fp16 value tile
-constexpr int kStageBytes = 4 * kTile;            // 4 packed page tiles of one head
-constexpr int kVPart = kTileBf16K - kBf16VCodes;  // 1152: values of a bf16-key tile (staged alone)
+constexpr int kKBytes = kBlkTok * kD * 2;         // 32 KB per fp16 key tile
+constexpr int kVBytes = kBlkTok * kD * 2;         // 32 KB fp16 value tile
+constexpr int kPlane = kBlkTok * 128;             // one 64-dim plane of a K or V tile (128-byte rows)
 constexpr int kOffQ = 0;                          // [tile][hi, lo]
 constexpr int kOffK = kOffQ + kTiles * 2 * kQBytes;   // 2 buffers
-constexpr int kOffV = kOffK + 2 * kKBytes;        // 2 buffers
-constexpr int kOffStage = kOffV + 2 * kVBytes;    // kStageN stages
-constexpr int kSmemBytes = kOffStage + kStageN * kStageBytes;
+constexpr int kOffV = kOffK + 2 * kKBytes;        // 1 buffer
+constexpr int kSmemBytes = kOffV + kVBytes;
 constexpr int kSmemAlloc = kSmemBytes + 1024;     // room to align the base
 
-// warps 8, 9 dequantise; warp 10 only issues the bulk copies (a copy costs
-// the issuing thread hundreds of cycles, which would otherwise sit on a
-// dequant warp's path every block)
-enum { kWarpsSoftmax = 4 * kTiles, kWarpsDequant = 2 };
-constexpr int kDequantWarp0 = kWarpsSoftmax;                   // warps 8, 9
-constexpr int kCopyWarp = kDequantWarp0 + kWarpsDequant;       // warp 10
-constexpr int kMmaWarp = kCopyWarp + 1;                        // warp 11
+// warps 0-7 softmax (two warpgroups), 8-10 dequantise, 11 issues the MMAs
+enum { kWarpsSoftmax = 4 * kTiles, kWarpsDequant = 3 };
+constexpr int kDequantWarp0 = kWarpsSoftmax;
+constexpr int kMmaWarp = kDequantWarp0 + kWarpsDequant;
 constexpr int kThreads = 32 * (kMmaWarp + 1);
+constexpr int kDqThreads = 32 * kWarpsDequant;
+// dequant work items of a block: (token, half of head_dim)
+constexpr int kItems = 2 * kBlkTok;
+constexpr int kPer = (kItems + kDqThreads - 1) / kDqThreads;
 
 struct PrefillBars {
     uint64_t q_ready;                 // both softmax warpgroups wrote their query tiles (count 8)
-    uint64_t stage_full[kStageN];     // packed pages landed (tx bytes)
-    uint64_t stage_empty[kStageN];    // dequant warps read the stage (count 2)
-    uint64_t k_full[2];               // K tile j%2 written (count 2)
-    uint64_t v_full[2];               // V tile j%2 written (count 2)
-    uint64_t s_full[kTiles][2];       // QK(tile, j) done (commit)
-    uint64_t p_full[kTiles][2];       // P(tile, j) stored in TMEM, O rescaled (count 4)
-    uint64_t pv_done[kTiles][2];      // PV(tile, j) done (commit)
+    uint64_t k_full[2];               // K tile j % 2 written (count 3)
+    uint64_t k_free[2];               // QK of both tiles read K tile j % 2 (commit)
+    uint64_t v_full;                  // V tile written (count 3)
+    uint64_t v_free;                  // PV of both tiles read the V tile (commit)
+    uint64_t s_full[kTiles];          // QK(tile, j) done (commit)
+    uint64_t p_full[kTiles];          // P(tile, j) stored in TMEM, O rescaled (count 4)
+    uint64_t pv_done[kTiles];         // PV(tile, j) done (commit)
     uint64_t drain;                   // last commit before TMEM is freed after a timeout
     uint32_t tmem_base;
     int flags;                        // 1: a bounded wait ran out
-    int issued;                       // packed-page stages issued
 };
+
+// 128 consecutive fp32 columns of this thread's TMEM lane, the wait for the
+// load inside the same asm statement (so no use of the registers can be
+// scheduled before it)
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v) {
+    uint32_t r[128];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,"
+                 "%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,"
+                 "%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,"
+                 "%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,"
+                 "%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,"
+                 "%127}, [%128];\n"
+                 "tcgen05.wait::ld.sync.aligned;"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+                   "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+                   "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+                   "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]),
+                   "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
+                   "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
+                   "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]),
+                   "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]),
+                   "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]),
+                   "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]),
+                   "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]),
+                   "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]),
+                   "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]),
+                   "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]),
+                   "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]),
+                   "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]),
+                   "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]),
+                   "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+                 : "r"(taddr)
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 64 consecutive 32-bit columns of this thread's TMEM lane, waited for
+__device__ __forceinline__ void tmem_st64u(uint32_t taddr, const uint32_t* r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+                 "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,"
+                 "%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,"
+                 "%63,%64};\n"
+                 "tcgen05.wait::st.sync.aligned;"
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                   "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+                   "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]),
+                   "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]),
+                   "r"(r[31]), "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]), "r"(r[37]), "r"(r[38]),
+                   "r"(r[39]), "r"(r[40]), "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]),
+                   "r"(r[47]), "r"(r[48]), "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]),
+                   "r"(r[55]), "r"(r[56]), "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]),
+                   "r"(r[63])
+                 : "memory");
+}
+
+// 128 consecutive 32-bit columns of this thread's TMEM lane, waited for
+__device__ __forceinline__ void tmem_st128(uint32_t taddr, const float* v) {
+    uint32_t r[128];
+#pragma unroll
+    for (int i = 0; i < 128; ++i) r[i] = __float_as_uint(v[i]);
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x128.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127,%128};\n"
+                 "tcgen05.wait::st.sync.aligned;"
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]), "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]), "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]), "r"(r[56]), "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63]), "r"(r[64]), "r"(r[65]), "r"(r[66]), "r"(r[67]), "r"(r[68]), "r"(r[69]), "r"(r[70]), "r"(r[71]), "r"(r[72]), "r"(r[73]), "r"(r[74]), "r"(r[75]), "r"(r[76]), "r"(r[77]), "r"(r[78]), "r"(r[79]), "r"(r[80]), "r"(r[81]), "r"(r[82]), "r"(r[83]), "r"(r[84]), "r"(r[85]), "r"(r[86]), "r"(r[87]), "r"(r[88]), "r"(r[89]), "r"(r[90]), "r"(r[91]), "r"(r[92]), "r"(r[93]), "r"(r[94]), "r"(r[95]), "r"(r[96]), "r"(r[97]), "r"(r[98]), "r"(r[99]), "r"(r[100]), "r"(r[101]), "r"(r[102]), "r"(r[103]), "r"(r[104]), "r"(r[105]), "r"(r[106]), "r"(r[107]), "r"(r[108]), "r"(r[109]), "r"(r[110]), "r"(r[111]), "r"(r[112]), "r"(r[113]), "r"(r[114]), "r"(r[115]), "r"(r[116]), "r"(r[117]), "r"(r[118]), "r"(r[119]), "r"(r[120]), "r"(r[121]), "r"(r[122]), "r"(r[123]), "r"(r[124]), "r"(r[125]), "r"(r[126]), "r"(r[127])
+                 : "memory");
+}
 
 // ------------------------------------------------------------------ kernel
 // grid (query-tile pairs, batch * Hkv, nlayers), block 384.
-// KB: mixed cache (bf16 keys, untransformed; only the value parts of the
-// tiles are staged, the key rows are copied into the key tile directly, and
-// Q.K runs on bf16 operands).
+// KB: mixed cache (bf16 keys, untransformed: the key rows are copied into
+// the key tile as they are, and Q.K runs on bf16 operands).
 template <typename TQ, typename TO, bool KB>
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ PrefillBars bars;
-    __shared__ int32_t s_pid[kPidCap];   // the sequence's page ids, read once for every copy
+    __shared__ int32_t s_pid[kPidCap];   // the sequence's first page ids, read once
+
+    constexpr int tile = KB ? kTileBf16K : kTile;           // bytes of one kv head of one page
+    constexpr int vcodes = KB ? kBf16VCodes : kVCodes;
+    constexpr int vscales = KB ? kBf16VScales : kVScales;
 
     const int pair = blockIdx.x, b = blockIdx.y / a.Hkv, h = blockIdx.y % a.Hkv, li = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -109,27 +188,24 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
     // keys needed by the pair: positions < min(len, q_start + q0 + qn)
     int kv_end = bad_len ? 0 : min(len, qs + q0 + qn);
     if (kv_end < 0) kv_end = 0;
-    const int nb = (kv_end + kBlkTok - 1) / kBlkTok;          // 64-token blocks
+    const int nb = (kv_end + kBlkTok - 1) / kBlkTok;          // 128-token blocks
     const int npg = (kv_end + kPage - 1) / kPage;             // pages touched
     const int32_t* pt = a.page_table + (size_t)b * a.max_pages;
     const uint8_t* layer_base = a.cache + (size_t)li * a.layer_stride;
 
     if (threadIdx.x == 0) {
         bars.flags = 0;
-        bars.issued = 0;
         mbar_init(&bars.q_ready, kWarpsSoftmax);
-        for (int i = 0; i < kStageN; ++i) {
-            mbar_init(&bars.stage_full[i], 1);
-            mbar_init(&bars.stage_empty[i], kWarpsDequant);
-        }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars.k_full[i], kWarpsDequant);
-            mbar_init(&bars.v_full[i], kWarpsDequant);
-            for (int t = 0; t < kTiles; ++t) {
-                mbar_init(&bars.s_full[t][i], 1);
-                mbar_init(&bars.p_full[t][i], 4);
-                mbar_init(&bars.pv_done[t][i], 1);
-            }
+            mbar_init(&bars.k_free[i], 1);
+        }
+        mbar_init(&bars.v_full, kWarpsDequant);
+        mbar_init(&bars.v_free, 1);
+        for (int t = 0; t < kTiles; ++t) {
+            mbar_init(&bars.s_full[t], 1);
+            mbar_init(&bars.p_full[t], 4);
+            mbar_init(&bars.pv_done[t], 1);
         }
         mbar_init(&bars.drain, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -157,9 +233,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars.tmem_base;
-    // per tile t: O at tmem + 128 t; S buffer u at tmem + 256 + 128 t + 64 u
+    // per tile t: O at tmem + 128 t; S (and P over its first 64 columns) at tmem + 256 + 128 t
     auto tO = [&](int t) { return tmem + 128u * t; };
-    auto tS = [&](int t, int u) { return tmem + 256u + 128u * t + 64u * u; };
+    auto tS = [&](int t) { return tmem + 256u + 128u * t; };
 
     // per-row state of the softmax warps, kept to the epilogue
     float m_run = -INFINITY, l_run = 0.0f, isig = 1.0f;
@@ -250,12 +326,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
             }
             const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
             for (int j = 0; j < nb; ++j) {
-                const int u = j & 1;
-                if (!mbar_wait_warp(&bars.s_full[t][u], (j >> 1) & 1)) { atomicOr(&bars.flags, 1); break; }
+                if (!mbar_wait_warp(&bars.s_full[t], j & 1)) { atomicOr(&bars.flags, 1); break; }
                 tc_fence_after();
                 float s[kBlkTok];
-                tmem_ld32(tS(t, u) + lane_addr, s);
-                tmem_ld32(tS(t, u) + 32 + lane_addr, s + 32);
+                tmem_ld128(tS(t) + lane_addr, s);
                 const int kp0 = j * kBlkTok;
                 // interior blocks (every key visible to this row) skip the mask
                 if (kp0 + kBlkTok - 1 > qpos || kp0 + kBlkTok > kv_end) {
@@ -265,207 +339,176 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                         s[c] = (kp <= qpos && kp < kv_end) ? s[c] : -INFINITY;
                     }
                 }
-                // block max as a tree of three-input maxima (depth 4, not 64)
-                float m21[22];
+                // block max as a tree of three-input maxima
+                float m43[43];
 #pragma unroll
-                for (int c = 0; c < 21; ++c) m21[c] = fmax3(s[3 * c], s[3 * c + 1], s[3 * c + 2]);
-                m21[21] = s[63];
-                float m8[8];
+                for (int c = 0; c < 42; ++c) m43[c] = fmax3(s[3 * c], s[3 * c + 1], s[3 * c + 2]);
+                m43[42] = fmaxf(s[126], s[127]);
+                float m15[15];
 #pragma unroll
-                for (int c = 0; c < 7; ++c) m8[c] = fmax3(m21[3 * c], m21[3 * c + 1], m21[3 * c + 2]);
-                m8[7] = m21[21];
-                float bm = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], fmax3(m8[5], m8[6], m8[7])));
+                for (int c = 0; c < 14; ++c) m15[c] = fmax3(m43[3 * c], m43[3 * c + 1], m43[3 * c + 2]);
+                m15[14] = m43[42];
+                float m5[5];
+#pragma unroll
+                for (int c = 0; c < 5; ++c) m5[c] = fmax3(m15[3 * c], m15[3 * c + 1], m15[3 * c + 2]);
+                float bm = fmaxf(fmax3(m5[0], m5[1], m5[2]), fmaxf(m5[3], m5[4]));
                 bm *= isig;
-                // lazy rescale: move the reference max only when it grows by > 2^8
+                // lazy reference: it moves only when the block max passes it by
+                // more than kRescaleThreshold (log2 units), so most blocks leave
+                // O alone; the weights, at most 2^(threshold + kPScaleLog2) = 2^15,
+                // stay inside fp16
                 const bool grow = bm > m_run + kRescaleThreshold || (m_run == -INFINITY && bm > -INFINITY);
-                bool stop = false;
-                if (__any_sync(0xFFFFFFFFu, grow)) {
+                const bool any_grow = __any_sync(0xFFFFFFFFu, grow);
+                float al = 1.0f;
+                if (any_grow) {
                     const float mn = grow ? bm : m_run;
-                    const float al = (m_run == -INFINITY) ? 0.0f : ex2(m_run - mn);
-                    if (j > 0) {
-                        // the previous P.V must have landed before O is rescaled
-                        if (!mbar_wait_warp(&bars.pv_done[t][u ^ 1], ((j - 1) >> 1) & 1)) {
-                            atomicOr(&bars.flags, 1);
-                            stop = true;
-                        }
-                        if (!stop) {
-                            tc_fence_after();
-#pragma unroll 1
-                            for (int cc = 0; cc < 4; ++cc) {
-                                float o[32];
-                                tmem_ld32(tO(t) + cc * 32 + lane_addr, o);
-#pragma unroll
-                                for (int i = 0; i < 32; ++i) o[i] *= al;
-                                tmem_st32(tO(t) + cc * 32 + lane_addr, o);
-                            }
-                        }
-                    }
+                    al = (m_run == -INFINITY) ? 0.0f : ex2(m_run - mn);
                     l_run *= al;
                     m_run = mn;
                 }
-                if (stop) break;
-                // probabilities, fp16, stored over the first 32 columns of the score
-                // buffer; one pair in four is exponentiated on the FMA pipe
-                const float2 sc2 = make_float2(isig, isig), nm2 = make_float2(-m_run, -m_run);
-                // four independent partial sums (the row sum is a 32-deep chain otherwise)
+                // probabilities, fp16, stored over the first 64 columns of the score
+                // buffer (every exponential on the MUFU unit: this loop is bound by
+                // instruction issue, which a polynomial share would only add to)
+                const float2 sc2 = make_float2(isig, isig);
+                const float2 nm2 = make_float2(kPScaleLog2 - m_run, kPScaleLog2 - m_run);
+                // four independent partial sums (the row sum is a long chain otherwise)
                 float2 lsum[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
                                   make_float2(0.0f, 0.0f)};
+                uint32_t pk[kBlkTok / 2];
 #pragma unroll
-                for (int hv = 0; hv < 2; ++hv) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        const float2 x = ffma2(make_float2(s[32 * hv + 2 * c], s[32 * hv + 2 * c + 1]), sc2, nm2);
-                        float2 pp;
-                        if ((c & 3) == 3) {
-                            pp.x = poly_exp2(x.x);
-                            pp.y = poly_exp2(x.y);
-                        } else {
-                            pp.x = ex2(x.x);
-                            pp.y = ex2(x.y);
-                        }
-                        lsum[c & 3] = fadd2(lsum[c & 3], pp);
-                        pk[c] = h2(pp.x, pp.y);
-                    }
-                    tmem_st16u(tS(t, u) + 16 * hv + lane_addr, pk);
+                for (int c = 0; c < kBlkTok / 2; ++c) {
+                    const float2 x = ffma2(make_float2(s[2 * c], s[2 * c + 1]), sc2, nm2);
+                    float2 pp;
+                    pp.x = ex2(x.x);
+                    pp.y = ex2(x.y);
+                    lsum[c & 3] = fadd2(lsum[c & 3], pp);
+                    pk[c] = h2(pp.x, pp.y);
                 }
+                tmem_st64u(tS(t) + lane_addr, pk);
                 const float2 l2 = fadd2(fadd2(lsum[0], lsum[1]), fadd2(lsum[2], lsum[3]));
                 l_run += l2.x + l2.y;
+                if (any_grow && j > 0) {
+                    // O holds P.V of the blocks before j, complete (QK(j) was issued
+                    // only after PV(j - 1) finished): bring it to the new reference
+                    // before PV(j) adds to it, in one TMEM round trip
+                    float o[kD];
+                    tmem_ld128(tO(t) + lane_addr, o);
+#pragma unroll
+                    for (int i = 0; i < kD; i += 2) {
+                        const float2 v = fmul2(make_float2(o[i], o[i + 1]), make_float2(al, al));
+                        o[i] = v.x;
+                        o[i + 1] = v.y;
+                    }
+                    tmem_st128(tO(t) + lane_addr, o);
+                }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars.p_full[t][u]);
-            }
-        } else if (warp == kCopyWarp) {
-            // ------------------------------------------------------ copy warp
-            // block j's page tiles (the value parts only for bf16 keys) into
-            // stage j % kStageN, once the dequant warps have read block
-            // j - kStageN out of it; page ids come from shared memory
-            if (lane == 0) {
-                constexpr int part = KB ? kVPart : kTile;          // bytes staged per page
-                constexpr int part0 = KB ? kBf16VCodes : 0;       // offset of that part in the tile
-                constexpr int tile = KB ? kTileBf16K : kTile;
-                int issued = 0;
-                for (; issued < nb; ++issued) {
-                    const int st = issued % kStageN;
-                    if (issued >= kStageN &&
-                        !mbar_wait(&bars.stage_empty[st], ((issued - kStageN) / kStageN) & 1)) {
-                        atomicOr(&bars.flags, 1);
-                        break;
-                    }
-                    const int p_lo = issued * 4, n_p = min(npg, p_lo + 4) - p_lo;
-                    mbar_arrive_expect_tx(&bars.stage_full[st], (uint32_t)n_p * part);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        if (k < n_p) {
-                            const int p = p_lo + k;
-                            const int pg = p < kPidCap ? s_pid[p] : __ldg(pt + p);
-                            bulk_g2s(smem + kOffStage + st * kStageBytes + k * part,
-                                     layer_base + ((size_t)pg * a.Hkv + h) * tile + part0, part, &bars.stage_full[st]);
-                        }
-                }
-                bars.issued = issued;
+                if (lane == 0) mbar_arrive(&bars.p_full[t]);
             }
         } else if (warp < kMmaWarp) {
             // ------------------------------------------------------ dequant warps
-            const int dt = threadIdx.x - 32 * kDequantWarp0;   // 0..63
-            // items (token, half of head_dim): 128 per block over 64 threads
-            constexpr int kItems = 2 * kBlkTok, kDqThreads = 32 * kWarpsDequant;
-            constexpr int kPer = (kItems + kDqThreads - 1) / kDqThreads;
+            // Each block's packed tiles are read straight from global memory
+            // into registers one block ahead of their dequantisation.
+            const int dt = threadIdx.x - 32 * kDequantWarp0;   // 0..95
             struct Staged {
                 uint4 kc[kPer][2], vc[kPer][2];
-                uint32_t ks[kPer], vs[kPer][4];
+                uint32_t ks[kPer], vs[kPer];
             };
-            // read block j's codes and scales out of its stage and release it
-            auto load_block = [&](int j, Staged& S) -> bool {
-                const int st = j % kStageN;
-                if (!mbar_wait_warp(&bars.stage_full[st], (j / kStageN) & 1)) return false;
+            auto page_of = [&](int p) { return p < kPidCap ? s_pid[p] : __ldg(pt + p); };
+            // global address of item `it`'s page tile for block j, or null past the keys
+            auto tile_of = [&](int j, int it) -> const uint8_t* {
+                const int tkn = it >> 1;
+                if (it >= kItems || j * kBlkTok + tkn >= kv_end) return nullptr;
+                const int pg = page_of(j * kBlkPages + (tkn >> 4));
+                return layer_base + ((size_t)pg * a.Hkv + h) * tile;
+            };
+            auto load_k = [&](int j, Staged& S) {
 #pragma unroll
                 for (int e = 0; e < kPer; ++e) {
                     const int it = dt + e * kDqThreads;
-                    const int tkn = it >> 1, half = it & 1;
-                    S.kc[e][0] = S.kc[e][1] = S.vc[e][0] = S.vc[e][1] = make_uint4(0, 0, 0, 0);
+                    S.kc[e][0] = S.kc[e][1] = make_uint4(0, 0, 0, 0);
                     S.ks[e] = 0;
-                    S.vs[e][0] = S.vs[e][1] = S.vs[e][2] = S.vs[e][3] = 0;
-                    if (it < kItems && j * kBlkTok + tkn < kv_end) {
-                        const int trow = tkn & 15;
-                        if constexpr (KB) {
-                            // the stage holds the value parts only
-                            const uint8_t* T = smem + kOffStage + st * kStageBytes + (tkn >> 4) * kVPart;
-                            S.vc[e][0] = *reinterpret_cast<const uint4*>(T + trow * 64 + half * 32);
-                            S.vc[e][1] = *reinterpret_cast<const uint4*>(T + trow * 64 + half * 32 + 16);
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) S.vs[e][q] = T[1024 + (half * 4 + q) * 16 + trow];
-                        } else {
-                            const uint8_t* T = smem + kOffStage + st * kStageBytes + (tkn >> 4) * kTile;
-                            S.kc[e][0] = *reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32);
-                            S.kc[e][1] = *reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32 + 16);
-                            S.ks[e] = *reinterpret_cast<const uint32_t*>(T + kKScales + trow * 8 + half * 4);
-                            S.vc[e][0] = *reinterpret_cast<const uint4*>(T + kVCodes + trow * 64 + half * 32);
-                            S.vc[e][1] = *reinterpret_cast<const uint4*>(T + kVCodes + trow * 64 + half * 32 + 16);
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) S.vs[e][q] = T[kVScales + (half * 4 + q) * 16 + trow];
+                    if constexpr (!KB) {
+                        const uint8_t* T = tile_of(j, it);
+                        if (T) {
+                            const int trow = (it >> 1) & 15, half = it & 1;
+                            S.kc[e][0] = __ldg(reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32));
+                            S.kc[e][1] = __ldg(reinterpret_cast<const uint4*>(T + kKCodes + trow * 64 + half * 32 + 16));
+                            S.ks[e] = __ldg(reinterpret_cast<const uint32_t*>(T + kKScales + trow * 8 + half * 4));
                         }
                     }
                 }
-                __syncwarp();
-                if ((dt & 31) == 0) mbar_arrive(&bars.stage_empty[st]);
-                return true;
             };
-            // keys of block j into K buffer j & 1, free once both tiles'
-            // Q.K(j - 2) are done (the commit after the last MMA covers all)
+            auto load_v = [&](int j, Staged& S) {
+#pragma unroll
+                for (int e = 0; e < kPer; ++e) {
+                    const int it = dt + e * kDqThreads;
+                    S.vc[e][0] = S.vc[e][1] = make_uint4(0, 0, 0, 0);
+                    S.vs[e] = 0;
+                    const uint8_t* T = tile_of(j, it);
+                    if (T) {
+                        const int trow = (it >> 1) & 15, half = it & 1;
+                        S.vc[e][0] = __ldg(reinterpret_cast<const uint4*>(T + vcodes + trow * 64 + half * 32));
+                        S.vc[e][1] = __ldg(reinterpret_cast<const uint4*>(T + vcodes + trow * 64 + half * 32 + 16));
+                        uint32_t w = 0;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) w |= (uint32_t)__ldg(T + vscales + (half * 4 + q) * 16 + trow) << (8 * q);
+                        S.vs[e] = w;
+                    }
+                }
+            };
+            // fp16 rows of one item into a 128B-swizzled tile: 4 blocks of 16 dims,
+            // each 8 code bytes and one scale; a zero scale (past the keys) zeroes the row
+            auto write_rows = [&](uint8_t* tl, int it, const uint4* c, uint32_t scales) {
+                const int tkn = it >> 1, half = it & 1;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4& c0 = c[q >> 1];
+                    const uint32_t w0 = (q & 1) ? c0.z : c0.x, w1 = (q & 1) ? c0.w : c0.y;
+                    uint32_t ra[4], rb[4];
+                    e2m1x8(w0, ra);
+                    e2m1x8(w1, rb);
+                    const uint32_t sh = e4m3x2_to_f16x2((scales >> (8 * q)) & 0xFFu) & 0xFFFFu;
+                    const uint32_t sc = sh | (sh << 16);
+                    // chunk index along head_dim: 2 chunks (8 dims each) per block
+                    const int dim_chunk = half * 8 + 2 * q;          // 0..15
+                    const int plane = dim_chunk >> 3, ch = dim_chunk & 7;
+                    sts128(tl + plane * kPlane + sw128(tkn, ch), hmul2u(ra[0], sc), hmul2u(ra[1], sc),
+                           hmul2u(ra[2], sc), hmul2u(ra[3], sc));
+                    sts128(tl + plane * kPlane + sw128(tkn, ch + 1), hmul2u(rb[0], sc), hmul2u(rb[1], sc),
+                           hmul2u(rb[2], sc), hmul2u(rb[3], sc));
+                }
+            };
+            // keys of block j into K buffer j & 1, once both tiles' QK(j - 2) read it
             auto store_k = [&](int j, const Staged& S) -> bool {
                 const int buf = j & 1;
-                if (j >= 2 && !mbar_wait_warp(&bars.s_full[kTiles - 1][buf], ((j - 2) >> 1) & 1)) return false;
+                if (j >= 2 && !mbar_wait_warp(&bars.k_free[buf], ((j - 2) >> 1) & 1)) return false;
                 uint8_t* Kt = smem + kOffK + buf * kKBytes;
 #pragma unroll
                 for (int e = 0; e < kPer; ++e) {
                     const int it = dt + e * kDqThreads;
-                    if (it >= kItems) break;
-                    const int tkn = it >> 1, half = it & 1;
-                    const bool valid = j * kBlkTok + tkn < kv_end;
-                    // 4 blocks of 16 dims: 8 code bytes and one scale each
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4& c0 = S.kc[e][q >> 1];
-                        const uint32_t kw0 = (q & 1) ? c0.z : c0.x, kw1 = (q & 1) ? c0.w : c0.y;
-                        uint32_t ka[4], kb[4];
-                        e2m1x8(kw0, ka);
-                        e2m1x8(kw1, kb);
-                        const uint32_t ksh = e4m3x2_to_f16x2((S.ks[e] >> (8 * q)) & 0xFFu) & 0xFFFFu;
-                        const uint32_t ksc = valid ? (ksh | (ksh << 16)) : 0u;
-                        // chunk index along head_dim: 2 chunks (8 dims each) per block
-                        const int dim_chunk = half * 8 + 2 * q;          // 0..15
-                        const int plane = dim_chunk >> 3, ch = dim_chunk & 7;
-                        // keys: K-major, row = token, dims 0..63 / 64..127 in planes of 64 rows x 128 B
-                        sts128(Kt + plane * (kBlkTok * 128) + sw128(tkn, ch), hmul2u(ka[0], ksc),
-                               hmul2u(ka[1], ksc), hmul2u(ka[2], ksc), hmul2u(ka[3], ksc));
-                        sts128(Kt + plane * (kBlkTok * 128) + sw128(tkn, ch + 1), hmul2u(kb[0], ksc),
-                               hmul2u(kb[1], ksc), hmul2u(kb[2], ksc), hmul2u(kb[3], ksc));
-                    }
+                    if (it < kItems) write_rows(Kt, it, S.kc[e], S.ks[e]);
                 }
                 fence_async_smem();
                 __syncwarp();
                 if ((dt & 31) == 0) mbar_arrive(&bars.k_full[buf]);
                 return true;
             };
-            // bf16 keys of block j: once K buffer j & 1 is free, 16-byte async
-            // copies of each row straight into its swizzled place (zeros past
-            // the sequence); finish_k waits for them and hands the tile over
+            // bf16 keys of block j: 16-byte asynchronous copies of each row straight
+            // into its swizzled place (zeros past the keys); finish_k waits for them
             auto issue_k = [&](int j) -> bool {
                 const int buf = j & 1;
-                if (j >= 2 && !mbar_wait_warp(&bars.s_full[kTiles - 1][buf], ((j - 2) >> 1) & 1)) return false;
+                if (j >= 2 && !mbar_wait_warp(&bars.k_free[buf], ((j - 2) >> 1) & 1)) return false;
                 uint8_t* Kt = smem + kOffK + buf * kKBytes;
 #pragma unroll
                 for (int e = 0; e < kPer; ++e) {
                     const int it = dt + e * kDqThreads;
                     if (it >= kItems) break;
                     const int tkn = it >> 1, half = it & 1;
-                    uint8_t* dst = Kt + half * (kBlkTok * 128);
-                    if (j * kBlkTok + tkn < kv_end) {
-                        const int p = j * 4 + (tkn >> 4);
-                        const int pg = p < kPidCap ? s_pid[p] : __ldg(pt + p);
-                        const uint8_t* src = layer_base + ((size_t)pg * a.Hkv + h) * kTileBf16K + (tkn & 15) * 256 +
-                                             half * 128;
+                    uint8_t* dst = Kt + half * kPlane;
+                    const uint8_t* T = tile_of(j, it);
+                    if (T) {
+                        const uint8_t* src = T + (tkn & 15) * 256 + half * 128;
 #pragma unroll
                         for (int ch = 0; ch < 8; ++ch) cp_async16(dst + sw128(tkn, ch), src + ch * 16);
                     } else {
@@ -482,66 +525,45 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
                 __syncwarp();
                 if ((dt & 31) == 0) mbar_arrive(&bars.k_full[j & 1]);
             };
-            // values of block j into V buffer j & 1, free once both tiles'
-            // P.V(j - 2) are done
+            // values of block j into the V tile, once both tiles' PV(j - 1) read it
             auto store_v = [&](int j, const Staged& S) -> bool {
-                const int buf = j & 1;
-                if (j >= 2 && !mbar_wait_warp(&bars.pv_done[kTiles - 1][buf], ((j - 2) >> 1) & 1)) return false;
-                uint8_t* Vt = smem + kOffV + buf * kVBytes;
+                if (j >= 1 && !mbar_wait_warp(&bars.v_free, (j - 1) & 1)) return false;
+                uint8_t* Vt = smem + kOffV;
 #pragma unroll
                 for (int e = 0; e < kPer; ++e) {
                     const int it = dt + e * kDqThreads;
-                    if (it >= kItems) break;
-                    const int tkn = it >> 1, half = it & 1;
-                    const bool valid = j * kBlkTok + tkn < kv_end;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4& c1 = S.vc[e][q >> 1];
-                        const uint32_t vw0 = (q & 1) ? c1.z : c1.x, vw1 = (q & 1) ? c1.w : c1.y;
-                        uint32_t va[4], vb[4];
-                        e2m1x8(vw0, va);
-                        e2m1x8(vw1, vb);
-                        const uint32_t vsh = e4m3x2_to_f16x2(S.vs[e][q]) & 0xFFFFu;
-                        const uint32_t sc = valid ? (vsh | (vsh << 16)) : 0u;
-                        const int dim_chunk = half * 8 + 2 * q;
-                        const int plane = dim_chunk >> 3, ch = dim_chunk & 7;
-                        // values: MN-major, row = token (the K of P.V), 128-byte rows of 64 dims
-                        sts128(Vt + plane * (kBlkTok * 128) + sw128(tkn, ch), hmul2u(va[0], sc), hmul2u(va[1], sc),
-                               hmul2u(va[2], sc), hmul2u(va[3], sc));
-                        sts128(Vt + plane * (kBlkTok * 128) + sw128(tkn, ch + 1), hmul2u(vb[0], sc),
-                               hmul2u(vb[1], sc), hmul2u(vb[2], sc), hmul2u(vb[3], sc));
-                    }
+                    if (it < kItems) write_rows(Vt, it, S.vc[e], S.vs[e]);
                 }
                 fence_async_smem();
                 __syncwarp();
-                if ((dt & 31) == 0) mbar_arrive(&bars.v_full[buf]);
+                if ((dt & 31) == 0) mbar_arrive(&bars.v_full);
                 return true;
             };
-            // Software-pipelined: the keys of block j + 1 are written before
-            // the values of block j, because the MMA warp needs them first
-            // (Q.K(j + 1) is issued before P.V(j)).
-            Staged cur, nxt;
+            // The keys of block j + 1 are wanted before the values of block j + 1
+            // but after the values of block j (QK(j + 1) follows PV(j)).
+            Staged S;
             bool dq_ok = true;
+            load_k(0, S);
+            load_v(0, S);
             if constexpr (KB) {
-                // the copies of block j + 1's keys overlap the values of block j
-                if (nb > 0) {
-                    dq_ok = load_block(0, cur) && issue_k(0);
-                    if (dq_ok) finish_k(0);
-                }
+                dq_ok = issue_k(0);
+                if (dq_ok) finish_k(0);
                 for (int j = 0; dq_ok && j < nb; ++j) {
                     const bool more = j + 1 < nb;
-                    if (more) dq_ok = load_block(j + 1, nxt) && issue_k(j + 1);
-                    dq_ok = dq_ok && store_v(j, cur);
-                    if (more && dq_ok) finish_k(j + 1);
-                    cur = nxt;
+                    if (more) dq_ok = issue_k(j + 1);
+                    dq_ok = dq_ok && store_v(j, S);
+                    if (more && dq_ok) {
+                        load_v(j + 1, S);
+                        finish_k(j + 1);
+                    }
                 }
                 cp_async_wait_all();   // nothing in flight past this point
             } else {
-                dq_ok = nb == 0 || (load_block(0, cur) && store_k(0, cur));
                 for (int j = 0; dq_ok && j < nb; ++j) {
-                    if (j + 1 < nb) dq_ok = load_block(j + 1, nxt) && store_k(j + 1, nxt);
-                    dq_ok = dq_ok && store_v(j, cur);
-                    cur = nxt;
+                    dq_ok = store_k(j, S);
+                    if (dq_ok && j + 1 < nb) load_k(j + 1, S);
+                    dq_ok = dq_ok && store_v(j, S);
+                    if (dq_ok && j + 1 < nb) load_v(j + 1, S);
                 }
             }
             if (!dq_ok) atomicOr(&bars.flags, 1);
@@ -553,57 +575,52 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
             // bf16 keys: both Q.K operands bf16 (A and B formats 1)
             const uint32_t qk = f16_idesc(kRows, kBlkTok, false) | (KB ? ((1u << 7) | (1u << 10)) : 0u);
             const uint32_t pv = f16_idesc(kRows, kD, true);
-            uint64_t qd[kTiles][2], kd[2], vd[2];
+            uint64_t qd[kTiles][2], kd[2];
 #pragma unroll
             for (int t = 0; t < kTiles; ++t)
 #pragma unroll
                 for (int part = 0; part < 2; ++part)
                     qd[t][part] = sw128_desc(smem_u32(smem + kOffQ + (2 * t + part) * kQBytes), 16, 1024);
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                kd[u] = sw128_desc(smem_u32(smem + kOffK + u * kKBytes), 16, 1024);
-                vd[u] = sw128_desc(smem_u32(smem + kOffV + u * kVBytes), kBlkTok * 128, 1024);
-            }
+            for (int u = 0; u < 2; ++u) kd[u] = sw128_desc(smem_u32(smem + kOffK + u * kKBytes), 16, 1024);
+            const uint64_t vd = sw128_desc(smem_u32(smem + kOffV), kPlane, 1024);
             bool ok = mbar_wait(&bars.q_ready, 0);
-            for (int j = 0; ok && j <= nb; ++j) {
-                if (j < nb) {
-                    const int buf = j & 1;
-                    if (!mbar_wait(&bars.k_full[buf], (j >> 1) & 1)) { ok = false; break; }
+            for (int j = 0; ok && j < nb; ++j) {
+                const int buf = j & 1;
+                if (!mbar_wait(&bars.k_full[buf], (j >> 1) & 1)) { ok = false; break; }
+                tc_fence_after();
+                const uint64_t kb = kd[buf];
+#pragma unroll
+                for (int t = 0; t < kTiles; ++t) {
+                    // the tile's P(j - 1) sits in its score columns until PV(j - 1) is done
+                    if (j > 0 && !mbar_wait(&bars.pv_done[t], (j - 1) & 1)) { ok = false; break; }
                     tc_fence_after();
-                    const uint64_t kb = kd[buf];
-                    // tile by tile, so that tile A's softmax starts while the
-                    // tensor pipe works on tile B
+                    const uint32_t sd = tS(t);
 #pragma unroll
-                    for (int t = 0; t < kTiles; ++t) {
-                        const uint32_t sd = tS(t, buf);
+                    for (int part = 0; part < 2; ++part)
 #pragma unroll
-                        for (int part = 0; part < 2; ++part)
-#pragma unroll
-                            for (int s = 0; s < 8; ++s)
-                                mma_f16(sd, qd[t][part] + (uint64_t)(((s >> 2) * (kRows * 128) + (s & 3) * 32) >> 4),
-                                        kb + (uint64_t)(((s >> 2) * (kBlkTok * 128) + (s & 3) * 32) >> 4), qk,
-                                        (part | s) ? 1u : 0u);
-                        mma_commit(&bars.s_full[t][buf]);
-                    }
+                        for (int s = 0; s < 8; ++s)
+                            mma_f16(sd, qd[t][part] + (uint64_t)(((s >> 2) * (kRows * 128) + (s & 3) * 32) >> 4),
+                                    kb + (uint64_t)(((s >> 2) * kPlane + (s & 3) * 32) >> 4), qk,
+                                    (part | s) ? 1u : 0u);
+                    mma_commit(&bars.s_full[t]);
                 }
-                if (j >= 1) {
-                    const int jp = j - 1, buf = jp & 1;
-                    const uint64_t vb = vd[buf];
-                    if (!mbar_wait(&bars.v_full[buf], (jp >> 1) & 1)) { ok = false; break; }
+                if (!ok) break;
+                mma_commit(&bars.k_free[buf]);
+                if (!mbar_wait(&bars.v_full, j & 1)) { ok = false; break; }
 #pragma unroll
-                    for (int t = 0; t < kTiles; ++t) {
-                        if (!mbar_wait(&bars.p_full[t][buf], (jp >> 1) & 1)) { ok = false; break; }
-                        tc_fence_after();
-                        // P: 16 tokens = 8 packed columns of the score buffer;
-                        // V: 16 tokens = two 8-row atoms (2048 bytes)
+                for (int t = 0; t < kTiles; ++t) {
+                    if (!mbar_wait(&bars.p_full[t], j & 1)) { ok = false; break; }
+                    tc_fence_after();
+                    // P: 16 tokens = 8 packed columns of the score buffer;
+                    // V: 16 tokens = two 8-row atoms (2048 bytes)
 #pragma unroll
-                        for (int s = 0; s < 4; ++s)
-                            mma_f16_ta(tO(t), tS(t, buf) + 8 * s, vb + (uint64_t)((s * 2048) >> 4), pv,
-                                       (jp | s) ? 1u : 0u);
-                        mma_commit(&bars.pv_done[t][buf]);
-                    }
-                    if (!ok) break;
+                    for (int s = 0; s < kBlkTok / 16; ++s)
+                        mma_f16_ta(tO(t), tS(t) + 8 * s, vd + (uint64_t)((s * 2048) >> 4), pv, (j | s) ? 1u : 0u);
+                    mma_commit(&bars.pv_done[t]);
                 }
+                if (!ok) break;
+                mma_commit(&bars.v_free);
             }
             if (!ok) atomicOr(&bars.flags, 1);
         }
@@ -613,13 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
     __syncthreads();
     tc_fence_after();
     const bool timed_out = bars.flags != 0;
-    if (timed_out && threadIdx.x == 32 * kDequantWarp0) {
-        // drain: the packed-page copies still in flight
-        const int issued = bars.issued;
-        for (int j = max(0, issued - kStageN); j < issued; ++j)
-            (void)mbar_wait(&bars.stage_full[j % kStageN], (j / kStageN) & 1);
-        set_status(a.status, KVQ_DEV_TIMEOUT);
-    }
+    if (timed_out && threadIdx.x == 32 * kDequantWarp0) set_status(a.status, KVQ_DEV_TIMEOUT);
     if (timed_out && threadIdx.x == 32 * kMmaWarp) {
         // drain: every MMA issued by this thread completes before the commit
         // arrives; TMEM is freed only after that
@@ -639,8 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(AttnArgs a) {
         float res[kD];
         if (!dead) {
             // the last P.V of this tile has landed once its pv_done completes
-            const int jl = nb - 1;
-            const bool ok = mbar_wait_warp(&bars.pv_done[t][jl & 1], (jl >> 1) & 1);
+            const bool ok = mbar_wait_warp(&bars.pv_done[t], (nb - 1) & 1);
             tc_fence_after();
             const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
             const float sc = (ok && l_run > 0.0f) ? __ldg(a.gv + li) / l_run : 0.0f;

@@ -98,22 +98,6 @@ __device__ __forceinline__ void e2m1x8(uint32_t w, uint32_t* r) {
         "  cvt.rn.f16x2.e2m1x2 %2, b2; cvt.rn.f16x2.e2m1x2 %3, b3; }"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(w));
 }
-// 2^x on the FMA pipe, for the share of the softmax exponentials taken off
-// the MUFU unit.  x = n + f with n = floor(x) (a round-down add of 1.5 * 2^23
-// leaves n in the low mantissa bits), 2^f from a cubic fitted to 2^f on
-// [0, 1] by iteratively reweighted least squares in relative error (maximum
-// relative error 7.6e-5, below the fp16 rounding the probabilities get
-// next), and n added to the exponent field.  Valid for -126 <= x < 128.
-__device__ __forceinline__ float poly_exp2(float x) {
-    constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
-    x = fmaxf(x, -126.0f);
-    const float t = __fadd_rd(x, kMagic);
-    const float f = x - (t - kMagic);
-    const float p = fmaf(fmaf(fmaf(0.07802344113588333f, f, 0.22606651484966278f), f, 0.6958349347114563f), f,
-                         0.9999249577522278f);
-    const int n = __float_as_int(t) - __float_as_int(kMagic);
-    return __int_as_float(__float_as_int(p) + (n << 23));
-}
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
