@@ -50,7 +50,12 @@ constexpr int kBlkTok = 64;         // key tokens per block (4 pages)
 constexpr int kStageN = 6;          // packed-page staging stages
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 256, kColP = 384, kColSFA = 448, kColSFB = 464;
-constexpr float kRescaleThreshold = 8.0f;   // log2 units
+// The softmax reference moves only when a block's max passes it by more than
+// kRescaleThreshold (log2 units); the probabilities are scaled by
+// 2^kPScaleLog2, so they stay below 2^(12 + 3) = 2^15, inside fp16, and a
+// weight 2^-17 of the row's largest is still a normal fp16 number.
+constexpr float kRescaleThreshold = 12.0f;
+constexpr float kPScaleLog2 = 3.0f;
 constexpr int kPidCap = 1024;       // page ids held in shared memory (keys up to 16384 tokens)
 
 // shared memory map (offsets from a 1024-aligned base)
@@ -293,24 +298,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_fp4_kernel(AttnArgs a) {
                     return pv_ok;
                 };
                 const bool grow = bm > m_run + kRescaleThreshold || (m_run == -INFINITY && bm > -INFINITY);
-                if (__any_sync(0xFFFFFFFFu, grow)) {
+                const bool any_grow = __any_sync(0xFFFFFFFFu, grow);
+                float al = 1.0f;
+                if (any_grow) {
                     const float mn = grow ? bm : m_run;
-                    const float al = (m_run == -INFINITY) ? 0.0f : ex2(m_run - mn);
-                    if (j > 0) {
-                        if (!wait_pv()) { atomicOr(&bars.flags, 1); break; }
-#pragma unroll 1
-                        for (int cc = 0; cc < 4; ++cc) {
-                            float o[32];
-                            tmem_ld32(tO(t) + cc * 32 + lane_addr, o);
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) o[i] *= al;
-                            tmem_st32(tO(t) + cc * 32 + lane_addr, o);
-                        }
-                    }
+                    al = (m_run == -INFINITY) ? 0.0f : ex2(m_run - mn);
                     l_run *= al;
                     m_run = mn;
                 }
-                const float2 sc2 = make_float2(isig, isig), nm2 = make_float2(-m_run, -m_run);
+                const float2 sc2 = make_float2(isig, isig);
+                const float2 nm2 = make_float2(kPScaleLog2 - m_run, kPScaleLog2 - m_run);
                 float2 lsum[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
                                   make_float2(0.0f, 0.0f)};
                 uint32_t pk[32];
@@ -328,6 +325,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_fp4_kernel(AttnArgs a) {
                 tmem_st16u(tP(t) + 16 + lane_addr, pk + 16);
                 const float2 l2 = fadd2(fadd2(lsum[0], lsum[1]), fadd2(lsum[2], lsum[3]));
                 l_run += l2.x + l2.y;
+                if (any_grow && j > 0) {
+                    // P.V(j - 1) is done (waited above): bring O to the new
+                    // reference before P.V(j) adds to it, in one TMEM round trip
+                    float o[kD];
+                    tmem_ld128(tO(t) + lane_addr, o);
+#pragma unroll
+                    for (int i = 0; i < kD; i += 2) {
+                        const float2 v = fmul2(make_float2(o[i], o[i + 1]), make_float2(al, al));
+                        o[i] = v.x;
+                        o[i + 1] = v.y;
+                    }
+                    tmem_st128(tO(t) + lane_addr, o);
+                }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars.p_full[t]);
