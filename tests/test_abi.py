@@ -117,6 +117,29 @@ def test_decode_split_plan_is_deterministic(kvq_lib):
     assert a > 0 and a == kvq.decode_workspace_bytes(kvq.Shape(1, 32, 8), 1, 1, 512)
 
 
+def test_workspace_layout(kvq_lib):
+    # a workspace starts with the split merge's 4096-byte counter header, then
+    # the partials [nl][B][Hq][splits][132] fp32 (256-byte aligned), then with
+    # a KLT cache the rotated queries [nl][B][Hq][128] fp32; the prefill's
+    # rotated queries also start after the header
+    kvq = kvq_lib
+    s = kvq.Shape(1, 32, 8)
+    ws = kvq.decode_workspace_bytes(s, 1, 1, 512)
+    splits = (ws - 4096) // (32 * 132 * 4)
+    assert ws == 4096 + 32 * splits * 132 * 4 and splits > 1
+    klt = kvq.Shape(1, 32, 8, use_klt=True)
+    part = 32 * splits * 132 * 4
+    assert kvq.decode_workspace_bytes(klt, 1, 1, 512) == 4096 + (part + 255) // 256 * 256 + 32 * 128 * 4
+    # no split, no KLT: no workspace; no split with a KLT cache: header + queries
+    assert kvq.decode_workspace_bytes(kvq.Shape(36, 32, 8), 36, 64, 516) == 0
+    assert kvq.decode_workspace_bytes(kvq.Shape(36, 32, 8, use_klt=True), 36, 64, 516) == 4096 + 36 * 64 * 32 * 128 * 4
+    assert kvq.prefill_workspace_bytes(kvq.Shape(2, 32, 8), 2, 8, 512) == 0
+    assert kvq.prefill_workspace_bytes(kvq.Shape(2, 32, 8, use_klt=True), 2, 8, 512) == 4096 + 2 * 8 * 512 * 32 * 128 * 4
+    # the binding's workspaces are zero-filled
+    w = kvq.new_workspace(64, "cpu")
+    assert w.dtype.itemsize == 1 and int(w.sum()) == 0
+
+
 def test_mixed_cache_key_format_validation(kvq_lib):
     kvq = kvq_lib
     bf = kvq.Shape(2, 32, 8, k_format=kvq.K_BF16)

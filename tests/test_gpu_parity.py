@@ -166,6 +166,47 @@ def test_long_sequence_many_splits(kvq):
     harness.check_attention(out[0, 0], want[0], "5000 tokens f32")
 
 
+def test_split_merge_counters_and_workspace_reuse(kvq):
+    # The fused split merge keeps one arrival counter per (layer, sequence) in
+    # the first 4096 bytes of the workspace: zero before the first call, left
+    # zero by every call.  One zero-filled workspace then serves split decodes
+    # of different shapes in any order, bit for bit like fresh workspaces; a
+    # header that was not zero-filled is reported (KVQ_DEV_BAD_WORKSPACE), not
+    # trapped.
+    w = small(num_layers=2, batch=3, calib_windows=1, calib_len=64)
+    pa = harness.build_problem(kvq, w, lens=[3000, 45, 700])
+    pb = harness.build_problem(kvq, small(num_layers=1, batch=1, calib_windows=1, calib_len=64), lens=[5000])
+    qa = torch.stack([synth.decode_queries(pa.w, l, 0) for l in pa.layers]).cuda()
+    qb = torch.stack([synth.decode_queries(pb.w, l, 0) for l in pb.layers]).cuda()
+    need = [kvq.decode_workspace_bytes(p.shape, len(p.layers), len(p.lens), p.page_table.shape[1]) for p in (pa, pb)]
+    assert min(need) > 4096
+    shared = kvq.new_workspace(max(need))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def run(p, q, ws):
+        return kvq.decode_attention(p.shape, p.calib, p.cache, q, p.page_table.cuda(), p.lens.cuda(),
+                                    out_dtype=torch.float32, workspace=ws, status=status)
+
+    ref_a = run(pa, qa, kvq.new_workspace(need[0]))
+    ref_b = run(pb, qb, kvq.new_workspace(need[1]))
+    for p, q, ref in ((pa, qa, ref_a), (pb, qb, ref_b), (pa, qa, ref_a), (pb, qb, ref_b)):
+        assert torch.equal(run(p, q, shared), ref)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.count_nonzero(shared[:4096]).item() == 0          # the counters are back to zero
+    cal = harness.oracle_calibration(pa)
+    qh = qa.cpu().numpy()
+    for li in range(2):
+        for b, n in enumerate(pa.lens.tolist()):
+            want = harness.oracle_attend(pa, li, b, qh[li, b][None], n - 1, n, cal)
+            harness.check_attention(ref_a[li, b].cpu().numpy(), want[0], f"reused workspace layer {li} seq {b}")
+    # a header that was not zero-filled: flagged
+    bad = torch.full((need[0],), 0x7F, dtype=torch.uint8, device="cuda")
+    run(pa, qa, bad)
+    torch.cuda.synchronize()
+    assert status.item() & kvq.DEV_BAD_WORKSPACE
+
+
 @pytest.mark.parametrize("scale", [1.0 / 64, 3.0])
 def test_flat_and_peaked_softmax(kvq, scale):
     # The decode keeps a lazy softmax reference that moves only when a score
