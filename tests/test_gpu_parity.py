@@ -195,7 +195,7 @@ def test_split_merge_counters_and_workspace_reuse(kvq):
     assert status.item() == 0
     assert torch.count_nonzero(shared[:4096]).item() == 0          # the counters are back to zero
     cal = harness.oracle_calibration(pa)
-    qh = qa.cpu().numpy()
+    qh = qa.float().cpu().numpy()
     for li in range(2):
         for b, n in enumerate(pa.lens.tolist()):
             want = harness.oracle_attend(pa, li, b, qh[li, b][None], n - 1, n, cal)
