@@ -254,8 +254,10 @@ size_t kvq_decode_workspace_bytes(const kvq_shape* shape, int32_t nlayers, int32
  *                may then serve any sequence of decode and prefill calls).
  *                The rest is scratch (split partials, rotated queries) whose
  *                contents are undefined after the call.  A counter found
- *                non-zero sets KVQ_DEV_BAD_WORKSPACE.  Calls that share a
- *                workspace must not overlap on the GPU.
+ *                at or above the split count (a header that was not
+ *                zero-filled) sets KVQ_DEV_BAD_WORKSPACE; a smaller stale
+ *                value cannot be told from an arrival and gives wrong rows.
+ *                Calls that share a workspace must not overlap on the GPU.
  * With KVQ_K_BF16 keys the query is used as given (no smoothing, no
  * rotation, no key tensor scale): scores are q . k / sqrt(128).
  * Errors: KVQ_EINVAL / KVQ_EWORKSPACE on the host; KVQ_DEV_BAD_PAGE and
