@@ -297,6 +297,28 @@ def test_device_faults_are_flagged_not_trapped(kvq):
     assert changed.numel() > 0 and torch.all(changed[:, 1] == 0)           # only page 0 (slot 5) touched
 
 
+def test_bad_page_in_a_split_unit(kvq):
+    # A page id outside the pool in one split of a long sequence: the split
+    # poisons its partial, the fused merge writes the row as zeros (not NaN)
+    # and the status says why; the other sequence, also split, is unaffected.
+    w = small(num_layers=1, batch=2, calib_windows=1, calib_len=64)
+    lens = [3000, 2500]
+    p = harness.build_problem(kvq, w, lens=lens)
+    assert kvq.decode_workspace_bytes(p.shape, 1, 2, p.page_table.shape[1]) > 0     # split
+    cal = harness.oracle_calibration(p)
+    pt = p.page_table.clone()
+    pt[0, 100] = p.num_pages + 7
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q = synth.decode_queries(w, 0, 0)[None].cuda()
+    out = kvq.decode_attention(p.shape, p.calib, p.cache, q, pt.cuda(), p.lens.cuda(), status=status,
+                               out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert status.item() & kvq.DEV_BAD_PAGE
+    assert torch.all(out[0, 0] == 0)
+    want = harness.oracle_attend(p, 0, 1, q[0, 1].float().cpu().numpy()[None], lens[1] - 1, lens[1], cal)
+    harness.check_attention(out[0, 1].cpu().numpy(), want[0], "split sequence beside a bad page f32")
+
+
 def test_bounded_wait_gives_up_and_context_survives(kvq):
     """A wait on a barrier nothing arrives at runs out and reports DEV_TIMEOUT."""
     import time
