@@ -307,36 +307,58 @@ __global__ void klt_finalize_kernel(float* __restrict__ gk, float* __restrict__ 
 }
 
 // ------------------------------------------------------------------ append
-// Keys of the KLT cache: grid (CTAs per (layer, head), Hkv, nlayers), 128
-// threads, two CTAs per SM; each CTA loads the basis once and walks tiles of
-// 64 tokens (one CTA's tile load overlaps the other's transform).  Smoothing y = k * inv_s,
-// the transform y' = U^T y (one fp32 FMA chain per output over c = 0..127),
-// then the NVFP4 quantiser of the append (absmax -> E4M3 scale -> reciprocal
-// -> E2M1, each step one fp32 rounding) and the scatter to the token's slot.
+// Keys of the KLT cache: grid (CTAs per (layer, head), Hkv, nlayers), one CTA
+// per SM of two tile groups (128 threads each) that share the basis and walk
+// tiles of 128 tokens of their (layer, head); one group's tile load overlaps
+// the other's transform.  Smoothing y = k * inv_s, the transform y' = U^T y
+// (one fp32 FMA chain per output over c = 0..127), then the NVFP4 quantiser
+// of the append (absmax -> E4M3 scale -> reciprocal -> E2M1, each step one
+// fp32 rounding) and the scatter to the token's slot.
 //
-// Thread (warp w, lane l) holds 8 tokens (8 (2w + l / 16) .. + 7) x 8 dims
-// (4 (l % 16) .. + 3 and 64 + 4 (l % 16) .. + 3): per step c it reads 8
-// token values (the same for a half-warp) and two runs of 4 basis values
-// (contiguous over a quarter-warp), 16 shared-memory wavefronts for 64 FMAs,
-// which keeps shared memory and the FMA pipe in balance.  The 4 lanes of a
-// 16-block are neighbours and share its absmax by two shuffles.
-constexpr int kKltTok = 64;   // tokens per append tile
-constexpr size_t kKltAppendSmem =
-    (size_t)kD * kD * sizeof(float) + (size_t)kD * kKltTok * sizeof(float) + 128 * sizeof(float) +
-    kKltTok * sizeof(int64_t) + 16;
+// Thread (warp w, lane l) of a group holds 8 tokens (8 (4w + l / 8) .. + 7)
+// x one 16-block of dims (16 (l % 8) .. + 15): 128 accumulators, and the
+// block's absmax without a shuffle.  Per step c it reads the 8 token values
+// (two 16-byte loads, shared by 8 lanes) and the block's 16 basis values
+// (four 16-byte loads).  The basis rows are stored with their 16-byte chunks
+// permuted, so the 8 blocks' i-th chunks sit in 8 distinct bank groups: 6
+// shared-memory wavefronts per warp and step for 128 FMAs.  The FMAs run in
+// packed pairs of dims (fma.rn.f32x2, each half rounded as fmaf), 64
+// instructions per step; the chains and their order are unchanged.
+constexpr int kKltTok = 128;  // tokens per append tile
+constexpr int kKltGroups = 2; // tile groups per CTA
+constexpr int kKltThreads = 128 * kKltGroups;
+constexpr size_t kKltAppendSmem = (size_t)kD * kD * sizeof(float) +
+                                  (size_t)kKltGroups * kD * kKltTok * sizeof(float) + 128 * sizeof(float) +
+                                  (size_t)kKltGroups * kKltTok * sizeof(int64_t) + 16;
+
+// Physical 16-byte chunk, within a basis row, of dims 16 blk + 4 i .. + 3:
+// chunk i of the 8 blocks lands in 8 distinct bank groups.
+__device__ __forceinline__ int klt_chunk(int blk, int i) { return 8 * i + ((blk + i) & 7); }
+
+// barrier of one 128-thread tile group (named barriers 1..kKltGroups)
+__device__ __forceinline__ void group_sync(int grp) {
+    asm volatile("bar.sync %0, 128;" ::"r"(grp + 1) : "memory");
+}
 
 template <typename T>
-__global__ void __launch_bounds__(128, 2)
+__global__ void __launch_bounds__(kKltThreads, 1)
 klt_append_keys_kernel(const T* __restrict__ k, const int64_t* __restrict__ slots, int num_tokens, int Hkv,
                        const float* __restrict__ inv_s, const float* __restrict__ U, const float* __restrict__ gk,
                        uint8_t* __restrict__ cache, int64_t layer_stride, int num_pages, int32_t* __restrict__ status) {
     extern __shared__ __align__(16) float sm[];
-    float* Us = sm;                              // [c][i]
-    float* Yt = Us + kD * kD;                    // [c][token]
-    float* rtab = Yt + kD * kKltTok;
-    int64_t* sslot = reinterpret_cast<int64_t*>(rtab + 128);
+    const int grp = threadIdx.x >> 7, tid = threadIdx.x & 127;
+    float* Us = sm;                                            // [c][permuted chunks of i]
+    float* Yt = Us + kD * kD + grp * kD * kKltTok;             // this group's [c][token]
+    float* rtab = Us + kD * kD + kKltGroups * kD * kKltTok;
+    int64_t* sslot = reinterpret_cast<int64_t*>(rtab + 128) + grp * kKltTok;
     const int h = blockIdx.y, li = blockIdx.z;
-    klt_load_basis(Us, U + ((size_t)li * Hkv + h) * kD * kD);
+    {
+        const float4* src = reinterpret_cast<const float4*>(U + ((size_t)li * Hkv + h) * kD * kD);
+        for (int e = threadIdx.x; e < kD * kD / 4; e += kKltThreads) {
+            const int c = e >> 5, q = e & 31;                  // row, logical chunk (block q / 4, i = q % 4)
+            reinterpret_cast<float4*>(Us)[c * 32 + klt_chunk(q >> 2, q & 3)] = __ldg(src + e);
+        }
+    }
     const float g = __ldg(gk + li);
     const float enc = __frcp_rn(__fmul_rn(6.0f, g));
     if (threadIdx.x < 128) {
@@ -348,89 +370,91 @@ klt_append_keys_kernel(const T* __restrict__ k, const int64_t* __restrict__ slot
     const int64_t num_slots = (int64_t)num_pages * kPage;
     uint8_t* layer_cache = cache + (size_t)li * layer_stride;
     const int lane = threadIdx.x & 31;
-    const int tgi = 2 * (threadIdx.x >> 5) + (lane >> 4);   // token group: tokens 8 tgi .. + 7
-    const int dl = lane & 15;                               // dims 4 dl .. + 3 and 64 + 4 dl .. + 3
+    const int tg = 4 * (tid >> 5) + (lane >> 3);               // tokens 8 tg .. + 7
+    const int blk = lane & 7;                                  // dims 16 blk .. + 15
     const int ntiles = (num_tokens + kKltTok - 1) / kKltTok;
-    // The next tile's key rows and slots are loaded one tile ahead, into
-    // registers, so their global-memory latency overlaps this tile's
-    // transform.  Rows of 8 elements: 64 tokens x 16 groups; neighbouring
-    // lanes take neighbouring tokens, so the transposed stores hit distinct
-    // banks.
-    constexpr int kRowLoads = kKltTok * 16 / 128;
-    static_assert(kRowLoads * 128 == kKltTok * 16, "128 threads");
-    const int rr = threadIdx.x & (kKltTok - 1), cg = threadIdx.x >> 6;   // token, first 8-group
-    Raw8<T> raw[kRowLoads];
+    // Thread tid loads token tid's key row, 16 runs of 8 elements, and its
+    // slot.  The first kAhead runs (bf16: a quarter of the row) and the slot are
+    // loaded one tile ahead, into registers, so their global-memory latency
+    // overlaps this tile's transform; the rest when the tile starts.
+    constexpr int kAhead = sizeof(T) == 2 ? 4 : 0;
+    Raw8<T> raw[16];
     int64_t nslot = -1;
-    auto fetch = [&](int tile_i) {
+    auto fetch = [&](int tile_i, int e0, int e1) {
         const int t0 = tile_i * kKltTok;
-        const bool live = tile_i < ntiles && t0 + rr < num_tokens;
+        const bool live = tile_i < ntiles && t0 + tid < num_tokens;
+        const T* row = k + (((size_t)li * num_tokens + t0 + tid) * Hkv + h) * kD;
 #pragma unroll
-        for (int e = 0; e < kRowLoads; ++e) {
-            if (live) raw[e].load(k + (((size_t)li * num_tokens + t0 + rr) * Hkv + h) * kD + (cg + 2 * e) * 8);
+        for (int e = 0; e < 16; ++e) {
+            if (e < e0 || e >= e1) continue;
+            if (live) raw[e].load(row + 8 * e);
             else raw[e].zero();
         }
-        if (threadIdx.x < kKltTok)
-            nslot = (tile_i < ntiles && t0 + threadIdx.x < num_tokens) ? __ldg(slots + t0 + threadIdx.x) : -1;
+        if (e0 == 0) nslot = live ? __ldg(slots + t0 + tid) : -1;
     };
-    fetch(blockIdx.x);
-    for (int tile_i = blockIdx.x; tile_i < ntiles; tile_i += gridDim.x) {
-        __syncthreads();     // the previous tile's Yt and slots are consumed
-        if (threadIdx.x < kKltTok) sslot[threadIdx.x] = nslot;
+    // each group walks its own tiles; the basis and the table are shared
+    const int first = blockIdx.x * kKltGroups + grp, stride = gridDim.x * kKltGroups;
+    if (kAhead > 0) fetch(first, 0, kAhead);
+    __syncthreads();         // the basis and the table are in place
+    for (int tile_i = first; tile_i < ntiles; tile_i += stride) {
+        group_sync(grp);     // the previous tile's Yt and slots are consumed
+        fetch(tile_i, kAhead, 16);
+        sslot[tid] = nslot;
 #pragma unroll
-        for (int e = 0; e < kRowLoads; ++e) {
-            const int c8 = (cg + 2 * e) * 8;
+        for (int e = 0; e < 16; ++e) {
             float x[8];
             raw[e].unpack(x);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) Yt[(c8 + j) * kKltTok + rr] = __fmul_rn(x[j], __ldg(inv + c8 + j));
+            for (int j = 0; j < 8; ++j) Yt[(8 * e + j) * kKltTok + tid] = __fmul_rn(x[j], __ldg(inv + 8 * e + j));
         }
-        __syncthreads();
-        fetch(tile_i + gridDim.x);
-        float acc[8][8];
+        group_sync(grp);
+        if (kAhead > 0) fetch(tile_i + stride, 0, kAhead);
+        float2 acc[8][8];    // token a, dims 16 blk + 2 p, + 1
 #pragma unroll
         for (int a = 0; a < 8; ++a)
 #pragma unroll
-            for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
+            for (int p = 0; p < 8; ++p) acc[a][p] = make_float2(0.0f, 0.0f);
+        const float* yrow = Yt + 8 * tg;
+        const float4* urow = reinterpret_cast<const float4*>(Us);
 #pragma unroll 2
         for (int c = 0; c < kD; ++c) {
-            const float4 y0 = *reinterpret_cast<const float4*>(Yt + c * kKltTok + 8 * tgi);
-            const float4 y1 = *reinterpret_cast<const float4*>(Yt + c * kKltTok + 8 * tgi + 4);
-            const float4 u0 = *reinterpret_cast<const float4*>(Us + c * kD + 4 * dl);
-            const float4 u1 = *reinterpret_cast<const float4*>(Us + c * kD + 64 + 4 * dl);
+            const float4 y0 = *reinterpret_cast<const float4*>(yrow + c * kKltTok);
+            const float4 y1 = *reinterpret_cast<const float4*>(yrow + c * kKltTok + 4);
+            float2 u[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 t = urow[c * 32 + klt_chunk(blk, i)];
+                u[2 * i] = make_float2(t.x, t.y);
+                u[2 * i + 1] = make_float2(t.z, t.w);
+            }
             const float y[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
-            const float u[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            // packed pairs of dims: each half is fma(u, y, acc), rounded once
 #pragma unroll
-            for (int a = 0; a < 8; ++a)
+            for (int a = 0; a < 8; ++a) {
+                const float2 yy = make_float2(y[a], y[a]);
 #pragma unroll
-                for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(u[b], y[a], acc[a][b]);
+                for (int p = 0; p < 8; ++p) acc[a][p] = ffma2(u[p], yy, acc[a][p]);
+            }
         }
 #pragma unroll
         for (int a = 0; a < 8; ++a) {
-            const int tt = 8 * tgi + a;
-            const int64_t slot = sslot[tt];
+            const int64_t slot = sslot[8 * tg + a];
+            float2 v[8];
 #pragma unroll
-            for (int gi = 0; gi < 2; ++gi) {
-                // this lane's 4 dims of block 4 gi + dl / 4; the block's 4 lanes are neighbours
-                float m = fmaxf(fmaxf(fabsf(acc[a][4 * gi]), fabsf(acc[a][4 * gi + 1])),
-                                fmaxf(fabsf(acc[a][4 * gi + 2]), fabsf(acc[a][4 * gi + 3])));
-                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-                const uint32_t sf = e4m3_rn(__fmul_rn(m, enc));
-                const float r = rtab[sf & 0x7Fu];
-                // two code bytes (the other two pairs of the routine are unused)
-                const uint32_t w =
-                    e2m1x8_rn(make_float2(__fmul_rn(acc[a][4 * gi], r), __fmul_rn(acc[a][4 * gi + 1], r)),
-                              make_float2(__fmul_rn(acc[a][4 * gi + 2], r), __fmul_rn(acc[a][4 * gi + 3], r)),
-                              make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)) & 0xFFFFu;
-                if (slot >= num_slots) {
-                    if (dl == 0 && gi == 0) set_status(status, KVQ_DEV_BAD_SLOT);
-                } else if (slot >= 0) {
-                    uint8_t* tile = layer_cache + ((size_t)(slot >> 4) * Hkv + h) * kTile;
-                    const int off = (int)(slot & 15);
-                    // dims 64 gi + 4 dl .. + 3: code bytes 32 gi + 2 dl, + 1
-                    *reinterpret_cast<uint16_t*>(tile + kKCodes + off * 64 + 32 * gi + 2 * dl) = (uint16_t)w;
-                    if ((dl & 3) == 0) tile[kKScales + off * 8 + 4 * gi + (dl >> 2)] = (uint8_t)sf;
-                }
+            for (int p = 0; p < 8; ++p) v[p] = acc[a][p];
+            const uint32_t sf = e4m3_rn(__fmul_rn(absmax16(v), enc));
+            const float r = rtab[sf & 0x7Fu];
+#pragma unroll
+            for (int p = 0; p < 8; ++p) v[p] = make_float2(__fmul_rn(v[p].x, r), __fmul_rn(v[p].y, r));
+            const uint2 w = make_uint2(e2m1x8_rn(v[0], v[1], v[2], v[3]), e2m1x8_rn(v[4], v[5], v[6], v[7]));
+            if (slot >= num_slots) {
+                if (blk == 0) set_status(status, KVQ_DEV_BAD_SLOT);
+            } else if (slot >= 0) {
+                uint8_t* tile = layer_cache + ((size_t)(slot >> 4) * Hkv + h) * kTile;
+                const int off = (int)(slot & 15);
+                // dims 16 blk .. + 15: code bytes 8 blk .. + 7, scale byte blk
+                *reinterpret_cast<uint2*>(tile + kKCodes + off * 64 + 8 * blk) = w;
+                tile[kKScales + off * 8 + blk] = (uint8_t)sf;
             }
         }
     }
@@ -444,25 +468,28 @@ kvq_status append_klt_keys(const kvq_shape& s, const kvq_calib& c, const kvq_cac
     const float* U = c.k_klt + (size_t)layer0 * H * kD * kD;
     const float* gk = c.k_gscale + layer0;
     uint8_t* base = cache.data + (size_t)layer0 * cache.layer_stride_bytes;
-    // about two CTAs per SM in all; each walks tiles of its (layer, head)
+    // one CTA per SM at most (no partial second wave); each CTA's tile groups
+    // walk tiles of its (layer, head)
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long ntiles = (num_tokens + kKltTok - 1) / kKltTok;
-    const long per = (2L * sms + (long)H * nlayers - 1) / ((long)H * nlayers);
-    const dim3 grid((unsigned)(ntiles < per ? ntiles : (per < 1 ? 1 : per)), H, nlayers);
+    const long walkers = (ntiles + kKltGroups - 1) / kKltGroups;
+    long per = (long)sms / ((long)H * nlayers);
+    if (per < 1) per = 1;
+    const dim3 grid((unsigned)(walkers < per ? walkers : per), H, nlayers);
     cudaError_t e;
     if (dtype == KVQ_F32) {
         e = cudaFuncSetAttribute(klt_append_keys_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kKltAppendSmem);
         if (e != cudaSuccess) return KVQ_ECUDA;
-        klt_append_keys_kernel<float><<<grid, 128, kKltAppendSmem, st>>>((const float*)k, slots, num_tokens, H, inv,
+        klt_append_keys_kernel<float><<<grid, kKltThreads, kKltAppendSmem, st>>>((const float*)k, slots, num_tokens, H, inv,
                                                                        U, gk, base, cache.layer_stride_bytes,
                                                                        cache.num_pages, status);
     } else {
         e = cudaFuncSetAttribute(klt_append_keys_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kKltAppendSmem);
         if (e != cudaSuccess) return KVQ_ECUDA;
-        klt_append_keys_kernel<__nv_bfloat16><<<grid, 128, kKltAppendSmem, st>>>(
+        klt_append_keys_kernel<__nv_bfloat16><<<grid, kKltThreads, kKltAppendSmem, st>>>(
             (const __nv_bfloat16*)k, slots, num_tokens, H, inv, U, gk, base, cache.layer_stride_bytes,
             cache.num_pages, status);
     }
