@@ -132,3 +132,19 @@ def test_klt_prefill_within_tolerance(kvq, qk_fp4):
         for b in range(2):
             want = attend(p, li, b, q[li, b].float().numpy(), P0[b], lens[b], cal)
             harness.check_attention(out[li, b], want, f"klt prefill{' fp4' if qk_fp4 else ''} layer {li} seq {b}")
+
+
+def test_klt_append_bad_slot_skipped_and_flagged(kvq):
+    """A slot beyond the cache in a KLT append: the key kernel (and the value
+    kernel) skip it and set KVQ_DEV_BAD_SLOT; the other token is written."""
+    p = _klt_problem(kvq, [40])
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    before = p.cache.data.clone()
+    k, v = synth.sequence_kv(p.w, 0, 0, 2, "cuda")
+    slots = torch.tensor([p.num_pages * 16 + 3, 5], dtype=torch.int64, device="cuda")
+    kvq.quantize_append(p.shape, p.calib, p.cache, k.contiguous(), v.contiguous(), slots, status=status)
+    torch.cuda.synchronize()
+    assert status.item() & kvq.DEV_BAD_SLOT
+    changed = (p.cache.data != before).nonzero()
+    # only layer 0's page 0 (slot 5) is touched
+    assert changed.numel() > 0 and torch.all(changed[:, 0] == 0) and torch.all(changed[:, 1] == 0)
