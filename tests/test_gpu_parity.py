@@ -156,6 +156,34 @@ def test_many_units_single_split(kvq):
             harness.check_attention(out[li, b], want[0], f"layer {li} seq {b} bf16")
 
 
+def test_split_batch_edge_lengths_and_a_bad_page(kvq):
+    # 2 layers x 64 sequences = 128 (layer, sequence) units, too few to fill
+    # the GPU unsplit: a split decode.  Lengths include 0, one token, a full
+    # page and one past it; a bad page id poisons one sequence only, in both
+    # layers, and leaves the others within tolerance.
+    w = small(num_layers=2, batch=64, calib_windows=1, calib_len=64)
+    lens = [0, 1, 16, 17] + [(37 * b) % 600 + 2 for b in range(4, 64)]
+    p = harness.build_problem(kvq, w, lens=lens)
+    assert kvq.decode_workspace_bytes(p.shape, 2, 64, p.page_table.shape[1]) > 0     # split
+    cal = harness.oracle_calibration(p)
+    bad = 5
+    pt = p.page_table.clone()
+    pt[bad, 1] = p.num_pages + 5
+    q = torch.stack([synth.decode_queries(w, l, 0) for l in p.layers])
+    for dt, tag in ((torch.float32, "f32"), (torch.bfloat16, "bf16")):
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        out = kvq.decode_attention(p.shape, p.calib, p.cache, q.cuda(), pt.cuda(), p.lens.cuda(), status=status,
+                                   out_dtype=dt).float().cpu().numpy()
+        torch.cuda.synchronize()
+        assert status.item() & kvq.DEV_BAD_PAGE
+        assert np.all(out[:, bad] == 0) and np.all(out[:, 0] == 0)
+        for li in (0, 1):
+            for b in (1, 2, 3, 4, 17, 63):
+                n = lens[b]
+                want = harness.oracle_attend(p, li, b, q[li, b].float().numpy()[None], n - 1, n, cal)
+                harness.check_attention(out[li, b], want[0], f"split batch, layer {li} seq {b} {tag}")
+
+
 def test_long_sequence_many_splits(kvq):
     w = small(num_layers=1, batch=1, calib_windows=1, calib_len=128)
     p = harness.build_problem(kvq, w, lens=[5000])
