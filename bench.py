@@ -146,13 +146,21 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
-    def _poll(self):
+    def _sample(self) -> bool:
         nv, h = self._nvml, self._h
+        try:
+            self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                 int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))))
+            return True
+        except Exception:
+            return False
+
+    def _poll(self):
+        # every 5 ms while the timed region runs (the thread may be scheduled
+        # late while the main thread holds the interpreter; stop() adds a
+        # closing sample, so a short region still has its two ends)
         while not self._stop.is_set():
-            try:
-                self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
-                                     int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))))
-            except Exception:
+            if not self._sample():
                 return
             self._stop.wait(0.005)
 
@@ -160,6 +168,7 @@ class ClockSampler:
         if self._thread is not None:
             self._stop.set()
             self._thread.join(timeout=5)
+            self._sample()
             if not self.samples:
                 return None
             reasons = sorted({name for _, bits in self.samples for bit, name in self.REASONS.items() if bits & bit})
