@@ -749,13 +749,15 @@ def other_workload(args, kvq, synth, rank, world):
         dist.destroy_process_group()
 
 
-def secondary_workloads(kvq, synth, warm=3, steps=5):
+def secondary_workloads(kvq, synth, warm=3, steps=5, prefix_steps=20):
     """The other workloads' kernel numbers, measured in the same run as the
     headline (each with its own clock samples), so they sit on the record
     beside it: the chunked prefill with fp16 and with FP4 Q.K (36 layers,
     batch 8, 8192 + 512 tokens) and the qwen3_8b and hadamard prefix
     workloads (bulk append + one decode step).  Each workload is freed before
-    the next one is built."""
+    the next one is built.  The prefix workloads' decode launches are short
+    (qwen3_8b: about 82 us) against the CUDA event clock's 2.048 us steps, so
+    they are averaged over more steps."""
     out = {}
     for key, qk_fp4 in (("prefill_fp16_qk", False), ("prefill_fp4_qk", True)):
         clock = ClockSampler(torch.cuda.current_device())
@@ -768,9 +770,9 @@ def secondary_workloads(kvq, synth, warm=3, steps=5):
                     "dtype": PREFILL_DTYPE_FP4 if qk_fp4 else PREFILL_DTYPE_F16, "clocks": clock.stop()}
     for name in ("qwen3_8b", "hadamard"):
         clock = ClockSampler(torch.cuda.current_device())
-        r = measure_prefix(kvq, synth, name, 36, warm, steps, 1)
+        r = measure_prefix(kvq, synth, name, 36, warm, prefix_steps, 1)
         out[name] = {"workload": PREFIX_WORKLOAD.format(name=name, L=r["L"], B=r["B"], T=r["T"]),
-                     "steps": steps, "warmup": warm,
+                     "steps": prefix_steps, "warmup": warm,
                      "decode": {k: r["decode"][k] for k in ("ms", "achieved", "frac", "unit")},
                      "append": {k: r["append"][k] for k in ("ms", "achieved", "frac", "unit")},
                      "clocks": clock.stop()}
