@@ -756,8 +756,8 @@ def secondary_workloads(kvq, synth, warm=3, steps=5, prefix_steps=20):
     batch 8, 8192 + 512 tokens) and the qwen3_8b and hadamard prefix
     workloads (bulk append + one decode step).  Each workload is freed before
     the next one is built.  The prefix workloads' decode launches are short
-    (qwen3_8b: about 82 us) against the CUDA event clock's 2.048 us steps, so
-    they are averaged over more steps."""
+    (qwen3_8b: about 82 us) against the coarse grid CUDA event times fall on
+    here (about 2 us), so they are averaged over more steps."""
     out = {}
     for key, qk_fp4 in (("prefill_fp16_qk", False), ("prefill_fp4_qk", True)):
         clock = ClockSampler(torch.cuda.current_device())
