@@ -307,10 +307,11 @@ __global__ void klt_finalize_kernel(float* __restrict__ gk, float* __restrict__ 
 }
 
 // ------------------------------------------------------------------ append
-// Keys of the KLT cache: grid (CTAs per (layer, head), Hkv, nlayers), one CTA
-// per SM of two tile groups (128 threads each) that share the basis and walk
-// tiles of 128 tokens of their (layer, head); one group's tile load overlaps
-// the other's transform.  Smoothing y = k * inv_s, the transform y' = U^T y
+// Keys of the KLT cache: one CTA per SM, each taking an equal run of the
+// 128-token tiles of all (layer, head) units in (layer, head)-major order.  A
+// CTA is two tile groups (128 threads each) that share the unit's basis and
+// take every other tile of the run; one group's tile load overlaps the
+// other's transform.  Smoothing y = k * inv_s, the transform y' = U^T y
 // (one fp32 FMA chain per output over c = 0..127), then the NVFP4 quantiser
 // of the append (absmax -> E4M3 scale -> reciprocal -> E2M1, each step one
 // fp32 rounding) and the scatter to the token's slot.
@@ -343,36 +344,26 @@ __device__ __forceinline__ void group_sync(int grp) {
 template <typename T>
 __global__ void __launch_bounds__(kKltThreads, 1)
 klt_append_keys_kernel(const T* __restrict__ k, const int64_t* __restrict__ slots, int num_tokens, int Hkv,
-                       const float* __restrict__ inv_s, const float* __restrict__ U, const float* __restrict__ gk,
-                       uint8_t* __restrict__ cache, int64_t layer_stride, int num_pages, int32_t* __restrict__ status) {
+                       int nlayers, const float* __restrict__ inv_s, const float* __restrict__ U,
+                       const float* __restrict__ gk, uint8_t* __restrict__ cache, int64_t layer_stride, int num_pages,
+                       int32_t* __restrict__ status) {
     extern __shared__ __align__(16) float sm[];
     const int grp = threadIdx.x >> 7, tid = threadIdx.x & 127;
     float* Us = sm;                                            // [c][permuted chunks of i]
     float* Yt = Us + kD * kD + grp * kD * kKltTok;             // this group's [c][token]
     float* rtab = Us + kD * kD + kKltGroups * kD * kKltTok;
     int64_t* sslot = reinterpret_cast<int64_t*>(rtab + 128) + grp * kKltTok;
-    const int h = blockIdx.y, li = blockIdx.z;
-    {
-        const float4* src = reinterpret_cast<const float4*>(U + ((size_t)li * Hkv + h) * kD * kD);
-        for (int e = threadIdx.x; e < kD * kD / 4; e += kKltThreads) {
-            const int c = e >> 5, q = e & 31;                  // row, logical chunk (block q / 4, i = q % 4)
-            reinterpret_cast<float4*>(Us)[c * 32 + klt_chunk(q >> 2, q & 3)] = __ldg(src + e);
-        }
-    }
-    const float g = __ldg(gk + li);
-    const float enc = __frcp_rn(__fmul_rn(6.0f, g));
-    if (threadIdx.x < 128) {
-        // the append's reciprocal of every E4M3 scale code: 1/(val(c) g)
-        const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), g);
-        rtab[threadIdx.x] = (d == 0.0f) ? 0.0f : __frcp_rn(d);
-    }
-    const float* inv = inv_s + ((size_t)li * Hkv + h) * kD;
     const int64_t num_slots = (int64_t)num_pages * kPage;
-    uint8_t* layer_cache = cache + (size_t)li * layer_stride;
     const int lane = threadIdx.x & 31;
     const int tg = 4 * (tid >> 5) + (lane >> 3);               // tokens 8 tg .. + 7
     const int blk = lane & 7;                                  // dims 16 blk .. + 15
     const int ntiles = (num_tokens + kKltTok - 1) / kKltTok;
+    // This CTA's share of the tiles of all (layer, head) units, taken in
+    // (layer, head)-major order: a run that crosses a unit boundary loads the
+    // next unit's basis (and, past a layer, its table) between the two parts,
+    // so every SM gets an equal share whatever the number of units.
+    const long total = (long)nlayers * Hkv * ntiles;
+    const long r0 = total * blockIdx.x / gridDim.x, r1 = total * (blockIdx.x + 1) / gridDim.x;
     // Thread tid loads token tid's key row, 16 runs of 8 elements, and its
     // slot.  The first kAhead runs (bf16: a quarter of the row) and the slot are
     // loaded one tile ahead, into registers, so their global-memory latency
@@ -380,81 +371,111 @@ klt_append_keys_kernel(const T* __restrict__ k, const int64_t* __restrict__ slot
     constexpr int kAhead = sizeof(T) == 2 ? 4 : 0;
     Raw8<T> raw[16];
     int64_t nslot = -1;
-    auto fetch = [&](int tile_i, int e0, int e1) {
-        const int t0 = tile_i * kKltTok;
-        const bool live = tile_i < ntiles && t0 + tid < num_tokens;
-        const T* row = k + (((size_t)li * num_tokens + t0 + tid) * Hkv + h) * kD;
+    int cur_li = -1;
+    float enc = 0.0f;
+    for (long s0 = r0; s0 < r1;) {
+        // segment: tiles [tb, te) of unit u
+        const int u = (int)(s0 / ntiles);
+        const int tb = (int)(s0 - (long)u * ntiles);
+        const int te = (int)(min(r1, (long)(u + 1) * ntiles) - (long)u * ntiles);
+        s0 = (long)u * ntiles + te;
+        const int li = u / Hkv, h = u - li * Hkv;
+        const float* inv = inv_s + ((size_t)li * Hkv + h) * kD;
+        uint8_t* layer_cache = cache + (size_t)li * layer_stride;
+        auto fetch = [&](int tile_i, int e0, int e1) {
+            const int t0 = tile_i * kKltTok;
+            const bool live = tile_i < te && t0 + tid < num_tokens;
+            const T* row = k + (((size_t)li * num_tokens + t0 + tid) * Hkv + h) * kD;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            if (e < e0 || e >= e1) continue;
-            if (live) raw[e].load(row + 8 * e);
-            else raw[e].zero();
-        }
-        if (e0 == 0) nslot = live ? __ldg(slots + t0 + tid) : -1;
-    };
-    // each group walks its own tiles; the basis and the table are shared
-    const int first = blockIdx.x * kKltGroups + grp, stride = gridDim.x * kKltGroups;
-    if (kAhead > 0) fetch(first, 0, kAhead);
-    __syncthreads();         // the basis and the table are in place
-    for (int tile_i = first; tile_i < ntiles; tile_i += stride) {
-        group_sync(grp);     // the previous tile's Yt and slots are consumed
-        fetch(tile_i, kAhead, 16);
-        sslot[tid] = nslot;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            float x[8];
-            raw[e].unpack(x);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) Yt[(8 * e + j) * kKltTok + tid] = __fmul_rn(x[j], __ldg(inv + 8 * e + j));
-        }
-        group_sync(grp);
-        if (kAhead > 0) fetch(tile_i + stride, 0, kAhead);
-        float2 acc[8][8];    // token a, dims 16 blk + 2 p, + 1
-#pragma unroll
-        for (int a = 0; a < 8; ++a)
-#pragma unroll
-            for (int p = 0; p < 8; ++p) acc[a][p] = make_float2(0.0f, 0.0f);
-        const float* yrow = Yt + 8 * tg;
-        const float4* urow = reinterpret_cast<const float4*>(Us);
-#pragma unroll 2
-        for (int c = 0; c < kD; ++c) {
-            const float4 y0 = *reinterpret_cast<const float4*>(yrow + c * kKltTok);
-            const float4 y1 = *reinterpret_cast<const float4*>(yrow + c * kKltTok + 4);
-            float2 u[8];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float4 t = urow[c * 32 + klt_chunk(blk, i)];
-                u[2 * i] = make_float2(t.x, t.y);
-                u[2 * i + 1] = make_float2(t.z, t.w);
+            for (int e = 0; e < 16; ++e) {
+                if (e < e0 || e >= e1) continue;
+                if (live) raw[e].load(row + 8 * e);
+                else raw[e].zero();
             }
-            const float y[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
-            // packed pairs of dims: each half is fma(u, y, acc), rounded once
+            if (e0 == 0) nslot = live ? __ldg(slots + t0 + tid) : -1;
+        };
+        const int first = tb + grp;
+        if (kAhead > 0) fetch(first, 0, kAhead);
+        __syncthreads();     // both groups are done with the previous unit's basis and table
+        {
+            const float4* src = reinterpret_cast<const float4*>(U + ((size_t)li * Hkv + h) * kD * kD);
+            for (int e = threadIdx.x; e < kD * kD / 4; e += kKltThreads) {
+                const int c = e >> 5, q = e & 31;              // row, logical chunk (block q / 4, i = q % 4)
+                reinterpret_cast<float4*>(Us)[c * 32 + klt_chunk(q >> 2, q & 3)] = __ldg(src + e);
+            }
+        }
+        if (li != cur_li) {
+            const float g = __ldg(gk + li);
+            enc = __frcp_rn(__fmul_rn(6.0f, g));
+            if (threadIdx.x < 128) {
+                // the append's reciprocal of every E4M3 scale code: 1/(val(c) g)
+                const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), g);
+                rtab[threadIdx.x] = (d == 0.0f) ? 0.0f : __frcp_rn(d);
+            }
+            cur_li = li;
+        }
+        __syncthreads();     // the basis and the table are in place
+        // each group walks every other tile of the segment
+        for (int tile_i = first; tile_i < te; tile_i += kKltGroups) {
+            group_sync(grp);     // the previous tile's Yt and slots are consumed
+            fetch(tile_i, kAhead, 16);
+            sslot[tid] = nslot;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                float x[8];
+                raw[e].unpack(x);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) Yt[(8 * e + j) * kKltTok + tid] = __fmul_rn(x[j], __ldg(inv + 8 * e + j));
+            }
+            group_sync(grp);
+            if (kAhead > 0) fetch(tile_i + kKltGroups, 0, kAhead);
+            float2 acc[8][8];    // token a, dims 16 blk + 2 p, + 1
+#pragma unroll
+            for (int a = 0; a < 8; ++a)
+#pragma unroll
+                for (int p = 0; p < 8; ++p) acc[a][p] = make_float2(0.0f, 0.0f);
+            const float* yrow = Yt + 8 * tg;
+            const float4* urow = reinterpret_cast<const float4*>(Us);
+#pragma unroll 2
+            for (int c = 0; c < kD; ++c) {
+                const float4 y0 = *reinterpret_cast<const float4*>(yrow + c * kKltTok);
+                const float4 y1 = *reinterpret_cast<const float4*>(yrow + c * kKltTok + 4);
+                float2 u[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 t = urow[c * 32 + klt_chunk(blk, i)];
+                    u[2 * i] = make_float2(t.x, t.y);
+                    u[2 * i + 1] = make_float2(t.z, t.w);
+                }
+                const float y[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+                // packed pairs of dims: each half is fma(u, y, acc), rounded once
+#pragma unroll
+                for (int a = 0; a < 8; ++a) {
+                    const float2 yy = make_float2(y[a], y[a]);
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) acc[a][p] = ffma2(u[p], yy, acc[a][p]);
+                }
+            }
 #pragma unroll
             for (int a = 0; a < 8; ++a) {
-                const float2 yy = make_float2(y[a], y[a]);
+                const int64_t slot = sslot[8 * tg + a];
+                float2 v[8];
 #pragma unroll
-                for (int p = 0; p < 8; ++p) acc[a][p] = ffma2(u[p], yy, acc[a][p]);
-            }
-        }
+                for (int p = 0; p < 8; ++p) v[p] = acc[a][p];
+                const uint32_t sf = e4m3_rn(__fmul_rn(absmax16(v), enc));
+                const float r = rtab[sf & 0x7Fu];
 #pragma unroll
-        for (int a = 0; a < 8; ++a) {
-            const int64_t slot = sslot[8 * tg + a];
-            float2 v[8];
-#pragma unroll
-            for (int p = 0; p < 8; ++p) v[p] = acc[a][p];
-            const uint32_t sf = e4m3_rn(__fmul_rn(absmax16(v), enc));
-            const float r = rtab[sf & 0x7Fu];
-#pragma unroll
-            for (int p = 0; p < 8; ++p) v[p] = make_float2(__fmul_rn(v[p].x, r), __fmul_rn(v[p].y, r));
-            const uint2 w = make_uint2(e2m1x8_rn(v[0], v[1], v[2], v[3]), e2m1x8_rn(v[4], v[5], v[6], v[7]));
-            if (slot >= num_slots) {
-                if (blk == 0) set_status(status, KVQ_DEV_BAD_SLOT);
-            } else if (slot >= 0) {
-                uint8_t* tile = layer_cache + ((size_t)(slot >> 4) * Hkv + h) * kTile;
-                const int off = (int)(slot & 15);
-                // dims 16 blk .. + 15: code bytes 8 blk .. + 7, scale byte blk
-                *reinterpret_cast<uint2*>(tile + kKCodes + off * 64 + 8 * blk) = w;
-                tile[kKScales + off * 8 + blk] = (uint8_t)sf;
+                for (int p = 0; p < 8; ++p) v[p] = make_float2(__fmul_rn(v[p].x, r), __fmul_rn(v[p].y, r));
+                const uint2 w = make_uint2(e2m1x8_rn(v[0], v[1], v[2], v[3]), e2m1x8_rn(v[4], v[5], v[6], v[7]));
+                if (slot >= num_slots) {
+                    if (blk == 0) set_status(status, KVQ_DEV_BAD_SLOT);
+                } else if (slot >= 0) {
+                    uint8_t* tile = layer_cache + ((size_t)(slot >> 4) * Hkv + h) * kTile;
+                    const int off = (int)(slot & 15);
+                    // dims 16 blk .. + 15: code bytes 8 blk .. + 7, scale byte blk
+                    *reinterpret_cast<uint2*>(tile + kKCodes + off * 64 + 8 * blk) = w;
+                    tile[kKScales + off * 8 + blk] = (uint8_t)sf;
+                }
             }
         }
     }
@@ -468,29 +489,28 @@ kvq_status append_klt_keys(const kvq_shape& s, const kvq_calib& c, const kvq_cac
     const float* U = c.k_klt + (size_t)layer0 * H * kD * kD;
     const float* gk = c.k_gscale + layer0;
     uint8_t* base = cache.data + (size_t)layer0 * cache.layer_stride_bytes;
-    // one CTA per SM at most (no partial second wave); each CTA's tile groups
-    // walk tiles of its (layer, head)
+    // one CTA per SM (no partial second wave), each with an equal share of
+    // all units' tiles
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const long ntiles = (num_tokens + kKltTok - 1) / kKltTok;
-    const long walkers = (ntiles + kKltGroups - 1) / kKltGroups;
-    long per = (long)sms / ((long)H * nlayers);
-    if (per < 1) per = 1;
-    const dim3 grid((unsigned)(walkers < per ? walkers : per), H, nlayers);
+    const long total = (long)(num_tokens + kKltTok - 1) / kKltTok * H * nlayers;
+    if (total == 0) return KVQ_OK;
+    const long pairs = (total + kKltGroups - 1) / kKltGroups;
+    const dim3 grid((unsigned)(pairs < sms ? pairs : sms));
     cudaError_t e;
     if (dtype == KVQ_F32) {
         e = cudaFuncSetAttribute(klt_append_keys_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kKltAppendSmem);
         if (e != cudaSuccess) return KVQ_ECUDA;
-        klt_append_keys_kernel<float><<<grid, kKltThreads, kKltAppendSmem, st>>>((const float*)k, slots, num_tokens, H, inv,
-                                                                       U, gk, base, cache.layer_stride_bytes,
-                                                                       cache.num_pages, status);
+        klt_append_keys_kernel<float><<<grid, kKltThreads, kKltAppendSmem, st>>>(
+            (const float*)k, slots, num_tokens, H, nlayers, inv, U, gk, base, cache.layer_stride_bytes, cache.num_pages,
+            status);
     } else {
         e = cudaFuncSetAttribute(klt_append_keys_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kKltAppendSmem);
         if (e != cudaSuccess) return KVQ_ECUDA;
         klt_append_keys_kernel<__nv_bfloat16><<<grid, kKltThreads, kKltAppendSmem, st>>>(
-            (const __nv_bfloat16*)k, slots, num_tokens, H, inv, U, gk, base, cache.layer_stride_bytes,
+            (const __nv_bfloat16*)k, slots, num_tokens, H, nlayers, inv, U, gk, base, cache.layer_stride_bytes,
             cache.num_pages, status);
     }
     return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ECUDA;
