@@ -324,7 +324,9 @@ __global__ void klt_finalize_kernel(float* __restrict__ gk, float* __restrict__ 
 // permuted, so the 8 blocks' i-th chunks sit in 8 distinct bank groups: 6
 // shared-memory wavefronts per warp and step for 128 FMAs.  The FMAs run in
 // packed pairs of dims (fma.rn.f32x2, each half rounded as fmaf), 64
-// instructions per step; the chains and their order are unchanged.
+// instructions per step, ordered by dim pair and then token so that
+// consecutive ones share their basis operand; the chains and their order
+// are unchanged.
 constexpr int kKltTok = 128;  // tokens per append tile
 constexpr int kKltGroups = 2; // tile groups per CTA
 constexpr int kKltThreads = 128 * kKltGroups;
@@ -449,12 +451,13 @@ klt_append_keys_kernel(const T* __restrict__ k, const int64_t* __restrict__ slot
                 }
                 const float y[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
                 // packed pairs of dims: each half is fma(u, y, acc), rounded once
+                float2 yy[8];
 #pragma unroll
-                for (int a = 0; a < 8; ++a) {
-                    const float2 yy = make_float2(y[a], y[a]);
+                for (int a = 0; a < 8; ++a) yy[a] = make_float2(y[a], y[a]);
 #pragma unroll
-                    for (int p = 0; p < 8; ++p) acc[a][p] = ffma2(u[p], yy, acc[a][p]);
-                }
+                for (int p = 0; p < 8; ++p)
+#pragma unroll
+                    for (int a = 0; a < 8; ++a) acc[a][p] = ffma2(u[p], yy[a], acc[a][p]);
             }
 #pragma unroll
             for (int a = 0; a < 8; ++a) {
