@@ -438,7 +438,7 @@ klt_append_keys_kernel(const T* __restrict__ k, const int64_t* __restrict__ slot
                 for (int p = 0; p < 8; ++p) acc[a][p] = make_float2(0.0f, 0.0f);
             const float* yrow = Yt + 8 * tg;
             const float4* urow = reinterpret_cast<const float4*>(Us);
-#pragma unroll 2
+#pragma unroll 4
             for (int c = 0; c < kD; ++c) {
                 const float4 y0 = *reinterpret_cast<const float4*>(yrow + c * kKltTok);
                 const float4 y1 = *reinterpret_cast<const float4*>(yrow + c * kKltTok + 4);
